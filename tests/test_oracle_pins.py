@@ -1,0 +1,290 @@
+"""Pins of the CPU oracle against facts fixed outside of it (no GPU needed).
+
+Each test checks one oracle function against the pages, the number format's
+definition, a closed form, an invariant or an independent library routine, so
+that a dropped term, a wrong sign or index or a transposed operand in the
+oracle fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+from bf16_causal_prefill_fp8_b200 import synth
+from oracle import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --- e4m3 codec ----------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_for_all_256_codes():
+    ours = orc.e4m3_values()
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    nan_ours, nan_ref = np.isnan(ours), np.isnan(ref)
+    assert np.array_equal(nan_ours, nan_ref)
+    assert np.flatnonzero(nan_ours).tolist() == [0x7F, 0xFF]
+    assert np.array_equal(ours[~nan_ours], ref[~nan_ref])
+    assert ours[0x7E] == 448.0 and ours[0x08] == 2.0 ** -6 and ours[0x01] == 2.0 ** -9
+
+
+def test_e4m3_power_of_two_ladder_golden():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "e4m3_pow2_ladder.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert len(rows) == 15
+    for k, val, code in rows:
+        k, val, code = int(k), float(val), int(code)
+        assert val == 2.0 ** k
+        assert code == 8 * k + 56
+        assert orc.e4m3_value(code) == val
+        assert int(orc.e4m3_from_f32(val)[0]) == code
+
+
+def test_e4m3_encode_matches_torch_rne_in_range():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(4000) * 40,
+        rng.standard_normal(2000) * 0.01,                       # subnormal range
+        rng.uniform(-448, 448, 2000),
+        np.array([0.0, -0.0, 448.0, -448.0, 2.0 ** -10, 3 * 2.0 ** -11, 1.0625, 1.1875]),
+    ]).astype(np.float32)
+    ours = orc.e4m3_from_f32(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_ties_go_to_even_and_saturate():
+    vals = orc.e4m3_values()
+    # midpoints between consecutive positive finite codes: tie -> the even code
+    for c in range(0, 0x7E):
+        mid = np.float32((vals[c] + vals[c + 1]) / 2)
+        if float(mid) != (vals[c] + vals[c + 1]) / 2:
+            continue
+        want = c if c % 2 == 0 else c + 1
+        assert int(orc.e4m3_from_f32(mid)[0]) == want, c
+    assert int(orc.e4m3_from_f32(1e9)[0]) == 0x7E
+    assert int(orc.e4m3_from_f32(-500.0)[0]) == 0xFE
+    assert int(orc.e4m3_from_f32(449.0)[0]) == 0x7E
+    # round trip of every finite code
+    for c in list(range(0, 0x7F)) + list(range(0x80, 0xFF)):
+        assert int(orc.e4m3_from_f32(np.float32(vals[c]))[0]) == c
+
+
+# --- Hadamard -----------------------------------------------------------------
+
+def test_fwht_equals_scipy_sylvester_hadamard():
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128.0)
+    rows = orc.fwht128(np.eye(128, dtype=np.float32))
+    assert np.allclose(rows, H, atol=1e-7, rtol=0)
+    # orthonormal: H H^T = I
+    Hf = rows.astype(np.float64)
+    assert np.allclose(Hf @ Hf.T, np.eye(128), atol=1e-6)
+    # applied to data it equals x @ H (H symmetric)
+    x = synth.gaussian(3, 1, (7, 128))
+    assert np.allclose(orc.fwht128(x), x.astype(np.float64) @ H, atol=1e-5)
+
+
+def test_rotation_leaves_qk_invariant_fp64():
+    q = synth.gaussian(4, 1, (16, 128)).astype(np.float64)
+    k = synth.gaussian(4, 2, (16, 128)).astype(np.float64)
+    H = orc.fwht128(np.eye(128, dtype=np.float32)).astype(np.float64)
+    H = H / np.sqrt(np.sum(H * H, axis=1, keepdims=True))  # exact orthonormal rows
+    assert np.allclose((q @ H) @ (k @ H).T, q @ k.T, atol=1e-9)
+
+
+# --- quantizer ------------------------------------------------------------------
+
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_quantize_scale_and_codes_properties(hadamard):
+    x = synth.gaussian(5, 1, (2, 200, 3, 128))
+    x[1, :, 2, :] = 0.0                                   # a zero head: scale 1, codes 0
+    codes, scale = orc.quantize(x, hadamard=hadamard)
+    vals = orc.e4m3_values()[codes]
+    xr = orc.fwht128(x) if hadamard else x.astype(np.float32)
+    for b in range(2):
+        for h in range(3):
+            blk = xr[b, :, h, :]
+            amax = np.float32(np.max(np.abs(blk)))
+            if amax == 0:
+                assert scale[b, h] == 1.0 and np.all(codes[b, :, h, :] % 128 == 0)
+                continue
+            # the largest element lands exactly on the largest finite code
+            assert np.float32(amax / np.float32(scale[b, h])) == np.float32(448.0) or \
+                abs(amax / scale[b, h] - 448.0) < 1e-3
+            assert np.max(np.abs(vals[b, :, h, :])) == 448.0
+            # every code is the nearest e4m3 value to x/scale (brute force over codes)
+            y = (blk / np.float32(scale[b, h])).astype(np.float32).astype(np.float64)
+            fin = orc.e4m3_values()[:0x7F]
+            d = np.abs(np.abs(y)[..., None] - fin[None, None, :])
+            best = d.min(axis=-1)
+            got = np.abs(vals[b, :, h, :] - np.abs(y) * 0) - 0  # decoded magnitudes
+            assert np.all(np.abs(np.abs(got) - np.abs(y)) <= best + 1e-12)
+            assert np.all(np.sign(vals[b, :, h, :]) * np.sign(y) >= 0)
+
+
+def test_hadamard_quantize_round_trip_within_e4m3_bound():
+    # rotating the dequantized codes back recovers x within e4m3's relative
+    # precision (3 mantissa bits: half an ulp is 2^-4 of the value); the
+    # pages' "roughly halves the input error" is reported, not asserted
+    x = synth.gaussian(6, 2, (1, 256, 2, 128))
+    std, _ = synth.outlier_channel_std(6, 2, 128)
+    x = (x * std[None, None]).astype(np.float32)
+    c1, s1 = orc.quantize(x, hadamard=True)
+    back = orc.fwht128(orc.dequantize(c1, s1).astype(np.float32)).astype(np.float64)
+    assert orc.rel_fro(back, x) < 2.0 ** -4
+    c0, s0 = orc.quantize(x, hadamard=False)
+    assert orc.rel_fro(orc.dequantize(c0, s0), x) < 2.0 ** -4
+
+
+# --- attention (fp64 definition) ------------------------------------------------
+
+def _sdpa_ref(q, k, v):
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    g = Hq // Hkv
+    qt = torch.from_numpy(np.asarray(q, np.float64)).permute(0, 2, 1, 3)
+    kt = torch.from_numpy(np.asarray(k, np.float64)).permute(0, 2, 1, 3).repeat_interleave(g, 1)
+    vt = torch.from_numpy(np.asarray(v, np.float64)).permute(0, 2, 1, 3).repeat_interleave(g, 1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1, 8, 8), (2, 7, 4, 2, 16, 8), (1, 33, 6, 3, 24, 16),
+                                   (1, 130, 2, 2, 128, 128), (1, 64, 2, 1, 192, 128)])
+def test_attention_matches_torch_sdpa(shape):
+    B, S, Hq, Hkv, Dqk, Dv = shape
+    q = synth.gaussian(7, 1, (B, S, Hq, Dqk)).astype(np.float64)
+    k = synth.gaussian(7, 2, (B, S, Hkv, Dqk)).astype(np.float64)
+    v = synth.gaussian(7, 3, (B, S, Hkv, Dv)).astype(np.float64)
+    o = orc.attention(q, k, v)
+    ref = _sdpa_ref(q, k, v)
+    assert np.allclose(o, ref, atol=1e-12, rtol=1e-10)
+    rows = [0, S - 1, S // 2]
+    o2 = orc.attention(q, k, v, rows=rows)
+    assert np.array_equal(o2, o[:, rows])
+
+
+def test_attention_row0_is_v0_and_zero_q_gives_prefix_means():
+    q = synth.gaussian(8, 1, (1, 50, 2, 16)).astype(np.float64)
+    k = synth.gaussian(8, 2, (1, 50, 2, 16)).astype(np.float64)
+    v = synth.gaussian(8, 3, (1, 50, 2, 16)).astype(np.float64)
+    o = orc.attention(q, k, v)
+    assert np.array_equal(o[:, 0], v[:, 0])
+    o0 = orc.attention(np.zeros_like(q), k, v)
+    pref = np.cumsum(v, axis=1) / np.arange(1, 51)[None, :, None, None]
+    assert np.allclose(o0, pref, atol=1e-13)
+
+
+def test_gqa_single_kv_head_equals_replicated_mha():
+    q = synth.gaussian(9, 1, (1, 40, 4, 16)).astype(np.float64)
+    k = synth.gaussian(9, 2, (1, 40, 1, 16)).astype(np.float64)
+    v = synth.gaussian(9, 3, (1, 40, 1, 8)).astype(np.float64)
+    a = orc.attention(q, k, v)
+    b = orc.attention(q, np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2))
+    assert np.allclose(a, b, atol=1e-14)
+
+
+# --- Lean P ----------------------------------------------------------------------
+
+def test_leanp_zero_scores_give_8j_plus_56():
+    for A in [1e-4, 0.37, 5.0]:
+        for j in [8, 9, 20, 126]:
+            assert orc.leanp_code(0.0, 0.0, A, j) == min(126, 8 * j + 56) or j > 8
+        assert orc.leanp_block_shift(0.0, 0.0, A) == 8
+        assert orc.leanp_code(0.0, 0.0, A, 8) == 120
+    assert orc.leanp_code(5.0, 5.0, 0.25, 8, masked=True) == 0
+    assert orc.leanp_code(-np.inf, 5.0, 0.25, 8) == 0
+    assert orc.leanp_block_shift(1.0, -np.inf, 0.5) == 8
+
+
+def test_leanp_slope_formula_constant():
+    A = orc.leanp_slope(1.0, 1.0, 128)
+    assert A == np.float32(8.0 * math.log2(math.e) / math.sqrt(128.0))
+    assert orc.leanp_slope(0.5, 0.25, 192) == np.float32(
+        np.float32(0.125) * np.float32(8.0 * math.log2(math.e) / math.sqrt(192.0)))
+
+
+def test_leanp_monotone_in_score():
+    m, A = np.float32(3.0), np.float32(0.731)
+    s = np.linspace(-200, 3.0, 20001).astype(np.float32)
+    bmax = np.full_like(s, m)
+    codes, js = orc.leanp_batch(s, np.full_like(s, m), bmax, np.full_like(s, A))
+    assert np.all(np.diff(codes.astype(int)) >= 0)
+    assert np.all(js == 8)
+
+
+def test_leanp_weight_inside_mitchell_band():
+    # decoded weight value(code) * 2^-j against exact 2^((s-m)A/8):
+    # ratio in (2^-1/8, 1.0615] for normal codes (Mitchell's linear
+    # approximation of log2 plus truncation of the code)
+    rng = np.random.default_rng(11)
+    n = 20000
+    m = rng.uniform(-30, 30, n).astype(np.float32)
+    A = np.exp(rng.uniform(np.log(1e-3), np.log(20), n)).astype(np.float32)
+    gap = rng.uniform(0, 100, n).astype(np.float32)           # m - bmax, in units of A/8
+    bmax = (m - gap * np.float32(8.0) / A).astype(np.float32)
+    bmax = np.minimum(bmax, m)
+    frac = rng.uniform(0, 1, n)
+    s = (bmax - frac * np.float32(40.0) / A).astype(np.float32)   # up to 5 binades under bmax
+    s = np.minimum(s, bmax)
+    codes, js = orc.leanp_batch(s, m, bmax, A)
+    vals = orc.e4m3_values()[codes]
+    exact = np.exp2((s.astype(np.float64) - m.astype(np.float64)) * A.astype(np.float64) / 8.0)
+    w = vals * np.exp2(-js.astype(np.float64))
+    normal = (codes >= 8) & (codes <= 126)
+    assert normal.mean() > 0.9
+    ratio = w[normal] / exact[normal]
+    assert ratio.min() > 2.0 ** (-1.0 / 8.0) - 1e-4
+    assert ratio.max() <= 1.0615 + 1e-4
+    # the block max lands in the top binade: u in (112, 120], so its code is
+    # in [112, 120] (one lower where the fp32 steps round across an integer)
+    cmax, _ = orc.leanp_batch(bmax, m, bmax, A)
+    cap = js < 126
+    assert np.all((cmax[cap] >= 111) & (cmax[cap] <= 120))
+    assert np.mean(cmax[cap] >= 112) > 0.99
+
+
+def test_leanp_block_shift_cap():
+    assert orc.leanp_block_shift(1e6, -1e6, 1.0) == 126
+    assert orc.leanp_block_shift(10.0, 2.0, 1.0) == 9        # gap 8*1 -> floor(1) = 1
+    assert orc.leanp_block_shift(10.0, 2.0001, 1.0) == 8
+
+
+# --- model oracle ----------------------------------------------------------------
+
+def _quantized_case(seed, B, S, Hq, Hkv, D, Dv=None):
+    Dv = Dv or D
+    q, k, v = synth.make_qkv(seed, B, S, Hq, Hkv, D, Dv)
+    qc, qs = orc.quantize(q); kc, ks = orc.quantize(k); vc, vs = orc.quantize(v)
+    return (qc, kc, vc, qs, ks, vs), (orc.dequantize(qc, qs), orc.dequantize(kc, ks),
+                                      orc.dequantize(vc, vs)), (q, k, v)
+
+
+def test_model_oracle_exact_p_equals_plain_definition():
+    codes, deq, _ = _quantized_case(12, 1, 300, 4, 2, 128)
+    qc, kc, vc, qs, ks, vs = codes
+    o_model = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True)
+    o_ref = orc.attention(*deq)
+    assert orc.rel_fro(o_model, o_ref) < 1e-6
+
+
+def test_model_oracle_zero_q_gives_prefix_means():
+    codes, deq, _ = _quantized_case(13, 1, 200, 2, 2, 128)
+    qc, kc, vc, qs, ks, vs = codes
+    qz = np.zeros_like(qc)
+    o = orc.fp8_model(qz, kc, vc, qs, ks, vs)
+    pref = np.cumsum(deq[2], axis=1) / np.arange(1, 201)[None, :, None, None]
+    assert np.allclose(o, pref, atol=1e-12)
+    assert np.array_equal(o[:, 0], deq[2][:, 0])
+
+
+def test_model_oracle_leanp_error_against_fp64_is_within_fp8_bar():
+    codes, deq, _ = _quantized_case(14, 1, 512, 2, 2, 128)
+    qc, kc, vc, qs, ks, vs = codes
+    o = orc.fp8_model(qc, kc, vc, qs, ks, vs)
+    ref = orc.attention(*deq)
+    err = orc.rel_fro(o, ref)
+    assert 1e-3 < err < 3e-2
