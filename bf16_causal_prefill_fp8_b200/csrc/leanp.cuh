@@ -1,0 +1,60 @@
+// leanp.cuh -- Lean P: an FP8 (e4m3) softmax probability written directly as
+// its code, one multiply-add plus one integer conversion per element, with a
+// power-of-two scale per 64-key block.
+//
+// Method (Zyphra ZYFA, as reported by the-ai.news "Zyphra presenteert ZYFA",
+// section "Drie technieken om de bottleneck te omzeilen", and spke.com
+// "Zyphra ZYFA", sections "Lean P" and "ブロックごとのスケーリングと丸められた
+// 行和"): the e4m3 bit pattern read as an integer grows by 8 per doubling, so
+// the code of 2^x is about 8x + 56; each 64-key block of P is multiplied by a
+// power of two before rounding and the block-scaled matrix instruction removes
+// that factor again.
+//
+// Exact fp32 steps (every step rounds to nearest-even in fp32; the FMAs are
+// fused):
+//   A    = (q_s * k_s) * C,  C = fp32(8 log2(e) / sqrt(Dqk))     per head pair
+//   j    = 8 if the block has no live key, else
+//          min(126, 8 + floor(((m - bmax) * A) * 0.125))         per row, block
+//   B    = fma(-m, A, 56 + 8 j)                                   per row, block
+//   u    = fma(s, A, B)                                           per element
+//   code = trunc(max(u, 0))           (the low byte of fp32(max(u,0) + 1.5*2^23)
+//                                       added with round-toward-zero)
+// s is the raw fp32 score (sum of products of e4m3 values), m the running row
+// maximum after this key tile and bmax the maximum of the element's 64-key
+// block.  Precondition: s <= bmax <= m, or s = -inf for a masked key; then
+// u <= 120 and the code never exceeds 126 (127 would be NaN).  The weight the
+// matrix unit applies is value(code) * 2^-j: E8M0 scale code 127 - j.
+#pragma once
+#include <cstdint>
+
+namespace zyfa {
+
+__device__ __forceinline__ float leanp_slope(float q_s, float k_s, float C) {
+  return __fmul_rn(__fmul_rn(q_s, k_s), C);
+}
+
+__device__ __forceinline__ int leanp_block_shift(float m, float bmax, float A) {
+  if (bmax == __int_as_float(0xff800000)) return 8;   // -inf: no live key in the block
+  const float f = floorf(__fmul_rn(__fmul_rn(__fsub_rn(m, bmax), A), 0.125f));
+  return f >= 118.0f ? 126 : 8 + static_cast<int>(f);
+}
+
+__device__ __forceinline__ float leanp_row_offset(float m, float A, int j) {
+  return __fmaf_rn(-m, A, static_cast<float>(56 + 8 * j));
+}
+
+// Returns a 32-bit word whose low byte is the e4m3 code of score s.
+__device__ __forceinline__ uint32_t leanp_code_word(float s, float A, float B) {
+  const float u = fmaxf(__fmaf_rn(s, A, B), 0.0f);
+  return __float_as_uint(__fadd_rz(u, 12582912.0f));
+}
+
+// Four code words -> one 32-bit word holding the four code bytes in order.
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t w0, uint32_t w1, uint32_t w2,
+                                                    uint32_t w3) {
+  const uint32_t lo = __byte_perm(w0, w1, 0x0040);
+  const uint32_t hi = __byte_perm(w2, w3, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+}  // namespace zyfa

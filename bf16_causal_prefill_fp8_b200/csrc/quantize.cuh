@@ -1,0 +1,166 @@
+// quantize.cuh -- the FP8 prepass: per-(batch, head) amax, scale = amax/448,
+// e4m3 codes, with an optional 128-point Hadamard rotation of each row.
+//
+// Method: kongchang.com "Zyphra ZYFA", section "ZYFA 的性能与精度数据" (per-head
+// scale factors map values into the e4m3 range) and spke.com "Zyphra ZYFA",
+// accuracy section (quantizing Q, K and V is the main FP8 error source; a
+// Hadamard rotation of Q and K roughly halves it).  HBM-bound: each kernel
+// streams the tensor once with 16-byte vector loads; a CTA covers whole
+// sequence rows of one batch.
+//
+// Steps (all on `stream`):
+//   1. memset(scale, 0)                         scale doubles as amax accumulator
+//   2. quant_amax_kernel:  scale[b,h] = max(scale[b,h], max |x'|)   (fp32 bits,
+//      atomicMax on the non-negative bit patterns, order-independent)
+//   3. quant_codes_kernel: s = amax/448 (1 if amax == 0); code = e4m3(x'/s)
+//   4. quant_finalize_kernel: scale[b,h] = s
+// x' is the row rotated by the orthonormal Sylvester transform when
+// hadamard != 0 (stages of stride 1, 2, ..., 64 in fp32, then one multiply by
+// fp32(2^-3.5)), else x itself.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace zyfa {
+
+constexpr int kQuantThreads = 256;
+constexpr float kFwhtNorm = 0.08838834764831844055f;   // 2^-3.5 rounded to fp32
+
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+__device__ __forceinline__ float head_scale(float amax) {
+  return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+}
+
+// Load 4 consecutive elements as fp32.
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float (&v)[4]);
+template <>
+__device__ __forceinline__ void load4<float>(const float* p, float (&v)[4]) {
+  const float4 t = *reinterpret_cast<const float4*>(p);
+  v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 t = *reinterpret_cast<const uint2*>(p);
+  v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xffff0000u);
+  v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xffff0000u);
+}
+
+// In-warp 128-point transform: lane l holds elements 4l .. 4l+3.
+__device__ __forceinline__ void fwht128_warp(float (&x)[4], int lane) {
+  float a, b;
+  // stride 1
+  a = x[0]; b = x[1]; x[0] = a + b; x[1] = a - b;
+  a = x[2]; b = x[3]; x[2] = a + b; x[3] = a - b;
+  // stride 2
+  a = x[0]; b = x[2]; x[0] = a + b; x[2] = a - b;
+  a = x[1]; b = x[3]; x[1] = a + b; x[3] = a - b;
+  // strides 4 .. 64: partner lane differs in one bit
+#pragma unroll
+  for (int sh = 1; sh < 32; sh <<= 1) {
+    const bool upper = (lane & sh) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[i], sh);
+      x[i] = upper ? (o - x[i]) : (x[i] + o);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = x[i] * kFwhtNorm;
+}
+
+struct QuantArgs {
+  const void* x;
+  uint8_t* out;
+  float* scale;            // [B*H]: amax accumulator, then the scales
+  int S, H, D;
+  int rows_per_cta;        // sequence rows of one batch per CTA
+};
+
+// Step 2.  grid = (ceil(S / rows_per_cta), B), block = kQuantThreads.
+template <typename T, bool HAD>
+__global__ void __launch_bounds__(kQuantThreads) quant_amax_kernel(QuantArgs a) {
+  extern __shared__ unsigned int s_amax[];   // [H]
+  const int b = blockIdx.y;
+  const int r0 = blockIdx.x * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
+  for (int h = threadIdx.x; h < a.H; h += blockDim.x) s_amax[h] = 0u;
+  __syncthreads();
+  const size_t HD = static_cast<size_t>(a.H) * a.D;
+  const T* base = static_cast<const T*>(a.x) + (static_cast<size_t>(b) * a.S + r0) * HD;
+  if (HAD) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nvec = (r1 - r0) * a.H;          // 128-element rows
+    for (int vi = warp; vi < nvec; vi += nw) {
+      float x[4];
+      load4<T>(base + static_cast<size_t>(vi) * 128 + 4 * lane, x);
+      fwht128_warp(x, lane);
+      float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) atomicMax(&s_amax[vi % a.H], __float_as_uint(mx));
+    }
+  } else {
+    const size_t n4 = (static_cast<size_t>(r1 - r0) * HD) / 4;
+    for (size_t i = threadIdx.x; i < n4; i += blockDim.x) {
+      float x[4];
+      load4<T>(base + 4 * i, x);
+      const float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+      const int h = static_cast<int>(((4 * i) % HD) / a.D);
+      atomicMax(&s_amax[h], __float_as_uint(mx));
+    }
+  }
+  __syncthreads();
+  for (int h = threadIdx.x; h < a.H; h += blockDim.x)
+    atomicMax(reinterpret_cast<unsigned int*>(a.scale) + static_cast<size_t>(b) * a.H + h, s_amax[h]);
+}
+
+// Step 3.  Same grid; reads the finished amax of each (b, h).
+template <typename T, bool HAD>
+__global__ void __launch_bounds__(kQuantThreads) quant_codes_kernel(QuantArgs a) {
+  extern __shared__ float s_sc[];   // [H]
+  const int b = blockIdx.y;
+  const int r0 = blockIdx.x * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
+  for (int h = threadIdx.x; h < a.H; h += blockDim.x)
+    s_sc[h] = head_scale(a.scale[static_cast<size_t>(b) * a.H + h]);
+  __syncthreads();
+  const size_t HD = static_cast<size_t>(a.H) * a.D;
+  const size_t off = (static_cast<size_t>(b) * a.S + r0) * HD;
+  const T* base = static_cast<const T*>(a.x) + off;
+  uint8_t* obase = a.out + off;
+  if (HAD) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nvec = (r1 - r0) * a.H;
+    for (int vi = warp; vi < nvec; vi += nw) {
+      float x[4];
+      load4<T>(base + static_cast<size_t>(vi) * 128 + 4 * lane, x);
+      fwht128_warp(x, lane);
+      const float sc = s_sc[vi % a.H];
+      const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[0], sc), __fdiv_rn(x[1], sc));
+      const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[2], sc), __fdiv_rn(x[3], sc));
+      *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(vi) * 128 + 4 * lane) = lo | (hi << 16);
+    }
+  } else {
+    const size_t n4 = (static_cast<size_t>(r1 - r0) * HD) / 4;
+    for (size_t i = threadIdx.x; i < n4; i += blockDim.x) {
+      float x[4];
+      load4<T>(base + 4 * i, x);
+      const float sc = s_sc[((4 * i) % HD) / a.D];
+      const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[0], sc), __fdiv_rn(x[1], sc));
+      const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[2], sc), __fdiv_rn(x[3], sc));
+      *reinterpret_cast<uint32_t*>(obase + 4 * i) = lo | (hi << 16);
+    }
+  }
+}
+
+// Step 4.
+__global__ void quant_finalize_kernel(float* scale, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) scale[i] = head_scale(scale[i]);
+}
+
+}  // namespace zyfa

@@ -1,0 +1,284 @@
+// zyfa.cu -- the C ABI of libzyfa.so (declared in include/zyfa.h): argument
+// validation, TMA descriptor encoding, instance selection and launches.  All
+// device code of the library is in this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/zyfa.h"
+#include "attn_fwd.cuh"
+#include "leanp.cuh"
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+namespace zyfa {
+
+// ---------------------------------------------------------------- helpers
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+
+std::atomic<unsigned long long> g_timeout_ns{0};
+
+unsigned long long wait_timeout_ns() {
+  unsigned long long t = g_timeout_ns.load(std::memory_order_relaxed);
+  if (t != 0) return t;
+  t = kDefaultTimeoutNs;
+  if (const char* e = std::getenv("ZYFA_WAIT_TIMEOUT_MS")) {
+    const double ms = std::atof(e);
+    if (ms > 0) t = static_cast<unsigned long long>(ms * 1e6);
+  }
+  g_timeout_ns.store(t, std::memory_order_relaxed);
+  return t;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool attr_set[4] = {false, false, false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// 4-D map over a BSHD tensor: dims (D, H, S, B) innermost first; a box is
+// `box_d` elements of one head for 128 consecutive sequence rows.  Rows past S
+// read as zero.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int el, int B, int S, int H,
+              int D, int box_d, CUtensorMapSwizzle swz) {
+  const EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * el, (cuuint64_t)H * D * el, (cuuint64_t)S * H * D * el};
+  cuuint32_t box[4] = {(cuuint32_t)box_d, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool FP8, int DQK>
+int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int S,
+                const float* qs, const float* ks, const float* vs, cudaStream_t stream, int dev,
+                int inst) {
+  using Cf = AttnCfg<FP8, DQK>;
+  AttnArgs a;
+  const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int el = FP8 ? 1 : 2;
+  const int box = 128 / el;   // 128 bytes of one row
+  bool ok = make_map(&a.map_q, q, dt, el, B, S, Hq, DQK, box, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_map(&a.map_k, k, dt, el, B, S, Hkv, DQK, box, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_map(&a.map_v, v, dt, el, B, S, Hkv, 128, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (Cf::TAIL) {
+    ok = ok && make_map(&a.map_q_tail, q, dt, el, B, S, Hq, DQK, 64, CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_map(&a.map_k_tail, k, dt, el, B, S, Hkv, DQK, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+  } else {
+    a.map_q_tail = a.map_q;
+    a.map_k_tail = a.map_k;
+  }
+  if (!ok) return ZYFA_ERR_CUDA;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.q_scale = qs;
+  a.k_scale = ks;
+  a.v_scale = vs;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.S = S;
+  a.Tq = (S + 127) / 128;
+  const double kv_slot_bytes = static_cast<double>(S) * (DQK + 128) * el;
+  long long gk = static_cast<long long>((48.0 * 1024 * 1024) / kv_slot_bytes);
+  const long long slots = static_cast<long long>(B) * Hkv;
+  if (gk < 1) gk = 1;
+  if (gk > slots) gk = slots;
+  a.group_slots = static_cast<int>(gk);
+  a.C = FP8 ? static_cast<float>(8.0 * 1.4426950408889634074 / std::sqrt(static_cast<double>(DQK)))
+            : static_cast<float>(1.4426950408889634074 / std::sqrt(static_cast<double>(DQK)));
+  a.timeout_ns = wait_timeout_ns();
+
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (di.sms == 0 && cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ZYFA_ERR_CUDA;
+    if (!di.attr_set[inst]) {
+      if (cudaFuncSetAttribute(attn_fwd_kernel<FP8, DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cf::SMEM) != cudaSuccess)
+        return ZYFA_ERR_CUDA;
+      di.attr_set[inst] = true;
+    }
+  }
+  const long long units = static_cast<long long>(B) * Hq * a.Tq;
+  const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
+  attn_fwd_kernel<FP8, DQK><<<grid, 192, Cf::SMEM, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- test kernels
+
+__global__ void leanp_codes_kernel(const float* s, const float* m, const float* bmax, const float* A,
+                                   const unsigned char* masked, int n, unsigned char* code, int* jout) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const float Ai = A[i], mi = m[i];
+    const int j = leanp_block_shift(mi, bmax[i], Ai);
+    const float B = leanp_row_offset(mi, Ai, j);
+    const float si = (masked && masked[i]) ? __int_as_float(0xff800000) : s[i];
+    code[i] = static_cast<unsigned char>(leanp_code_word(si, Ai, B) & 0xffu);
+    if (jout) jout[i] = j;
+  }
+}
+
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    const WaitCtl ctl{&abort_flag, timeout_ns};
+    (void)mbar_wait(smem_u32(&bar), 0, ctl);   // nothing arrives: runs out, records the status
+  }
+}
+
+}  // namespace zyfa
+
+using namespace zyfa;
+
+// ---------------------------------------------------------------- C ABI
+
+extern "C" const char* zyfa_status_string(int status) {
+  switch (status) {
+    case ZYFA_OK: return "ok";
+    case ZYFA_ERR_NULL_PTR: return "a required pointer is NULL";
+    case ZYFA_ERR_BAD_SHAPE: return "bad shape (B, S and head counts must be >= 1 and fit the index range)";
+    case ZYFA_ERR_UNSUPPORTED_HEADDIM: return "unsupported head dimension";
+    case ZYFA_ERR_BAD_GQA: return "Hq must be a multiple of Hkv";
+    case ZYFA_ERR_MISALIGNED: return "misaligned pointer (tensors need 16-byte, scales 4-byte alignment)";
+    case ZYFA_ERR_BAD_DTYPE: return "unsupported dtype or flag";
+    case ZYFA_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case ZYFA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    default: return "unknown status";
+  }
+}
+
+extern "C" void zyfa_set_wait_timeout_ns(unsigned long long ns) {
+  g_timeout_ns.store(ns, std::memory_order_relaxed);
+}
+
+extern "C" int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq,
+                             int Hkv, int S, int Dqk, int Dv, int dtype, const float* q_scale,
+                             const float* k_scale, const float* v_scale, void* stream) {
+  if (!q || !k || !v || !o) return ZYFA_ERR_NULL_PTR;
+  if (B < 1 || S < 1 || Hq < 1 || Hkv < 1) return ZYFA_ERR_BAD_SHAPE;
+  if (Hq % Hkv != 0) return ZYFA_ERR_BAD_GQA;
+  if (!((Dqk == 128 || Dqk == 192) && Dv == 128)) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (dtype != ZYFA_BF16 && dtype != ZYFA_FP8_E4M3) return ZYFA_ERR_BAD_DTYPE;
+  // TMA coordinates are 32-bit; the flat element count must fit comfortably
+  const long long tq = (static_cast<long long>(S) + 127) / 128;
+  if (static_cast<long long>(B) * Hq * tq > (1ll << 31) - 1) return ZYFA_ERR_BAD_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return ZYFA_ERR_MISALIGNED;
+  if (dtype == ZYFA_FP8_E4M3 &&
+      (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4)))
+    return ZYFA_ERR_MISALIGNED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == ZYFA_FP8_E4M3) {
+    if (Dqk == 128) return launch_attn<true, 128>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 0);
+    return launch_attn<true, 192>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 1);
+  }
+  if (Dqk == 128) return launch_attn<false, 128>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 2);
+  return launch_attn<false, 192>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 3);
+}
+
+extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* scale, int B, int S, int H,
+                             int D, int hadamard, void* stream) {
+  if (!x || !x_fp8 || !scale) return ZYFA_ERR_NULL_PTR;
+  if (B < 1 || S < 1 || H < 1 || B > 65535 || H > 4096) return ZYFA_ERR_BAD_SHAPE;
+  if (in_dtype != ZYFA_BF16 && in_dtype != ZYFA_FP32) return ZYFA_ERR_BAD_DTYPE;
+  if (hadamard != 0 && hadamard != 1) return ZYFA_ERR_BAD_DTYPE;
+  if (D < 8 || D > 1024 || D % 8 != 0 || (hadamard && D != 128)) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (!aligned(x, 16) || !aligned(x_fp8, 16) || !aligned(scale, 4)) return ZYFA_ERR_MISALIGNED;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ZYFA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ZYFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long want = 4ll * sms;
+  long long chunks = (want + B - 1) / B;
+  if (chunks > S) chunks = S;
+  if (chunks < 1) chunks = 1;
+  QuantArgs a;
+  a.x = x;
+  a.out = static_cast<uint8_t*>(x_fp8);
+  a.scale = scale;
+  a.S = S; a.H = H; a.D = D;
+  a.rows_per_cta = static_cast<int>((S + chunks - 1) / chunks);
+  const dim3 grid(static_cast<unsigned>((S + a.rows_per_cta - 1) / a.rows_per_cta), static_cast<unsigned>(B));
+  const size_t shm = static_cast<size_t>(H) * 4;
+  if (cudaMemsetAsync(scale, 0, static_cast<size_t>(B) * H * sizeof(float), st) != cudaSuccess)
+    return ZYFA_ERR_CUDA;
+  if (in_dtype == ZYFA_BF16) {
+    if (hadamard) {
+      quant_amax_kernel<__nv_bfloat16, true><<<grid, kQuantThreads, shm, st>>>(a);
+      quant_codes_kernel<__nv_bfloat16, true><<<grid, kQuantThreads, shm, st>>>(a);
+    } else {
+      quant_amax_kernel<__nv_bfloat16, false><<<grid, kQuantThreads, shm, st>>>(a);
+      quant_codes_kernel<__nv_bfloat16, false><<<grid, kQuantThreads, shm, st>>>(a);
+    }
+  } else {
+    if (hadamard) {
+      quant_amax_kernel<float, true><<<grid, kQuantThreads, shm, st>>>(a);
+      quant_codes_kernel<float, true><<<grid, kQuantThreads, shm, st>>>(a);
+    } else {
+      quant_amax_kernel<float, false><<<grid, kQuantThreads, shm, st>>>(a);
+      quant_codes_kernel<float, false><<<grid, kQuantThreads, shm, st>>>(a);
+    }
+  }
+  const int n = B * H;
+  quant_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(scale, n);
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+extern "C" int zyfa_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZYFA_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return ZYFA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return ZYFA_ERR_CUDA;
+  return v == kDevOk ? ZYFA_OK : ZYFA_ERR_DEVICE_TIMEOUT;
+}
+
+extern "C" int zyfa_leanp_codes(const float* s, const float* m, const float* bmax, const float* A,
+                                const unsigned char* masked, int n, unsigned char* code, int* j,
+                                void* stream) {
+  if (n < 0) return ZYFA_ERR_BAD_SHAPE;
+  if (n == 0) return ZYFA_OK;
+  if (!s || !m || !bmax || !A || !code) return ZYFA_ERR_NULL_PTR;
+  const int blocks = (n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024;
+  leanp_codes_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(s, m, bmax, A, masked, n, code, j);
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+extern "C" int zyfa_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns > 1000000000ull) return ZYFA_ERR_BAD_SHAPE;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}

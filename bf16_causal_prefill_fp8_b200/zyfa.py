@@ -1,0 +1,159 @@
+"""Thin ctypes binding of libzyfa.so (include/zyfa.h) for torch CUDA tensors.
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream.  If the
+library has not been built, importing the functions raises instead of falling
+back to anything else.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libzyfa.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "zyfa.h")
+
+BF16, FP8_E4M3, FP32 = 0, 1, 2
+OK, ERR_DEVICE_TIMEOUT = 0, -8
+
+
+class ZyfaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m bf16_causal_prefill_fp8_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.zyfa_attn_fwd.restype = i
+        L.zyfa_attn_fwd.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, p, p, p]
+        L.zyfa_quantize.restype = i
+        L.zyfa_quantize.argtypes = [p, i, p, p, i, i, i, i, i, p]
+        L.zyfa_status_string.restype = ctypes.c_char_p
+        L.zyfa_status_string.argtypes = [i]
+        L.zyfa_device_status.restype = i
+        L.zyfa_device_status.argtypes = [p]
+        L.zyfa_set_wait_timeout_ns.restype = None
+        L.zyfa_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+        L.zyfa_leanp_codes.restype = i
+        L.zyfa_leanp_codes.argtypes = [p, p, p, p, p, i, p, p, p]
+        L.zyfa_selftest_wait_timeout.restype = i
+        L.zyfa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, p]
+        _lib = L
+    return _lib
+
+
+def declared_symbols():
+    """Names of the entry points include/zyfa.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|void|char\s*\*|const char\s*\*)\s*\**\s*(zyfa_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def status_string(status: int) -> str:
+    return lib().zyfa_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise ZyfaError(status, what)
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t, name):
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=None):
+    """Causal attention forward.  q [B,S,Hq,Dqk], k [B,S,Hkv,Dqk], v [B,S,Hkv,Dv];
+    bf16 tensors (BF16 path) or uint8 / float8_e4m3fn codes with fp32 scales
+    [B,H] (FP8 path).  Returns o [B,S,Hq,Dv] bf16."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if q.dtype == torch.bfloat16:
+        dt = BF16
+    elif q.dtype in (torch.uint8, torch.float8_e4m3fn):
+        dt = FP8_E4M3
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    B, S, Hq, Dqk = q.shape
+    Hkv, Dv = k.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty((B, S, Hq, Dv), dtype=torch.bfloat16, device=q.device)
+    _dev(o, "o")
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        if t is not None:
+            _dev(t, n)
+            if t.dtype != torch.float32:
+                raise ValueError(f"{n} must be fp32")
+    st = lib().zyfa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, S, Dqk, Dv, dt,
+                             _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream(stream))
+    _check(st, "zyfa_attn_fwd")
+    return o
+
+
+def quantize(x, hadamard=False, out=None, scale=None, stream=None):
+    """x [B,S,H,D] bf16 or fp32 -> (codes uint8 [B,S,H,D], scale fp32 [B,H])."""
+    _dev(x, "x")
+    if x.dtype == torch.bfloat16:
+        dt = BF16
+    elif x.dtype == torch.float32:
+        dt = FP32
+    else:
+        raise ValueError(f"unsupported input dtype {x.dtype}")
+    B, S, H, D = x.shape
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    _dev(out, "out"); _dev(scale, "scale")
+    st = lib().zyfa_quantize(_ptr(x), dt, _ptr(out), _ptr(scale), B, S, H, D, int(bool(hadamard)),
+                             _stream(stream))
+    _check(st, "zyfa_quantize")
+    return out, scale
+
+
+def leanp_codes(s, m, bmax, A, masked=None, stream=None):
+    """Element-wise Lean-P codes from the kernel's device functions."""
+    n = s.numel()
+    for t, nm in ((s, "s"), (m, "m"), (bmax, "bmax"), (A, "A")):
+        _dev(t, nm)
+    code = torch.empty(n, dtype=torch.uint8, device=s.device)
+    j = torch.empty(n, dtype=torch.int32, device=s.device)
+    st = lib().zyfa_leanp_codes(_ptr(s), _ptr(m), _ptr(bmax), _ptr(A), _ptr(masked), n, _ptr(code),
+                                _ptr(j), _stream(stream))
+    _check(st, "zyfa_leanp_codes")
+    return code, j
+
+
+def device_status(stream=None) -> int:
+    return lib().zyfa_device_status(_stream(stream))
+
+
+def set_wait_timeout_ns(ns: int):
+    lib().zyfa_set_wait_timeout_ns(int(ns))
+
+
+def selftest_wait_timeout(ns: int, stream=None):
+    _check(lib().zyfa_selftest_wait_timeout(int(ns), _stream(stream)), "zyfa_selftest_wait_timeout")

@@ -1,0 +1,176 @@
+/*
+ * zyfa.h -- C ABI of libzyfa.so: causal prefill attention forward for NVIDIA
+ * B200 (sm_100a) with FP8 e4m3 or BF16 Q/K/V, following Zyphra's ZYFA method
+ * (Lean-P FP8 probabilities, a power-of-two scale per 64-key block, the row sum
+ * taken from the rounded probabilities), plus its quantize + Hadamard prepass.
+ *
+ * Sources (news pages about ZYFA):
+ *   the-ai.news, "Zyphra presenteert ZYFA: FlashAttention FP8 voor AMD MI355X"
+ *   ai-daily-news.org, "Zyphra ZYFA: FP8 FlashAttention para AMD MI355X"
+ *   kongchang.com, "Zyphra ZYFA: AMD MI355X 上的 FP8 FlashAttention 提速 1.76 倍"
+ *   spke.com, "Zyphra ZYFA: AMD MI355X向けFP8 FlashAttention、最大1.76倍高速化"
+ *
+ * Conventions for every entry point:
+ *  - Pointers named q, k, v, o, x, x_fp8, scale, *_scale and the Lean-P test
+ *    arrays are DEVICE pointers (CUDA global memory of the current device).
+ *    The caller allocates and owns every buffer; the library allocates no
+ *    memory and keeps no state between calls other than one device error
+ *    word (see zyfa_device_status) and per-device launch attributes.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *    enqueued asynchronously on it; no other stream is used.
+ *  - Return value: ZYFA_OK (0) once the work is enqueued, or a negative
+ *    zyfa_status.  On any argument error nothing is launched.  Faults inside
+ *    a kernel surface at the caller's next synchronisation; bounded waits that
+ *    run out inside the attention kernel are reported by zyfa_device_status.
+ *  - Layouts are BSHD, contiguous, innermost dimension last (the
+ *    flash_attn_func convention that the pages' drop-in Python interface
+ *    uses: spke.com "Zyphra ZYFA", TL;DR).
+ *  - All calls are reentrant; results are deterministic (fixed ascending
+ *    key-tile order, no atomics on data; the pages report bitwise identical
+ *    output across 7,200 runs: spke.com "Zyphra ZYFA", accuracy section).
+ */
+#ifndef ZYFA_H_
+#define ZYFA_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types. */
+enum zyfa_dtype {
+  ZYFA_BF16 = 0,      /* bfloat16 */
+  ZYFA_FP8_E4M3 = 1,  /* OCP e4m3 "fn": bias 7, max 448, 0x7F/0xFF NaN */
+  ZYFA_FP32 = 2       /* IEEE binary32 (prepass input only) */
+};
+
+/* Status codes (negative = error). */
+enum zyfa_status {
+  ZYFA_OK = 0,
+  ZYFA_ERR_NULL_PTR = -1,            /* a required pointer is NULL */
+  ZYFA_ERR_BAD_SHAPE = -2,           /* B, S, H < 1, or sizes overflow the TMA index range */
+  ZYFA_ERR_UNSUPPORTED_HEADDIM = -3, /* (Dqk, Dv) not (128,128) or (192,128); prepass D */
+  ZYFA_ERR_BAD_GQA = -4,             /* Hq is not a multiple of Hkv */
+  ZYFA_ERR_MISALIGNED = -5,          /* a tensor base is not 16-byte aligned (scales: 4) */
+  ZYFA_ERR_BAD_DTYPE = -6,           /* dtype / in_dtype / flag value not supported */
+  ZYFA_ERR_CUDA = -7,                /* a CUDA runtime/driver call or launch failed */
+  ZYFA_ERR_DEVICE_TIMEOUT = -8       /* a bounded device wait ran out (zyfa_device_status) */
+};
+
+/*
+ * zyfa_attn_fwd -- causal prefill attention forward (prefill only, Sq = Sk):
+ *
+ *     O = softmax(Q K^T / sqrt(Dqk) + causal mask) V
+ *
+ * The computation the pages describe (ai-daily-news.org "Zyphra ZYFA",
+ * "Qué cubren los kernels": causal forward attention in FP8 and BF16, head
+ * dimension 128 and DeepSeek-V2's latent-attention shape; spke.com TL;DR:
+ * MLA shape 192/128).
+ *
+ *   q  [B, S, Hq,  Dqk]   dtype elements
+ *   k  [B, S, Hkv, Dqk]   dtype elements
+ *   v  [B, S, Hkv, Dv ]   dtype elements
+ *   o  [B, S, Hq,  Dv ]   bfloat16 output (written for every row < S)
+ *   Query head h reads kv head h / (Hq / Hkv) (grouped-query attention).
+ *   (Dqk, Dv) in {(128, 128), (192, 128)}; S >= 1; B, Hq, Hkv >= 1.
+ *   Softmax scale is fixed at 1/sqrt(Dqk).
+ *
+ * dtype = ZYFA_BF16: exact softmax probabilities (exp2, fp32), P rounded to
+ *   bf16 for the P V product; the row sum is accumulated in fp32 from the
+ *   unrounded probabilities.  Scale pointers are ignored.
+ * dtype = ZYFA_FP8_E4M3: q/k/v hold e4m3 codes; the real values are
+ *   code * scale with one fp32 scale per (batch, head):
+ *     q_scale [B*Hq], k_scale [B*Hkv], v_scale [B*Hkv]  (device; NULL = 1.0),
+ *   indexed b*H + h.  P is written Lean-P style (the-ai.news "Zyphra presenteert
+ *   ZYFA", "Drie technieken om de bottleneck te omzeilen"; spke.com "Lean P"):
+ *   one multiply-add and one integer conversion per probability, code of 2^x
+ *   ~ 8x + 56, truncated, with a power-of-two 2^j per (row, 64-key block)
+ *   applied before rounding and removed by the block-scaled tensor-core MMA
+ *   (spke.com "ブロックごとのスケーリングと丸められた行和").  The softmax
+ *   denominator is the sum of the rounded, rescaled probabilities, taken by an
+ *   extra MMA against a ones matrix.  Accumulation is fp32 throughout.
+ *
+ * Alignment: q, k, v, o 16-byte aligned; scales 4-byte aligned.
+ * Errors: NULL_PTR (q, k, v or o NULL), BAD_SHAPE, BAD_GQA,
+ *   UNSUPPORTED_HEADDIM, BAD_DTYPE, MISALIGNED, CUDA.
+ */
+int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv,
+                  int S, int Dqk, int Dv, int dtype, const float* q_scale, const float* k_scale,
+                  const float* v_scale, void* stream);
+
+/*
+ * zyfa_quantize -- the prepass: per-(batch, head) FP8 e4m3 quantization, with
+ * an optional Hadamard rotation for Q and K (spke.com "Zyphra ZYFA", accuracy
+ * section: most FP8 error comes from quantizing Q, K and V, and a Hadamard
+ * rotation of Q and K roughly halves it; kongchang.com "ZYFA 的性能与精度数据":
+ * per-tensor or per-head scale factors map values into the e4m3 range).
+ *
+ *   x      [B, S, H, D]  in_dtype = ZYFA_BF16 or ZYFA_FP32
+ *   x_fp8  [B, S, H, D]  e4m3 codes (output)
+ *   scale  [B*H]         fp32 (output), indexed b*H + h
+ *   hadamard = 1: each D = 128 row is first rotated by the orthonormal
+ *     128-point Sylvester Walsh-Hadamard transform (butterflies of stride
+ *     1, 2, ..., 64 in fp32, then one multiply by fp32(2^-3.5)).  Apply it to
+ *     Q and K only (the rotation cancels in Q K^T); never to V.
+ *   For each (b, h): amax = max |x'| over (s, d); scale = amax / 448 (fp32,
+ *   IEEE division; 1.0 when amax == 0); code = e4m3 round-to-nearest-even,
+ *   saturating at +-448, of fp32(x' / scale) (IEEE division).
+ * D must be a multiple of 8 and at most 1024 (128 with hadamard).
+ * Alignment: x and x_fp8 16-byte aligned; scale 4-byte aligned.  The scale
+ * buffer is used as the amax accumulator while the prepass runs (four
+ * stream-ordered steps); it holds the final scales once the stream reaches
+ * the end of the call.
+ */
+int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* scale, int B, int S, int H,
+                  int D, int hadamard, void* stream);
+
+/* Human-readable text of a status code (static storage; never NULL). */
+const char* zyfa_status_string(int status);
+
+/*
+ * zyfa_device_status -- synchronises `stream`, then reads and clears the
+ * device error word of the current device.  Returns ZYFA_OK, or
+ * ZYFA_ERR_DEVICE_TIMEOUT if a bounded wait inside a kernel ran out since the
+ * last call (that kernel's output is then invalid), or ZYFA_ERR_CUDA.
+ */
+int zyfa_device_status(void* stream);
+
+/*
+ * zyfa_set_wait_timeout_ns -- time limit of every mbarrier wait inside the
+ * attention kernel, in nanoseconds (default 2e9; also read once from the
+ * environment variable ZYFA_WAIT_TIMEOUT_MS).  A wait that runs out records
+ * ZYFA_ERR_DEVICE_TIMEOUT and the kernel returns without writing the
+ * remaining output.  0 restores the default.  Process-wide.
+ */
+void zyfa_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * zyfa_leanp_codes -- runs, element-wise, the very __device__ functions the
+ * FP8 attention kernel uses to turn scores into Lean-P codes, so that the
+ * codes can be compared byte for byte with a CPU emulation.  For element i:
+ *   j[i]    = 8 if bmax[i] == -inf, else
+ *             min(126, 8 + floor(fp32(fp32(m[i] - bmax[i]) * A[i]) * 0.125))
+ *   B       = fma(-m[i], A[i], 56 + 8 j[i])
+ *   code[i] = masked[i] ? 0 : trunc(max(fma(s[i], A[i], B), 0))   (e4m3 code)
+ * (the-ai.news "Zyphra presenteert ZYFA", "Drie technieken ..."; spke.com
+ * "Lean P").  Precondition, as inside the kernel: s <= bmax <= m or s = -inf.
+ *   s, m, bmax, A: fp32 [n]; masked: uint8 [n] or NULL; code: uint8 [n];
+ *   j: int32 [n] or NULL.  n >= 0.  Errors: NULL_PTR, BAD_SHAPE, CUDA.
+ */
+int zyfa_leanp_codes(const float* s, const float* m, const float* bmax, const float* A,
+                     const unsigned char* masked, int n, unsigned char* code, int* j, void* stream);
+
+/*
+ * zyfa_selftest_wait_timeout -- launches a one-CTA kernel whose only thread
+ * waits on an mbarrier that nothing ever arrives on, with the given time
+ * limit (ns, at most 1e9), through the same bounded-wait routine the attention
+ * kernel uses.  The wait runs out, the kernel records ZYFA_ERR_DEVICE_TIMEOUT
+ * in the device error word and returns; no fault, trap or hang.  Used to test
+ * the failure path: call it, then zyfa_device_status() must report the timeout.
+ */
+int zyfa_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZYFA_H_ */

@@ -1,0 +1,73 @@
+"""Shared helpers of the GPU parity tests: seeded inputs, the CUDA path through
+the C-ABI binding, and the oracle's references for the same inputs."""
+import numpy as np
+import torch
+
+from bf16_causal_prefill_fp8_b200 import synth, zyfa
+from oracle import oracle as orc
+
+# Tolerances (relative Frobenius error of the bf16 output against the fp64
+# oracle on the values the GPU received): the acceptance bars of the method.
+TOL_BF16 = 5e-3
+TOL_FP8 = 3e-2
+# GPU against the CPU replay of the FP8 pipeline (same codes, same tile order):
+# separates kernel bugs from the method's own error.  Budget: bf16 output
+# rounding (2^-9/sqrt(3) ~ 1.1e-3) plus one-step Lean-P code flips (a weight
+# off by 2^(1/8)) wherever the tensor core's fp32 sum of a score differs from
+# the oracle's fp64 sum near an integer boundary of u; with heavy-tailed
+# outlier channels the scores are large and flips are more frequent (measured
+# 4.0e-3 on the outlier-K case).  A layout or scale bug in the kernel moves
+# the error to >= 1e-1, far above this budget.
+TOL_FP8_MODEL = 8e-3
+
+
+def bf16_round(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16)
+
+
+def inputs(seed, B, S, Hq, Hkv, Dqk, Dv, kind="gaussian", q_gain=1.0):
+    q, k, v = synth.make_qkv(seed, B, S, Hq, Hkv, Dqk, Dv, kind)
+    if q_gain != 1.0:
+        q = (q * np.float32(q_gain)).astype(np.float32)
+    return q, k, v
+
+
+def run_bf16(q, k, v):
+    qb, kb, vb = bf16_round(q), bf16_round(k), bf16_round(v)
+    o = zyfa.attn_fwd(qb.cuda(), kb.cuda(), vb.cuda())
+    torch.cuda.synchronize()
+    return o.float().cpu().numpy().astype(np.float64), (qb.double().numpy(), kb.double().numpy(),
+                                                       vb.double().numpy())
+
+
+def quantize_gpu(x: np.ndarray, hadamard=False, as_bf16=False):
+    t = bf16_round(x) if as_bf16 else torch.from_numpy(np.ascontiguousarray(x))
+    codes, scale = zyfa.quantize(t.cuda(), hadamard=hadamard)
+    torch.cuda.synchronize()
+    return codes, scale
+
+
+def run_fp8(q, k, v, hadamard=False, check_prepass=True):
+    """Quantize on the GPU, run FP8 attention, and return the output plus the
+    oracle's own quantization (asserted bit-identical to the GPU's)."""
+    qc, qs = quantize_gpu(q, hadamard)
+    kc, ks = quantize_gpu(k, hadamard)
+    vc, vs = quantize_gpu(v, False)
+    o = zyfa.attn_fwd(qc, kc, vc, q_scale=qs, k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    oq = orc.quantize(q, hadamard=hadamard)
+    ok = orc.quantize(k, hadamard=hadamard)
+    ov = orc.quantize(v, hadamard=False)
+    if check_prepass:
+        for (gc, gs), (rc, rs) in zip(((qc, qs), (kc, ks), (vc, vs)), (oq, ok, ov)):
+            assert np.array_equal(gc.cpu().numpy(), rc)
+            assert np.array_equal(gs.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    return o.float().cpu().numpy().astype(np.float64), (oq, ok, ov)
+
+
+def fp8_references(codes, rows=None):
+    (qc, qs), (kc, ks), (vc, vs) = codes
+    deq = (orc.dequantize(qc, qs), orc.dequantize(kc, ks), orc.dequantize(vc, vs))
+    ref = orc.attention(*deq, rows=rows)
+    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rows=rows)
+    return ref, model

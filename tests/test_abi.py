@@ -1,0 +1,77 @@
+"""The C-ABI library loads, exports every symbol include/zyfa.h declares, and
+rejects bad arguments on the host before touching the GPU (runs without a GPU)."""
+import ctypes
+
+import pytest
+
+from bf16_causal_prefill_fp8_b200 import build, zyfa
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return zyfa.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = zyfa.declared_symbols()
+    assert set(names) >= {"zyfa_attn_fwd", "zyfa_quantize", "zyfa_status_string", "zyfa_device_status",
+                          "zyfa_leanp_codes", "zyfa_selftest_wait_timeout", "zyfa_set_wait_timeout_ns"}
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for st in [0, -1, -2, -3, -4, -5, -6, -7, -8, 12345]:
+        s = zyfa.status_string(st)
+        assert isinstance(s, str) and s
+    assert zyfa.status_string(0) == "ok"
+    assert zyfa.status_string(12345) == "unknown status"
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced (validation fails first)
+
+
+def _attn(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, Hq=2, Hkv=2, S=128, Dqk=128, Dv=128, dt=0,
+          qs=None, ks=None, vs=None):
+    return L.zyfa_attn_fwd(q, k, v, o, B, Hq, Hkv, S, Dqk, Dv, dt, qs, ks, vs, None)
+
+
+def test_attn_argument_errors(L):
+    assert _attn(L, q=None) == -1
+    assert _attn(L, o=None) == -1
+    assert _attn(L, B=0) == -2
+    assert _attn(L, S=0) == -2
+    assert _attn(L, Hq=0) == -2
+    assert _attn(L, Hq=3, Hkv=2) == -4
+    assert _attn(L, Dqk=64) == -3
+    assert _attn(L, Dqk=128, Dv=64) == -3
+    assert _attn(L, Dqk=192, Dv=192) == -3
+    assert _attn(L, dt=2) == -6
+    assert _attn(L, dt=-1) == -6
+    assert _attn(L, q=FAKE + 8) == -5
+    assert _attn(L, o=FAKE + 2) == -5
+    assert _attn(L, dt=1, qs=FAKE + 1) == -5
+    assert _attn(L, B=1 << 20, Hq=1 << 12, Hkv=1, S=1 << 16) == -2
+
+
+def test_quantize_argument_errors(L):
+    def q(x=FAKE, dt=0, out=FAKE, sc=FAKE, B=1, S=16, H=2, D=128, had=0):
+        return L.zyfa_quantize(x, dt, out, sc, B, S, H, D, had, None)
+    assert q(x=None) == -1
+    assert q(sc=None) == -1
+    assert q(B=0) == -2
+    assert q(H=5000) == -2
+    assert q(dt=1) == -6
+    assert q(had=2) == -6
+    assert q(D=12) == -3
+    assert q(D=192, had=1) == -3
+    assert q(x=FAKE + 4) == -5
+    assert q(sc=FAKE + 2) == -5
+
+
+def test_leanp_and_selftest_argument_errors(L):
+    assert L.zyfa_leanp_codes(None, None, None, None, None, -1, None, None, None) == -2
+    assert L.zyfa_leanp_codes(None, None, None, None, None, 0, None, None, None) == 0
+    assert L.zyfa_leanp_codes(None, FAKE, FAKE, FAKE, None, 4, FAKE, None, None) == -1
+    assert L.zyfa_selftest_wait_timeout(ctypes.c_ulonglong(2_000_000_000), None) == -2

@@ -1,0 +1,117 @@
+"""Causal attention through zyfa_attn_fwd against the fp64 oracle.
+
+BF16: relative Frobenius error <= 5e-3 against fp64 attention on the bf16
+inputs.  FP8: <= 3e-2 against fp64 attention on the dequantized e4m3 inputs,
+and close to the CPU replay of the FP8 pipeline (same codes, same order).
+Sizes span several 128-row tiles and ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+from bf16_causal_prefill_fp8_b200 import zyfa
+from oracle import oracle as orc
+
+from helpers import (TOL_BF16, TOL_FP8, TOL_FP8_MODEL, fp8_references, inputs, run_bf16,
+                     run_fp8)
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [  # B, S, Hq, Hkv, Dqk, Dv
+    (1, 1, 1, 1, 128, 128),
+    (1, 64, 2, 2, 128, 128),
+    (1, 127, 2, 2, 128, 128),
+    (1, 128, 2, 2, 128, 128),
+    (1, 129, 2, 2, 128, 128),
+    (1, 512, 2, 2, 128, 128),        # the pages' tiny configuration
+    (2, 300, 4, 2, 128, 128),        # GQA, batch 2
+    (1, 1000, 6, 1, 128, 128),       # GQA, one kv head
+    (1, 300, 2, 2, 192, 128),        # MLA shape
+    (2, 200, 4, 4, 192, 128),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_parity(shape):
+    B, S, Hq, Hkv, Dqk, Dv = shape
+    q, k, v = inputs(41, B, S, Hq, Hkv, Dqk, Dv, kind="mla" if Dqk == 192 else "gaussian")
+    o, (qd, kd, vd) = run_bf16(q, k, v)
+    ref = orc.attention(qd, kd, vd)
+    err = orc.rel_fro(o, ref)
+    print(f"bf16 {shape}: vs fp64 {err:.3e}")
+    assert err <= TOL_BF16, err
+    assert np.array_equal(o[:, 0], np.asarray(torch.from_numpy(vd[:, 0]).repeat_interleave(Hq // Hkv, 1)
+                                              .to(torch.bfloat16).double()))
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_fp8_parity(shape):
+    B, S, Hq, Hkv, Dqk, Dv = shape
+    q, k, v = inputs(42, B, S, Hq, Hkv, Dqk, Dv, kind="mla" if Dqk == 192 else "gaussian")
+    o, codes = run_fp8(q, k, v)
+    ref, model = fp8_references(codes)
+    err = orc.rel_fro(o, ref)
+    err_model = orc.rel_fro(o, model)
+    print(f"fp8 {shape}: vs fp64 {err:.3e}  vs model {err_model:.3e}")
+    assert err <= TOL_FP8, err
+    assert err_model <= TOL_FP8_MODEL, err_model
+
+
+@pytest.mark.parametrize("q_gain,kind", [(6.0, "gaussian"), (1.0, "outlier_k"), (12.0, "gaussian")])
+def test_fp8_block_scales_engaged(q_gain, kind):
+    # peaked scores: many 64-key blocks sit far below the row max, so the
+    # per-block power-of-two shift j varies (exercises the scale factors)
+    q, k, v = inputs(43, 1, 700, 4, 2, 128, 128, kind=kind, q_gain=q_gain)
+    o, codes = run_fp8(q, k, v)
+    ref, model = fp8_references(codes)
+    e_model, e_ref = orc.rel_fro(o, model), orc.rel_fro(o, ref)
+    print(f"fp8 gain={q_gain} {kind}: vs fp64 {e_ref:.3e}  vs model {e_model:.3e}")
+    assert e_model <= TOL_FP8_MODEL
+    assert e_ref <= TOL_FP8
+
+
+def test_fp8_hadamard_prepass_path():
+    q, k, v = inputs(44, 1, 513, 4, 4, 128, 128)
+    o, codes = run_fp8(q, k, v, hadamard=True)
+    ref, model = fp8_references(codes)
+    assert orc.rel_fro(o, ref) <= TOL_FP8
+    assert orc.rel_fro(o, model) <= TOL_FP8_MODEL
+    # rotation cancels in Q K^T: compare with unquantized fp64 attention too (reported bar)
+    unq = orc.attention(q, k, v)
+    assert orc.rel_fro(o, unq) < 0.1
+
+
+def test_zero_q_gives_prefix_means_fp8_and_bf16():
+    q, k, v = inputs(45, 1, 260, 2, 2, 128, 128)
+    q[:] = 0.0
+    o8, codes = run_fp8(q, k, v)
+    vd = orc.dequantize(*codes[2])
+    pref = np.cumsum(vd, axis=1) / np.arange(1, 261)[None, :, None, None]
+    assert orc.rel_fro(o8, pref) <= 2e-3            # equal weights: only bf16 output rounding
+    ob, (_, _, vb) = run_bf16(q, k, v)
+    prefb = np.cumsum(vb, axis=1) / np.arange(1, 261)[None, :, None, None]
+    assert orc.rel_fro(ob, prefb) <= 2e-3
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_deterministic_repeated_runs_and_streams(dtype):
+    q, k, v = inputs(46, 1, 1100, 8, 2, 128, 128)
+    if dtype == "bf16":
+        args = [torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (q, k, v)]
+        kw = {}
+    else:
+        from bf16_causal_prefill_fp8_b200 import zyfa as z
+        qc, qs = z.quantize(torch.from_numpy(q).cuda())
+        kc, ks = z.quantize(torch.from_numpy(k).cuda())
+        vc, vs = z.quantize(torch.from_numpy(v).cuda())
+        args, kw = [qc, kc, vc], dict(q_scale=qs, k_scale=ks, v_scale=vs)
+    first = zyfa.attn_fwd(*args, **kw).clone()
+    s2 = torch.cuda.Stream()
+    for i in range(20):
+        if i % 2:
+            with torch.cuda.stream(s2):
+                o = zyfa.attn_fwd(*args, **kw)
+            s2.synchronize()
+        else:
+            o = zyfa.attn_fwd(*args, **kw)
+        assert torch.equal(o, first)
+    assert zyfa.device_status() == zyfa.OK

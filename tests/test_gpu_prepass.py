@@ -1,0 +1,39 @@
+"""Prepass (zyfa_quantize) against the oracle's quantizer: codes and scales
+must match byte for byte, with and without the Hadamard rotation."""
+import numpy as np
+import pytest
+
+from bf16_causal_prefill_fp8_b200 import synth
+from oracle import oracle as orc
+
+from helpers import bf16_round, quantize_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("shape,hadamard", [((1, 200, 3, 128), False), ((1, 200, 3, 128), True),
+                                            ((2, 77, 4, 192), False), ((3, 1, 5, 128), True),
+                                            ((1, 1000, 8, 128), True), ((2, 129, 2, 64), False)])
+@pytest.mark.parametrize("as_bf16", [False, True])
+def test_quantize_bit_exact(shape, hadamard, as_bf16):
+    x = synth.gaussian(21, 1, shape) * np.float32(3.0)
+    x[0, :, 0, :] *= np.float32(50.0)                     # heads with different ranges
+    if shape[2] > 2:
+        x[-1, :, 2, :] = 0.0                              # an all-zero head: scale 1
+    codes, scale = quantize_gpu(x, hadamard=hadamard, as_bf16=as_bf16)
+    xin = bf16_round(x).float().numpy() if as_bf16 else x
+    rc, rs = orc.quantize(xin, hadamard=hadamard)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    got = codes.cpu().numpy()
+    assert np.array_equal(got, rc), f"{np.count_nonzero(got != rc)} codes differ"
+
+
+def test_quantize_outlier_channels_and_subnormals():
+    x = synth.gaussian(22, 2, (1, 333, 4, 128))
+    std, _ = synth.outlier_channel_std(22, 4, 128)
+    x = (x * std[None, None]).astype(np.float32)
+    for had in (False, True):
+        codes, scale = quantize_gpu(x, hadamard=had)
+        rc, rs = orc.quantize(x, hadamard=had)
+        assert np.array_equal(scale.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+        assert np.array_equal(codes.cpu().numpy(), rc)
