@@ -1,6 +1,7 @@
 // attn_fwd.cuh -- causal prefill attention forward, O = softmax(Q K^T * scale
 // + causal mask) V, for sm_100a: persistent causal-aware scheduler, TMA-staged
-// K/V ring, tcgen05 MMAs into tensor memory, a warp-specialised softmax.
+// K/V ring, tcgen05 MMAs into tensor memory, warp-specialised softmax and
+// correction.
 //
 // Method: Zyphra ZYFA (news pages: the-ai.news "Zyphra presenteert ZYFA",
 // sections "Waarom presteert FP8 minder goed op de MI355X?" and "Drie
@@ -12,16 +13,27 @@
 // with block-scaled e4m3 MMAs that remove the scale.  BF16 path: the same
 // pipeline with exact exp2 probabilities rounded to bf16.
 //
-// CTA = 192 threads, one per SM (persistent grid):
-//   warps 0-3  softmax warpgroup: thread t owns query row t of the tile and
-//              TMEM lane t; online max, P, O rescale, epilogue
-//   warp 4     TMA producer (one thread): Q tile once per unit, K/V ring
-//   warp 5     MMA issuer (one thread): S = Q K^T, O += P V (+ row sum)
+// The pages overlap matrix and vector work by instruction order (two waves
+// per SIMD, ping-pong).  Blackwell tracks MMA completion in hardware, so the
+// overlap here is warp specialisation with mbarrier hand-offs.  CTA = 480
+// threads, one per SM (persistent grid):
+//   warps 0-7   softmax: warp w owns rows 32(w%4) .. 32(w%4)+31 of the tile
+//               (TMEM lane quarter w%4) and the 64-key block w/4 of each key
+//               tile; running max (block maxima exchanged between the two
+//               warps of a quarter), P (Lean-P codes or bf16), rescale factor
+//   warps 8-11  correction: rescales O (and the FP8 row sum) when the running
+//               max grew, then the epilogue O / l -> bf16 -> global
+//   warp 12     TMA producer (one elected thread): Q tile per unit, K/V ring
+//   warp 13     S issuer (one elected thread): S = Q K^T
+//   warp 14     P V issuer (one elected thread): O += P V (+ the FP8 row sum)
+// The two MMA streams are issued by different warps so that S of a later
+// tile never queues behind P V of an earlier one (each warp commits only its
+// own MMAs; the hand-offs between them go through the barriers).
 // Work unit = (batch, query head, 128-row query tile); KV tiles 0..qt only
 // (fully masked tiles are never issued), ascending, so results are
-// deterministic.  The MMA for S of tile j+1 overlaps the softmax of tile j
-// (two S buffers in TMEM); the P V MMA of tile j overlaps the softmax of
-// tile j+1.
+// deterministic.  S has two TMEM buffers: the MMA of S for tile j+1 runs
+// while the softmax works on tile j; P V of tile j runs while the softmax
+// works on tile j+1.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -48,6 +60,12 @@ struct AttnArgs {
   unsigned long long timeout_ns;
 };
 
+constexpr int kAttnThreads = 480;
+// BF16 only: the reference max of the exp2 is refreshed when the running max
+// exceeds it by more than this many binades (FlashAttention-4's lazy rescale;
+// the result is the same softmax, the O rescale becomes rare).
+constexpr float kBf16RescaleLog2 = 8.0f;
+
 template <bool FP8, int DQK>
 struct AttnCfg {
   static constexpr int EL = FP8 ? 1 : 2;            // bytes per input element
@@ -59,14 +77,23 @@ struct AttnCfg {
   static constexpr int KB = 128 * ROWB;
   static constexpr int VB = 128 * 128 * EL;          // Dv = 128
   static constexpr int ST = FP8 ? 4 : 2;             // K/V ring stages
+  static constexpr int QBUF = (!FP8 && DQK == 192) ? 1 : 2;   // Q tile buffers (units in flight)
   static constexpr int NK_QK = ROWB / 32;            // QK MMA K-steps of 32 bytes
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + QB;
+  static constexpr int OFF_K = OFF_Q + QBUF * QB;
   static constexpr int OFF_V = OFF_K + ST * KB;
   static constexpr int OFF_ONES = OFF_V + ST * VB;   // FP8: 16 x 128 bytes of e4m3 1.0
-  static constexpr int OFF_SFX = OFF_ONES + (FP8 ? 2048 : 0);
-  static constexpr int OFF_BAR = OFF_SFX + 2 * 128 * 4;
-  enum { QF = 0, QE, OD, OF, DRAIN, SF0, SF1, SC0, SC1, PF0, PF1, SX0, SX1, KF, };
+  static constexpr int OFF_SF = OFF_ONES + (FP8 ? 2048 : 0);   // FP8: 2 x 512 B scale factors
+  static constexpr int OFF_ALPHA = OFF_SF + (FP8 ? 1024 : 0);  // 2 x 128 fp32 rescale factors
+  static constexpr int OFF_LFIN = OFF_ALPHA + 1024;  // 2 buffers x 2 halves x 128 fp32 (BF16 final row sums)
+  static constexpr int OFF_XCH = OFF_LFIN + 2048;    // 2 buffers x 2 halves x 128 fp32 (block maxima)
+  static constexpr int OFF_BAR = OFF_XCH + 2048;
+  // Barriers (phase bookkeeping: every waiter is at most one phase behind,
+  // so a parity test cannot alias): Q full/empty per Q buffer; OF = O read
+  // by the epilogue (per unit); OFIN = last P V of a unit done (per unit);
+  // per S buffer: SF = S full, SC = S read, PF = P/alpha written, PE = P V
+  // done (P buffer free, O updated), OR = O corrected, ready for P V.
+  enum { QF0 = 0, QF1, QE0, QE1, OF, OFIN, DRAIN, DRAIN2, SF0, SF1, SC0, SC1, PF0, PF1, PE0, PE1, OR0, OR1, XC0, XC1, KF };
   static constexpr int KE = KF + ST, VF = KF + 2 * ST, VE = KF + 3 * ST;
   static constexpr int NBAR = KF + 4 * ST;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -117,10 +144,44 @@ struct UnitIter {
   }
 };
 
+// One lane of a converged warp (the same lane every time for the same mask).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// The CTA's sequence of (unit, KV tile) pairs in issue order; g counts tiles
+// and u counts units across the whole sequence (ring stages and barrier phases
+// derive from them).
+struct TileStream {
+  UnitIter units;
+  int b, hkv, hq, qt, j, nkv;
+  uint32_t g, u;
+  __device__ void init(int grid, int cta, int Tq, int Hq, int Hkv, int B, int Gk) {
+    units.init(grid, cta, Tq, Hq, Hkv, B, Gk);
+    j = 0; nkv = 0; g = 0xffffffffu; u = 0xffffffffu;
+  }
+  __device__ bool next() {
+    if (j + 1 < nkv) { ++j; ++g; return true; }
+    if (!units.next(b, hkv, hq, qt)) return false;
+    nkv = qt + 1; j = 0; ++g; ++u;
+    return true;
+  }
+};
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Two fp32 values -> bf16x2 (round to nearest even), first value in the low half.
@@ -146,20 +207,23 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-// Max of 64 consecutive fp32 values (held as bits) with 8 independent chains.
+// Max of 64 consecutive fp32 values (held as bits): 3-input max, 4 chains.
 __device__ __forceinline__ float max64(const uint32_t* s) {
-  float a[8];
+  float a[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(s[i]);
+  for (int i = 0; i < 4; ++i)                       // elements 0 .. 11
+    a[i] = max3f(__uint_as_float(s[i]), __uint_as_float(s[4 + i]), __uint_as_float(s[8 + i]));
 #pragma unroll
-  for (int c = 8; c < 64; c += 8)
+  for (int c = 12; c < 60; c += 8)                  // elements 12 .. 59
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], __uint_as_float(s[c + i]));
-  return fmaxf(fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])), fmaxf(fmaxf(a[4], a[5]), fmaxf(a[6], a[7])));
+    for (int i = 0; i < 4; ++i) a[i] = max3f(a[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 4 + i]));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = fmaxf(a[i], __uint_as_float(s[60 + i]));   // 60 .. 63
+  return max3f(fmaxf(a[0], a[1]), a[2], a[3]);
 }
 
 template <bool FP8, int DQK>
-__global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant__ AttnArgs a) {
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnArgs a) {
   using Cf = AttnCfg<FP8, DQK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -169,20 +233,28 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
   auto bar = [&](int i) -> uint32_t { return sb + Cf::OFF_BAR + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + Cf::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Cf::OFF_MISC + 4);
-  uint32_t* sfx = reinterpret_cast<uint32_t*>(sm + Cf::OFF_SFX);
+  float* alpha_s = reinterpret_cast<float*>(sm + Cf::OFF_ALPHA);
+  float* lfin_s = reinterpret_cast<float*>(sm + Cf::OFF_LFIN);
+  uint32_t* sf_s = reinterpret_cast<uint32_t*>(sm + Cf::OFF_SF);
+  float* xch_s = reinterpret_cast<float*>(sm + Cf::OFF_XCH);
 
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar(Cf::QF), 1);
-    mbar_init(bar(Cf::QE), 1);
-    mbar_init(bar(Cf::OD), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Cf::QF0 + i), 1);
+      mbar_init(bar(Cf::QE0 + i), 1);
+    }
     mbar_init(bar(Cf::OF), 128);
+    mbar_init(bar(Cf::OFIN), 1);
     mbar_init(bar(Cf::DRAIN), 1);
+    mbar_init(bar(Cf::DRAIN2), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(Cf::SF0 + i), 1);
-      mbar_init(bar(Cf::SC0 + i), 128);
-      mbar_init(bar(Cf::PF0 + i), 128);
-      mbar_init(bar(Cf::SX0 + i), 128);
+      mbar_init(bar(Cf::SC0 + i), 256);
+      mbar_init(bar(Cf::PF0 + i), 256);
+      mbar_init(bar(Cf::XC0 + i), 256);
+      mbar_init(bar(Cf::PE0 + i), 1);
+      mbar_init(bar(Cf::OR0 + i), 128);
     }
     for (int i = 0; i < Cf::ST; ++i) {
       mbar_init(bar(Cf::KF + i), 1);
@@ -192,7 +264,7 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
     }
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     prefetch_tensormap(&a.map_q);
     prefetch_tensormap(&a.map_k);
     prefetch_tensormap(&a.map_v);
@@ -204,7 +276,7 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
   }
   if (FP8) {
     uint32_t* ones = reinterpret_cast<uint32_t*>(sm + Cf::OFF_ONES);
-    for (int i = tid; i < 512; i += 192) ones[i] = 0x38383838u;   // e4m3 1.0
+    for (int i = tid; i < 512; i += kAttnThreads) ones[i] = 0x38383838u;   // e4m3 1.0
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -214,254 +286,334 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
   const WaitCtl ctl{abort_flag, a.timeout_ns};
   UnitIter units;
   units.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
-  const int gq = a.Hq / a.Hkv;
 
-  if (warp == 4) {
+  if (warp >= 12) {
+   // The producer and MMA warps run converged; one elected lane polls the
+   // barriers and issues the TMA copies / tcgen05 instructions and the
+   // commits, so every operand (descriptors, TMEM addresses, coordinates) is
+   // warp-uniform.
+   const bool leader = elect_one();
+   const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+   auto wait1 = [&](uint32_t br, uint32_t parity) -> bool {
+     bool ok = true;
+     if (leader) ok = mbar_wait(br, parity, ctl);
+     return __shfl_sync(0xffffffffu, ok ? 1 : 0, leader_lane) != 0;
+   };
+   if (warp == 12) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol_q = l2_policy_evict_first();
-      const uint64_t pol_kv = l2_policy_evict_last();
-      uint32_t kv_it = 0, u_it = 0;
-      int b, hkv, hq, qt;
-      bool ok = true;
-      auto load_qk = [&](uint32_t dst, const CUtensorMap* m, const CUtensorMap* mt, uint32_t br,
+    // K runs one tile ahead of V, in the order the MMAs consume them.
+    const uint64_t pol_q = l2_policy_evict_first();
+    const uint64_t pol_kv = l2_policy_evict_last();
+    TileStream ks, vs;
+    ks.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    vs.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    bool ok = true;
+    auto load_rows = [&](uint32_t dst, const CUtensorMap* m, const CUtensorMap* mt, uint32_t br,
                          int h, int row, int bb, uint64_t pol) {
 #pragma unroll
-        for (int c = 0; c < Cf::NCH; ++c)
-          tma_load_4d(dst + c * Cf::CHUNK, m, br, c * (128 / Cf::EL), h, row, bb, pol);
-        if (Cf::TAIL) tma_load_4d(dst + Cf::NCH * Cf::CHUNK, mt, br, 128, h, row, bb, pol);
-      };
-      while (ok && units.next(b, hkv, hq, qt)) {
-        if (u_it > 0 && !(ok = mbar_wait(bar(Cf::QE), (u_it - 1) & 1, ctl))) break;
-        mbar_arrive_expect_tx(bar(Cf::QF), Cf::QB);
-        load_qk(sb + Cf::OFF_Q, &a.map_q, &a.map_q_tail, bar(Cf::QF), hq, qt * 128, b, pol_q);
-        for (int j = 0; j <= qt; ++j, ++kv_it) {
-          const uint32_t st = kv_it % Cf::ST, n = kv_it / Cf::ST;
-          if (n > 0 && !(ok = mbar_wait(bar(Cf::KE + st), (n - 1) & 1, ctl))) break;
-          mbar_arrive_expect_tx(bar(Cf::KF + st), Cf::KB);
-          load_qk(sb + Cf::OFF_K + st * Cf::KB, &a.map_k, &a.map_k_tail, bar(Cf::KF + st), hkv,
-                  j * 128, b, pol_kv);
-          if (n > 0 && !(ok = mbar_wait(bar(Cf::VE + st), (n - 1) & 1, ctl))) break;
-          mbar_arrive_expect_tx(bar(Cf::VF + st), Cf::VB);
-#pragma unroll
-          for (int c = 0; c < Cf::VB / Cf::CHUNK; ++c)
-            tma_load_4d(sb + Cf::OFF_V + st * Cf::VB + c * Cf::CHUNK, &a.map_v, bar(Cf::VF + st),
-                        c * (128 / Cf::EL), hkv, j * 128, b, pol_kv);
+      for (int c = 0; c < Cf::NCH; ++c)
+        tma_load_4d(dst + c * Cf::CHUNK, m, br, c * (128 / Cf::EL), h, row, bb, pol);
+      if (Cf::TAIL) tma_load_4d(dst + Cf::NCH * Cf::CHUNK, mt, br, 128, h, row, bb, pol);
+    };
+    auto load_k = [&](const TileStream& t) -> bool {
+      if (t.j == 0) {                      // first tile of a unit: its Q tile first
+        const uint32_t slot = t.u % Cf::QBUF, n = t.u / Cf::QBUF;
+        if (n > 0 && !wait1(bar(Cf::QE0 + slot), (n - 1) & 1)) return false;
+        if (leader) {
+          mbar_arrive_expect_tx(bar(Cf::QF0 + slot), Cf::QB);
+          load_rows(sb + Cf::OFF_Q + slot * Cf::QB, &a.map_q, &a.map_q_tail, bar(Cf::QF0 + slot),
+                    t.hq, t.qt * 128, t.b, pol_q);
         }
-        ++u_it;
       }
-      if (!ok) {
-        // let copies already in flight land before the CTA exits
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+      const uint32_t st = t.g % Cf::ST, n = t.g / Cf::ST;
+      if (n > 0 && !wait1(bar(Cf::KE + st), (n - 1) & 1)) return false;
+      if (leader) {
+        mbar_arrive_expect_tx(bar(Cf::KF + st), Cf::KB);
+        load_rows(sb + Cf::OFF_K + st * Cf::KB, &a.map_k, &a.map_k_tail, bar(Cf::KF + st), t.hkv,
+                  t.j * 128, t.b, pol_kv);
       }
+      __syncwarp();
+      return true;
+    };
+    auto load_v = [&](const TileStream& t) -> bool {
+      const uint32_t st = t.g % Cf::ST, n = t.g / Cf::ST;
+      if (n > 0 && !wait1(bar(Cf::VE + st), (n - 1) & 1)) return false;
+      if (leader) {
+        mbar_arrive_expect_tx(bar(Cf::VF + st), Cf::VB);
+#pragma unroll
+        for (int c = 0; c < Cf::VB / Cf::CHUNK; ++c)
+          tma_load_4d(sb + Cf::OFF_V + st * Cf::VB + c * Cf::CHUNK, &a.map_v, bar(Cf::VF + st),
+                      c * (128 / Cf::EL), t.hkv, t.j * 128, t.b, pol_kv);
+      }
+      __syncwarp();
+      return true;
+    };
+    if (ks.next()) ok = load_k(ks);
+    while (ok && vs.next()) {
+      if (ks.next()) ok = load_k(ks);
+      if (ok) ok = load_v(vs);
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t qk_it = 0, u_it = 0;
-      int b, hkv, hq, qt;
-      bool ok = true;
-      auto issue_pv = [&](uint32_t kvi, bool first) -> bool {
-        const uint32_t st = kvi % Cf::ST, buf = kvi & 1;
-        if (!mbar_wait(bar(Cf::PF0 + buf), (kvi >> 1) & 1, ctl)) return false;
-        if (!mbar_wait(bar(Cf::VF + st), (kvi / Cf::ST) & 1, ctl)) return false;
-        if (first && u_it > 0 && !mbar_wait(bar(Cf::OF), (u_it - 1) & 1, ctl)) return false;
-        tc_fence_after();
-        const uint32_t vbase = sb + Cf::OFF_V + st * Cf::VB;
-        const uint32_t tp = tbase + (buf ? Cf::TP1 : Cf::TP0);
+    if (!ok) {
+      // let copies already in flight land before the CTA exits
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+   } else if (warp == 13 || warp == 14) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 9: S for tile g is issued as soon as its K tile is loaded and the
+    // softmax has read S of tile g-2 (two S buffers).  warp 10: P V of tile g
+    // once the softmax has written P and the correction has rescaled O.
+    TileStream ts;
+    ts.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    bool ok = true;
+    // descriptor bases; per-step descriptors add (byte offset >> 4) to the low word
+    const uint64_t dq = smem_desc(sb + Cf::OFF_Q, 16, 1024, kSw128);
+    const uint64_t dq_t = smem_desc(sb + Cf::OFF_Q + Cf::NCH * Cf::CHUNK, 16, 512, kSw64);
+    const uint64_t dk = smem_desc(sb + Cf::OFF_K, 16, 1024, kSw128);
+    const uint64_t dk_t = smem_desc(sb + Cf::OFF_K + Cf::NCH * Cf::CHUNK, 16, 512, kSw64);
+    const uint64_t dv = smem_desc(sb + Cf::OFF_V, 16384, 1024, kSw128);
+    const uint64_t dones = smem_desc(sb + Cf::OFF_ONES, 16, 1024, kSw128);
+    const uint64_t dsf = smem_desc(sb + Cf::OFF_SF, 16, 128, kSwNone);
+    auto issue_qk = [&](const TileStream& t) -> bool {
+      const uint32_t slot = t.u % Cf::QBUF;
+      if (t.j == 0 && !wait1(bar(Cf::QF0 + slot), (t.u / Cf::QBUF) & 1)) return false;
+      const uint32_t st = t.g % Cf::ST, buf = t.g & 1;
+      if (!wait1(bar(Cf::KF + st), (t.g / Cf::ST) & 1)) return false;
+      if (t.g >= 2 && !wait1(bar(Cf::SC0 + buf), ((t.g >> 1) - 1) & 1)) return false;
+      tc_fence_after();
+      const uint64_t dqs = dq + ((slot * Cf::QB) >> 4), dqs_t = dq_t + ((slot * Cf::QB) >> 4);
+      const uint64_t dks = dk + ((st * Cf::KB) >> 4), dks_t = dk_t + ((st * Cf::KB) >> 4);
+      const uint32_t ts = tbase + (buf ? Cf::TS1 : Cf::TS0);
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < Cf::NK_QK; ++kk) {
+          uint64_t ad, bd;
+          if (kk < Cf::NCH * 4) {
+            const uint32_t off = ((kk >> 2) * Cf::CHUNK + (kk & 3) * 32) >> 4;
+            ad = dqs + off; bd = dks + off;
+          } else {
+            const uint32_t off = ((kk - Cf::NCH * 4) * 32) >> 4;
+            ad = dqs_t + off; bd = dks_t + off;
+          }
+          if (FP8) mma_f8_ss(ts, ad, bd, Cf::IDESC_QK, kk > 0 ? 1u : 0u);
+          else mma_f16_ss(ts, ad, bd, Cf::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(Cf::SF0 + buf));
+        tc_commit(bar(Cf::KE + st));
+        if (t.j == t.nkv - 1) tc_commit(bar(Cf::QE0 + slot));
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_pv = [&](const TileStream& t) -> bool {
+      const uint32_t st = t.g % Cf::ST, buf = t.g & 1;
+      const bool first = t.j == 0;
+      // O is free once the previous unit's epilogue has read it
+      if (first && t.u > 0 && !wait1(bar(Cf::OF), (t.u - 1) & 1)) return false;
+      if (!wait1(bar(Cf::OR0 + buf), (t.g >> 1) & 1)) return false;   // P stored, O corrected
+      if (!wait1(bar(Cf::VF + st), (t.g / Cf::ST) & 1)) return false;
+      tc_fence_after();
+      const uint64_t dvs = dv + ((st * Cf::VB) >> 4);
+      const uint32_t tp = tbase + (buf ? Cf::TP1 : Cf::TP0);
+      if (leader) {
         if (FP8) {
           const uint32_t sfa = tbase + (buf ? Cf::TSFA1 : Cf::TSFA0);
           const uint32_t sfb = tbase + Cf::TSFB;
+          // scale factors of P: 32 rows x 16 bytes in shared memory, copied to
+          // all four lane quarters (the layout the block-scaled MMA reads)
+          tmem_cp_32x128b_warpx4(sfa, dsf + ((buf * 512) >> 4));
 #pragma unroll
-          for (uint32_t ks = 0; ks < 4; ++ks) {
-            const uint64_t bd = smem_desc(vbase + ks * 4096, 16384, 1024, kSw128);
-            mma_mxf8_ts(tbase + Cf::TO, tp + 8 * ks, bd, idesc_mxf8(1, 128, 128, ks, ks),
-                        sfa | (ks << 30), sfb | (ks << 30), (!first || ks > 0) ? 1u : 0u);
-          }
+          for (uint32_t k4 = 0; k4 < 4; ++k4)
+            mma_mxf8_ts(tbase + Cf::TO, tp + 8 * k4, dvs + ((k4 * 4096) >> 4), idesc_mxf8(1, 128, 128, k4, k4),
+                        sfa | (k4 << 30), sfb | (k4 << 30), (!first || k4 > 0) ? 1u : 0u);
 #pragma unroll
-          for (uint32_t ks = 0; ks < 4; ++ks) {
-            const uint64_t bd = smem_desc(sb + Cf::OFF_ONES + ks * 32, 16, 1024, kSw128);
-            mma_mxf8_ts(tbase + Cf::TL, tp + 8 * ks, bd, idesc_mxf8(0, 128, 16, ks, ks),
-                        sfa | (ks << 30), sfb | (ks << 30), (!first || ks > 0) ? 1u : 0u);
-          }
+          for (uint32_t k4 = 0; k4 < 4; ++k4)
+            mma_mxf8_ts(tbase + Cf::TL, tp + 8 * k4, dones + ((k4 * 32) >> 4), idesc_mxf8(0, 128, 16, k4, k4),
+                        sfa | (k4 << 30), sfb | (k4 << 30), (!first || k4 > 0) ? 1u : 0u);
         } else {
 #pragma unroll
-          for (uint32_t ks = 0; ks < 8; ++ks) {
-            const uint64_t bd = smem_desc(vbase + ks * 2048, 16384, 1024, kSw128);
-            mma_f16_ts(tbase + Cf::TO, tp + 8 * ks, bd, Cf::IDESC_PV_BF16,
-                       (!first || ks > 0) ? 1u : 0u);
-          }
+          for (uint32_t k8 = 0; k8 < 8; ++k8)
+            mma_f16_ts(tbase + Cf::TO, tp + 8 * k8, dvs + ((k8 * 2048) >> 4), Cf::IDESC_PV_BF16,
+                       (!first || k8 > 0) ? 1u : 0u);
         }
-        tc_commit(bar(Cf::OD));
         tc_commit(bar(Cf::VE + st));
-        return true;
-      };
-      while (ok && units.next(b, hkv, hq, qt)) {
-        const int nkv = qt + 1;
-        if (!(ok = mbar_wait(bar(Cf::QF), u_it & 1, ctl))) break;
-        for (int j = 0; j < nkv && ok; ++j) {
-          const uint32_t kvi = qk_it + j, st = kvi % Cf::ST, buf = kvi & 1;
-          if (!(ok = mbar_wait(bar(Cf::KF + st), (kvi / Cf::ST) & 1, ctl))) break;
-          if (kvi >= 2 && !(ok = mbar_wait(bar(Cf::SC0 + buf), ((kvi >> 1) - 1) & 1, ctl))) break;
-          tc_fence_after();
-          const uint32_t kbase = sb + Cf::OFF_K + st * Cf::KB;
-          const uint32_t ts = tbase + (buf ? Cf::TS1 : Cf::TS0);
-#pragma unroll
-          for (int kk = 0; kk < Cf::NK_QK; ++kk) {
-            uint32_t off, sbo, swz;
-            if (kk < Cf::NCH * 4) { off = (kk >> 2) * Cf::CHUNK + (kk & 3) * 32; sbo = 1024; swz = kSw128; }
-            else { off = Cf::NCH * Cf::CHUNK + (kk - Cf::NCH * 4) * 32; sbo = 512; swz = kSw64; }
-            const uint64_t ad = smem_desc(sb + Cf::OFF_Q + off, 16, sbo, swz);
-            const uint64_t bd = smem_desc(kbase + off, 16, sbo, swz);
-            if (FP8) mma_f8_ss(ts, ad, bd, Cf::IDESC_QK, kk > 0 ? 1u : 0u);
-            else mma_f16_ss(ts, ad, bd, Cf::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(Cf::SF0 + buf));
-          tc_commit(bar(Cf::KE + st));
-          if (j == nkv - 1) tc_commit(bar(Cf::QE));
-          if (j >= 1) ok = issue_pv(kvi - 1, j == 1);
-        }
-        if (ok) ok = issue_pv(qk_it + nkv - 1, nkv == 1);
-        qk_it += nkv;
-        ++u_it;
+        tc_commit(bar(Cf::PE0 + buf));    // P (and its scale factors) of this buffer consumed
+        if (t.j == t.nkv - 1) tc_commit(bar(Cf::OFIN));
       }
-      // all MMAs issued by this thread must finish before TMEM is released
-      tc_commit(bar(Cf::DRAIN));
-      drain_wait(bar(Cf::DRAIN), 0, 100000000ull);
+      __syncwarp();
+      return true;
+    };
+    if (warp == 13) {
+      while (ok && ts.next()) ok = issue_qk(ts);
+    } else {
+      while (ok && ts.next()) ok = issue_pv(ts);
     }
-  } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    const int row = tid;   // query row inside the tile == TMEM lane
-    const uint32_t lb = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-    uint32_t kv_it = 0, u_it = 0;
+    // all MMAs issued by this warp's leader must finish before TMEM is released
+    if (leader) {
+      const uint32_t dr = bar(warp == 13 ? Cf::DRAIN : Cf::DRAIN2);
+      tc_commit(dr);
+      drain_wait(dr, 0, 100000000ull);
+    }
+    __syncwarp();
+   }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax warpgroups
+    // warp w: lane quarter q = w % 4 (rows 32q .. 32q+31), key half h = w / 4
+    // (keys 64h .. 64h+63 of each tile = one 64-key scale block).  The two
+    // warps of a quarter exchange their block maxima once per tile.
+    const int q4 = warp & 3, half = warp >> 2;
+    const int row = 32 * q4 + lane;   // query row inside the tile == TMEM lane
+    const uint32_t lb = tbase + (static_cast<uint32_t>(q4 * 32) << 16);
+    uint32_t kv_it = 0;
     int b, hkv, hq, qt;
     bool ok = true;
-    if (FP8) {
+    if (FP8 && half == 0) {
       tmem_st4(lb + Cf::TSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);  // scale 1.0
       tmem_wait_st();
     }
+    // scale-factor word of row r: bytes at (r % 32) * 16 + (r / 32) * 4; this
+    // half writes the two bytes of its 64-key block
+    uint16_t* sf_h = reinterpret_cast<uint16_t*>(sf_s) + 2 * ((row & 31) * 4 + (row >> 5)) + half;
     while (ok && units.next(b, hkv, hq, qt)) {
       const int nkv = qt + 1;
-      float A = a.C, vsc = 1.0f;
+      float A = a.C;
       if (FP8) {
         const float qs = a.q_scale ? a.q_scale[b * a.Hq + hq] : 1.0f;
         const float ks = a.k_scale ? a.k_scale[b * a.Hkv + hkv] : 1.0f;
-        vsc = a.v_scale ? a.v_scale[b * a.Hkv + hkv] : 1.0f;
         A = leanp_slope(qs, ks, a.C);
       }
-      float m = __int_as_float(0xff800000);
-      float l = 0.0f;
+      float m = __int_as_float(0xff800000);   // FP8: running max; BF16: exp2 reference max
+      float l = 0.0f;                          // BF16 row sum over this half's keys
       for (int j = 0; j < nkv; ++j, ++kv_it) {
         const uint32_t buf = kv_it & 1;
         if (!(ok = warp_wait(bar(Cf::SF0 + buf), (kv_it >> 1) & 1, ctl))) break;
         tc_fence_after();
-        uint32_t r[128];
+        uint32_t r[64];
         {
-          const uint32_t ts = lb + (buf ? Cf::TS1 : Cf::TS0);
+          const uint32_t ts = lb + (buf ? Cf::TS1 : Cf::TS0) + 64 * half;
           tmem_ld32p(ts, &r[0]);
           tmem_ld32p(ts + 32, &r[32]);
-          tmem_ld32p(ts + 64, &r[64]);
-          tmem_ld32p(ts + 96, &r[96]);
           tmem_wait_ld();
         }
         tc_fence_before();
         mbar_arrive(bar(Cf::SC0 + buf));
         if (j == qt) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > row) r[c] = 0xff800000u;   // -inf: key after the query row
+          for (int c = 0; c < 64; ++c)
+            if (64 * half + c > row) r[c] = 0xff800000u;   // -inf: key after the query row
         }
-        const float bm0 = max64(r), bm1 = max64(r + 64);
-        const float m_new = fmaxf(m, fmaxf(bm0, bm1));
-        uint32_t p[32];
-        float tile_sum = 0.0f;
-        uint32_t sf0 = 0, sf1 = 0, sf2 = 0, sf3 = 0;
+        const float bm = max64(r);
+        xch_s[(buf * 2 + half) * 128 + row] = bm;
+        mbar_arrive(bar(Cf::XC0 + buf));
+        if (!(ok = warp_wait(bar(Cf::XC0 + buf), (kv_it >> 1) & 1, ctl))) break;
+        const float bo = xch_s[(buf * 2 + (half ^ 1)) * 128 + row];
+        float alpha = 1.0f;
         if (FP8) {
-          const int j0 = leanp_block_shift(m_new, bm0, A);
-          const int j1 = leanp_block_shift(m_new, bm1, A);
-          const float B0 = leanp_row_offset(m_new, A, j0);
-          const float B1 = leanp_row_offset(m_new, A, j1);
+          // Lean P against the running max after this tile
+          const float m_new = max3f(m, bm, bo);
+          if (j > 0 && m_new > m) alpha = ex2_approx(__fmul_rn(__fmul_rn(m - m_new, A), 0.125f));
+          m = m_new;
+          const int jb = leanp_block_shift(m, bm, A);
+          const float Bb = leanp_row_offset(m, A, jb);
+          const float a256 = __fmul_rn(A, 0.00390625f), b256 = __fmul_rn(Bb, 0.00390625f);
+          uint32_t p[16];
 #pragma unroll
-          for (int w = 0; w < 32; ++w) {
-            const float Bw = w < 16 ? B0 : B1;
-            p[w] = pack4_low_bytes(leanp_code_word(__uint_as_float(r[4 * w]), A, Bw),
-                                   leanp_code_word(__uint_as_float(r[4 * w + 1]), A, Bw),
-                                   leanp_code_word(__uint_as_float(r[4 * w + 2]), A, Bw),
-                                   leanp_code_word(__uint_as_float(r[4 * w + 3]), A, Bw));
-          }
-          // E8M0 scale codes 127 - j: bytes 0,1 cover keys 0-63, bytes 2,3 keys 64-127
-          const uint32_t e0 = static_cast<uint32_t>(127 - j0), e1 = static_cast<uint32_t>(127 - j1);
-          sfx[buf * 128 + row] = e0 * 0x0101u | (e1 * 0x0101u) << 16;
-          mbar_arrive(bar(Cf::SX0 + buf));
-          if (!(ok = warp_wait(bar(Cf::SX0 + buf), (kv_it >> 1) & 1, ctl))) break;
-          // scale-factor layout for M = 128: column c, lane 32w+i holds row 32c+i (all w)
-          sf0 = sfx[buf * 128 + lane];
-          sf1 = sfx[buf * 128 + 32 + lane];
-          sf2 = sfx[buf * 128 + 64 + lane];
-          sf3 = sfx[buf * 128 + 96 + lane];
+          for (int w = 0; w < 16; ++w)
+            p[w] = pack4_low_bytes(leanp_code_word(__uint_as_float(r[4 * w]), a256, b256),
+                                   leanp_code_word(__uint_as_float(r[4 * w + 1]), a256, b256),
+                                   leanp_code_word(__uint_as_float(r[4 * w + 2]), a256, b256),
+                                   leanp_code_word(__uint_as_float(r[4 * w + 3]), a256, b256));
+          // P V of tile kv_it-2 has read this P buffer and its scale factors
+          if (kv_it >= 2 && !(ok = warp_wait(bar(Cf::PE0 + buf), ((kv_it >> 1) - 1) & 1, ctl))) break;
+          tmem_st16p(lb + (buf ? Cf::TP1 : Cf::TP0) + 16 * half, p);
+          // E8M0 scale code 127 - j for both 32-key MX blocks of this 64-key block
+          sf_h[buf * 256] = static_cast<uint16_t>((127 - jb) * 0x0101);
+          fence_proxy_async_smem();   // the copy to TMEM reads it through the async proxy
         } else {
-          const float mc = m_new * A;
+          const float tmax = fmaxf(bm, bo);
+          if (j == 0) {
+            m = tmax;
+          } else if (__fmul_rn(tmax - m, A) > kBf16RescaleLog2) {
+            alpha = ex2_approx(__fmul_rn(m - tmax, A));
+            m = tmax;
+          }
+          const float mc = m * A;
           float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          uint32_t pb[64];
+          const uint32_t tp = lb + (buf ? Cf::TP1 : Cf::TP0) + 32 * half;
+          // P V of tile kv_it-2 has read this P buffer
+          if (kv_it >= 2 && !(ok = warp_wait(bar(Cf::PE0 + buf), ((kv_it >> 1) - 1) & 1, ctl))) break;
 #pragma unroll
-          for (int w = 0; w < 64; ++w) {
-            const float p0 = ex2_approx(__fmaf_rn(__uint_as_float(r[2 * w]), A, -mc));
-            const float p1 = ex2_approx(__fmaf_rn(__uint_as_float(r[2 * w + 1]), A, -mc));
-            acc[w & 3] += p0 + p1;
-            pb[w] = pack_bf16x2(p0, p1);
-          }
-          tile_sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-          const uint32_t tp = lb + (buf ? Cf::TP1 : Cf::TP0);
-          tmem_st32p(tp, &pb[0]);
-          tmem_st32p(tp + 32, &pb[32]);
-        }
-        // online-softmax correction of O (and l) when the running max grew
-        if (j > 0) {
-          const bool need = m_new > m;
-          const float alpha = need ? ex2_approx(__fmul_rn(__fmul_rn(m - m_new, A), FP8 ? 0.125f : 1.0f)) : 1.0f;
-          if (!FP8) l *= alpha;
-          if (__any_sync(0xffffffffu, need)) {
-            if (!(ok = warp_wait(bar(Cf::OD), (kv_it - 1) & 1, ctl))) break;
-            tc_fence_after();
+          for (int c4 = 0; c4 < 4; ++c4) {   // four chunks of 16 keys keep register pressure down
+            uint32_t pb[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t o[32];
-              tmem_ld32p(lb + Cf::TO + 32 * q, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32p(lb + Cf::TO + 32 * q, o);
+            for (int w = 0; w < 8; ++w) {
+              const float p0 = ex2_approx(__fmaf_rn(__uint_as_float(r[16 * c4 + 2 * w]), A, -mc));
+              const float p1 = ex2_approx(__fmaf_rn(__uint_as_float(r[16 * c4 + 2 * w + 1]), A, -mc));
+              acc[w & 3] += p0 + p1;
+              pb[w] = pack_bf16x2(p0, p1);
             }
-            if (FP8) {
-              const uint32_t lv = tmem_ld1(lb + Cf::TL);
-              tmem_wait_ld();
-              tmem_st1(lb + Cf::TL, __float_as_uint(__uint_as_float(lv) * alpha));
-            }
+            tmem_st8p(tp + 8 * c4, pb);
           }
+          l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+          if (j == nkv - 1) lfin_s[(buf * 2 + half) * 128 + row] = l;
         }
-        if (!FP8) l += tile_sum;
-        m = m_new;
-        if (FP8) {
-          const uint32_t tp = lb + (buf ? Cf::TP1 : Cf::TP0);
-          tmem_st32p(tp, p);
-          tmem_st4(lb + (buf ? Cf::TSFA1 : Cf::TSFA0), sf0, sf1, sf2, sf3);
-        }
+        if (half == 0) alpha_s[buf * 128 + row] = alpha;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(Cf::PF0 + buf));
       }
+    }
+  } else {
+    // ------------------------------------------------------------ correction warpgroup
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lb = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    uint32_t kv_it = 0, u_it = 0;
+    int b, hkv, hq, qt;
+    bool ok = true;
+    while (ok && units.next(b, hkv, hq, qt)) {
+      const int nkv = qt + 1;
+      float l_final = 1.0f;
+      for (int j = 0; j < nkv; ++j, ++kv_it) {
+        const uint32_t buf = kv_it & 1;
+        if (!(ok = warp_wait(bar(Cf::PF0 + buf), (kv_it >> 1) & 1, ctl))) break;
+        const float alpha = alpha_s[buf * 128 + row];
+        if (!FP8 && j == nkv - 1) l_final = lfin_s[(buf * 2) * 128 + row] + lfin_s[(buf * 2 + 1) * 128 + row];
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          // O holds tiles 0..j-1: wait for P V of tile j-1, then scale the rows
+          const uint32_t pg = kv_it - 1;
+          if (!(ok = warp_wait(bar(Cf::PE0 + (pg & 1)), (pg >> 1) & 1, ctl))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            tmem_ld32p(lb + Cf::TO + 32 * q, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32p(lb + Cf::TO + 32 * q, o);
+          }
+          if (FP8) {
+            const uint32_t lv = tmem_ld1(lb + Cf::TL);
+            tmem_wait_ld();
+            tmem_st1(lb + Cf::TL, __float_as_uint(__uint_as_float(lv) * alpha));
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(Cf::OR0 + buf));
+      }
       if (!ok) break;
       // ---- epilogue: O / l (* v_scale) -> bf16, rows past S are not written
-      if (!(ok = warp_wait(bar(Cf::OD), (kv_it - 1) & 1, ctl))) break;
+      if (!(ok = warp_wait(bar(Cf::OFIN), u_it & 1, ctl))) break;
       tc_fence_after();
       float inv;
       if (FP8) {
+        const float vsc = a.v_scale ? a.v_scale[b * a.Hkv + hkv] : 1.0f;
         const float lv = __uint_as_float(tmem_ld1(lb + Cf::TL));
         tmem_wait_ld();
         inv = vsc / lv;
       } else {
-        inv = 1.0f / l;
+        inv = 1.0f / l_final;
       }
       const int grow = qt * 128 + row;
       __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.S + grow) * a.Hq + hq) * 128;
@@ -490,7 +642,6 @@ __global__ void __launch_bounds__(192, 1) attn_fwd_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tbase, 512);
-  (void)gq;
 }
 
 }  // namespace zyfa

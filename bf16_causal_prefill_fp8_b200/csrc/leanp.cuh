@@ -17,8 +17,7 @@
 //          min(126, 8 + floor(((m - bmax) * A) * 0.125))         per row, block
 //   B    = fma(-m, A, 56 + 8 j)                                   per row, block
 //   u    = fma(s, A, B)                                           per element
-//   code = trunc(max(u, 0))           (the low byte of fp32(max(u,0) + 1.5*2^23)
-//                                       added with round-toward-zero)
+//   code = trunc(max(u, 0))           (see leanp_code_word)
 // s is the raw fp32 score (sum of products of e4m3 values), m the running row
 // maximum after this key tile and bmax the maximum of the element's 64-key
 // block.  Precondition: s <= bmax <= m, or s = -inf for a masked key; then
@@ -43,10 +42,29 @@ __device__ __forceinline__ float leanp_row_offset(float m, float A, int j) {
   return __fmaf_rn(-m, A, static_cast<float>(56 + 8 * j));
 }
 
-// Returns a 32-bit word whose low byte is the e4m3 code of score s.
-__device__ __forceinline__ uint32_t leanp_code_word(float s, float A, float B) {
-  const float u = fmaxf(__fmaf_rn(s, A, B), 0.0f);
-  return __float_as_uint(__fadd_rz(u, 12582912.0f));
+// The code of one score is computed as (leanp_code_word)
+//   x = sat(fma(s, A/256, B/256))       (= fp32(u)/256 clamped to [0, 1]; the
+//                                         division by 256 is exact and commutes
+//                                         with the rounding for normal values)
+//   w = fma_rz(x, 256, 1.5 * 2^23)       (= 1.5 * 2^23 + trunc(fp32(u)) exactly)
+// so the low byte of w's bits is trunc(max(u, 0)) for 0 <= u < 256: two
+// FMA-pipe instructions per score, no integer conversion.  a256 = A/256 and
+// b256 = B/256 are computed once per (row, block).
+__device__ __forceinline__ float leanp_scaled_u(float s, float a256, float b256) {
+  float x;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(x) : "f"(s), "f"(a256), "f"(b256));
+  return x;
+}
+
+__device__ __forceinline__ uint32_t leanp_word(float x) {
+  float w;
+  asm("fma.rz.f32 %0, %1, 0f43800000, 0f4B400000;" : "=f"(w) : "f"(x));   // x * 256 + 1.5 * 2^23
+  return __float_as_uint(w);
+}
+
+// One score -> a word whose low byte is its code (a256 = A/256, b256 = B/256).
+__device__ __forceinline__ uint32_t leanp_code_word(float s, float a256, float b256) {
+  return leanp_word(leanp_scaled_u(s, a256, b256));
 }
 
 // Four code words -> one 32-bit word holding the four code bytes in order.

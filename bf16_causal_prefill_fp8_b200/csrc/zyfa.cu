@@ -129,7 +129,7 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int
   }
   const long long units = static_cast<long long>(B) * Hq * a.Tq;
   const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
-  attn_fwd_kernel<FP8, DQK><<<grid, 192, Cf::SMEM, stream>>>(a);
+  attn_fwd_kernel<FP8, DQK><<<grid, kAttnThreads, Cf::SMEM, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
@@ -142,7 +142,8 @@ __global__ void leanp_codes_kernel(const float* s, const float* m, const float* 
     const int j = leanp_block_shift(mi, bmax[i], Ai);
     const float B = leanp_row_offset(mi, Ai, j);
     const float si = (masked && masked[i]) ? __int_as_float(0xff800000) : s[i];
-    code[i] = static_cast<unsigned char>(leanp_code_word(si, Ai, B) & 0xffu);
+    const uint32_t w = leanp_code_word(si, __fmul_rn(Ai, 0.00390625f), __fmul_rn(B, 0.00390625f));
+    code[i] = static_cast<unsigned char>(w & 0xffu);
     if (jout) jout[i] = j;
   }
 }

@@ -1,0 +1,42 @@
+"""Run one workload's kernels a few times, for a profiler to capture.
+
+    python -m bf16_causal_prefill_fp8_b200.profile_case --workload gqa32x8_s16k_outlier --iters 3
+
+Each iteration launches, in order: zyfa_quantize for Q, K and V (amax, codes
+and finalize kernels each), the FP8 attention kernel, then the BF16 attention
+kernel on the same bf16 inputs.  Prints nothing but a completion line; timing
+numbers come from bench.py, never from a profiled run.
+"""
+import argparse
+
+import torch
+
+from . import synth, zyfa
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="gqa32x8_s16k_outlier", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--hadamard", action="store_true")
+    ap.add_argument("--only", choices=["all", "fp8", "bf16"], default="all")
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    q, k, v = synth.make_qkv(0, wl["B"], wl["S"], wl["Hq"], wl["Hkv"], wl["Dqk"], wl["Dv"], wl["kind"])
+    dq, dk, dv = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (q, k, v))
+    for _ in range(args.iters):
+        if args.only in ("all", "fp8"):
+            cq, sq = zyfa.quantize(dq, hadamard=args.hadamard)
+            ck, sk = zyfa.quantize(dk, hadamard=args.hadamard)
+            cv, sv = zyfa.quantize(dv)
+            zyfa.attn_fwd(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv)
+        if args.only in ("all", "bf16"):
+            zyfa.attn_fwd(dq, dk, dv)
+    torch.cuda.synchronize()
+    st = zyfa.device_status()
+    print(f"profile_case {args.workload}: {args.iters} iterations done, device status {st}")
+    return 0 if st == zyfa.OK else 1
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())
