@@ -85,15 +85,15 @@ struct AttnCfg {
   static constexpr int OFF_ONES = OFF_V + ST * VB;   // FP8: 16 x 128 bytes of e4m3 1.0
   static constexpr int OFF_SF = OFF_ONES + (FP8 ? 2048 : 0);   // FP8: 2 x 512 B scale factors
   static constexpr int OFF_ALPHA = OFF_SF + (FP8 ? 1024 : 0);  // 2 x 128 fp32 rescale factors
-  static constexpr int OFF_LFIN = OFF_ALPHA + 1024;  // 2 buffers x 2 halves x 128 fp32 (BF16 final row sums)
-  static constexpr int OFF_XCH = OFF_LFIN + 2048;    // 2 buffers x 2 halves x 128 fp32 (block maxima)
+  static constexpr int OFF_LFIN = OFF_ALPHA + 1024;  // BF16 final partial row sums, per group (2 x 128 fp32, 1 KB used)
+  static constexpr int OFF_XCH = OFF_LFIN + 2048;    // running max per group (2 x 128) + BF16 final max per group (2 x 128)
   static constexpr int OFF_BAR = OFF_XCH + 2048;
   // Barriers (phase bookkeeping: every waiter is at most one phase behind,
   // so a parity test cannot alias): Q full/empty per Q buffer; OF = O read
   // by the epilogue (per unit); OFIN = last P V of a unit done (per unit);
   // per S buffer: SF = S full, SC = S read, PF = P/alpha written, PE = P V
   // done (P buffer free, O updated), OR = O corrected, ready for P V.
-  enum { QF0 = 0, QF1, QE0, QE1, OF, OFIN, DRAIN, DRAIN2, SF0, SF1, SC0, SC1, PF0, PF1, PE0, PE1, OR0, OR1, XC0, XC1, KF };
+  enum { QF0 = 0, QF1, QE0, QE1, OF, OFIN, DRAIN, DRAIN2, SF0, SF1, SC0, SC1, PF0, PF1, PE0, PE1, OR0, OR1, MX0, MX1, KF };
   static constexpr int KE = KF + ST, VF = KF + 2 * ST, VE = KF + 3 * ST;
   static constexpr int NBAR = KF + 4 * ST;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -250,9 +250,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     mbar_init(bar(Cf::DRAIN2), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(Cf::SF0 + i), 1);
-      mbar_init(bar(Cf::SC0 + i), 256);
-      mbar_init(bar(Cf::PF0 + i), 256);
-      mbar_init(bar(Cf::XC0 + i), 256);
+      mbar_init(bar(Cf::SC0 + i), 128);
+      mbar_init(bar(Cf::PF0 + i), 128);
+      mbar_init(bar(Cf::MX0 + i), 128);
       mbar_init(bar(Cf::PE0 + i), 1);
       mbar_init(bar(Cf::OR0 + i), 128);
     }
@@ -458,62 +458,104 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
    }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warpgroups
-    // warp w: lane quarter q = w % 4 (rows 32q .. 32q+31), key half h = w / 4
-    // (keys 64h .. 64h+63 of each tile = one 64-key scale block).  The two
-    // warps of a quarter exchange their block maxima once per tile.
-    const int q4 = warp & 3, half = warp >> 2;
-    const int row = 32 * q4 + lane;   // query row inside the tile == TMEM lane
-    const uint32_t lb = tbase + (static_cast<uint32_t>(q4 * 32) << 16);
-    uint32_t kv_it = 0;
-    int b, hkv, hq, qt;
+    // Two groups alternate over the KV tiles: group x = warp / 4 takes the
+    // tiles with (g & 1) == x, i.e. always S buffer x and P buffer x, so one
+    // group computes while the other waits for its next S.  Thread t of a
+    // group owns row 32 (w % 4) + lane (TMEM lane quarter w % 4) and all 128
+    // keys of its tiles.  The running max crosses between the groups once per
+    // tile (smem + per-buffer barrier MX), the only serial dependency.
+    const int grp = warp >> 2;
+    const int row = 32 * (warp & 3) + lane;   // query row inside the tile == TMEM lane
+    const uint32_t lb = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     bool ok = true;
-    if (FP8 && half == 0) {
+    if (FP8 && grp == 0) {
       tmem_st4(lb + Cf::TSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);  // scale 1.0
       tmem_wait_st();
     }
-    // scale-factor word of row r: bytes at (r % 32) * 16 + (r / 32) * 4; this
-    // half writes the two bytes of its 64-key block
-    uint16_t* sf_h = reinterpret_cast<uint16_t*>(sf_s) + 2 * ((row & 31) * 4 + (row >> 5)) + half;
-    while (ok && units.next(b, hkv, hq, qt)) {
-      const int nkv = qt + 1;
-      float A = a.C;
-      if (FP8) {
-        const float qs = a.q_scale ? a.q_scale[b * a.Hq + hq] : 1.0f;
-        const float ks = a.k_scale ? a.k_scale[b * a.Hkv + hkv] : 1.0f;
-        A = leanp_slope(qs, ks, a.C);
-      }
-      float m = __int_as_float(0xff800000);   // FP8: running max; BF16: exp2 reference max
-      float l = 0.0f;                          // BF16 row sum over this half's keys
-      for (int j = 0; j < nkv; ++j, ++kv_it) {
-        const uint32_t buf = kv_it & 1;
-        if (!(ok = warp_wait(bar(Cf::SF0 + buf), (kv_it >> 1) & 1, ctl))) break;
-        tc_fence_after();
-        uint32_t r[64];
-        {
-          const uint32_t ts = lb + (buf ? Cf::TS1 : Cf::TS0) + 64 * half;
-          tmem_ld32p(ts, &r[0]);
-          tmem_ld32p(ts + 32, &r[32]);
-          tmem_wait_ld();
+    // scale-factor word of row r: bytes at (r % 32) * 16 + (r / 32) * 4
+    uint32_t* sf_w = sf_s + grp * 128 + ((row & 31) * 4 + (row >> 5));
+    const uint32_t ts = lb + (grp ? Cf::TS1 : Cf::TS0);
+    const uint32_t tp = lb + (grp ? Cf::TP1 : Cf::TP0);
+    TileStream t;
+    t.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    float A = a.C;
+    float l = 0.0f, m_own = __int_as_float(0xff800000);   // BF16: this group's row sum and its max
+    while (ok && t.next()) {
+      const uint32_t g = t.g;
+      if (t.j == 0) {
+        l = 0.0f;
+        m_own = __int_as_float(0xff800000);
+        if (FP8) {
+          const float qs = a.q_scale ? a.q_scale[t.b * a.Hq + t.hq] : 1.0f;
+          const float ks = a.k_scale ? a.k_scale[t.b * a.Hkv + t.hkv] : 1.0f;
+          A = leanp_slope(qs, ks, a.C);
         }
-        tc_fence_before();
-        mbar_arrive(bar(Cf::SC0 + buf));
-        if (j == qt) {
+      }
+      if ((g & 1) != static_cast<uint32_t>(grp)) continue;
+      const bool diag = t.j == t.qt;
+      if (!(ok = warp_wait(bar(Cf::SF0 + grp), (g >> 1) & 1, ctl))) break;
+      tc_fence_after();
+      // pass 1: block maxima (loops over halves are kept rolled: a compact hot
+      // loop keeps the instruction cache warm for the 15 warps of the CTA)
+      float bmx0 = 0.0f, bmx1 = 0.0f;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[64];
+        tmem_ld32p(ts + 64 * h, &r[0]);
+        tmem_ld32p(ts + 64 * h + 32, &r[32]);
+        tmem_wait_ld();
+        if (diag) {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (64 * half + c > row) r[c] = 0xff800000u;   // -inf: key after the query row
+            if (64 * h + c > row) r[c] = 0xff800000u;   // -inf: key after the query row
         }
         const float bm = max64(r);
-        xch_s[(buf * 2 + half) * 128 + row] = bm;
-        mbar_arrive(bar(Cf::XC0 + buf));
-        if (!(ok = warp_wait(bar(Cf::XC0 + buf), (kv_it >> 1) & 1, ctl))) break;
-        const float bo = xch_s[(buf * 2 + (half ^ 1)) * 128 + row];
-        float alpha = 1.0f;
+        if (h == 0) bmx0 = bm; else bmx1 = bm;
+      }
+      // running max of the previous tile, from the other group (every tile
+      // waits for it, so the exchange buffers are never reused early)
+      float m_prev = __int_as_float(0xff800000);
+      if (g >= 1) {
+        const uint32_t pb = (g - 1) & 1;
+        if (!(ok = warp_wait(bar(Cf::MX0 + pb), ((g - 1) >> 1) & 1, ctl))) break;
+        if (t.j > 0) m_prev = xch_s[pb * 128 + row];
+      }
+      float m, alpha = 1.0f;
+      if (FP8) {
+        // Lean P against the running max after this tile
+        m = max3f(m_prev, bmx0, bmx1);
+        if (t.j > 0 && m > m_prev) alpha = ex2_approx(__fmul_rn(__fmul_rn(m_prev - m, A), 0.125f));
+      } else {
+        const float tmax = fmaxf(bmx0, bmx1);
+        if (t.j == 0) {
+          m = tmax;
+        } else if (__fmul_rn(tmax - m_prev, A) > kBf16RescaleLog2) {
+          alpha = ex2_approx(__fmul_rn(m_prev - tmax, A));
+          m = tmax;
+        } else {
+          m = m_prev;
+        }
+      }
+      xch_s[grp * 128 + row] = m;
+      mbar_arrive(bar(Cf::MX0 + grp));
+      // P V of tile g-2 has read this P buffer (and its scale factors)
+      if (g >= 2 && !(ok = warp_wait(bar(Cf::PE0 + grp), ((g >> 1) - 1) & 1, ctl))) break;
+      // pass 2: probabilities
+      float rowsum = 0.0f;
+      uint32_t sfw = 0;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[64];
+        tmem_ld32p(ts + 64 * h, &r[0]);
+        tmem_ld32p(ts + 64 * h + 32, &r[32]);
+        tmem_wait_ld();
+        if (diag) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (64 * h + c > row) r[c] = 0xff800000u;
+        }
         if (FP8) {
-          // Lean P against the running max after this tile
-          const float m_new = max3f(m, bm, bo);
-          if (j > 0 && m_new > m) alpha = ex2_approx(__fmul_rn(__fmul_rn(m - m_new, A), 0.125f));
-          m = m_new;
-          const int jb = leanp_block_shift(m, bm, A);
+          const int jb = leanp_block_shift(m, h ? bmx1 : bmx0, A);
           const float Bb = leanp_row_offset(m, A, jb);
           const float a256 = __fmul_rn(A, 0.00390625f), b256 = __fmul_rn(Bb, 0.00390625f);
           uint32_t p[16];
@@ -523,27 +565,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
                                    leanp_code_word(__uint_as_float(r[4 * w + 1]), a256, b256),
                                    leanp_code_word(__uint_as_float(r[4 * w + 2]), a256, b256),
                                    leanp_code_word(__uint_as_float(r[4 * w + 3]), a256, b256));
-          // P V of tile kv_it-2 has read this P buffer and its scale factors
-          if (kv_it >= 2 && !(ok = warp_wait(bar(Cf::PE0 + buf), ((kv_it >> 1) - 1) & 1, ctl))) break;
-          tmem_st16p(lb + (buf ? Cf::TP1 : Cf::TP0) + 16 * half, p);
+          tmem_st16p(tp + 16 * h, p);
           // E8M0 scale code 127 - j for both 32-key MX blocks of this 64-key block
-          sf_h[buf * 256] = static_cast<uint16_t>((127 - jb) * 0x0101);
-          fence_proxy_async_smem();   // the copy to TMEM reads it through the async proxy
+          sfw |= static_cast<uint32_t>((127 - jb) * 0x0101) << (16 * h);
         } else {
-          const float tmax = fmaxf(bm, bo);
-          if (j == 0) {
-            m = tmax;
-          } else if (__fmul_rn(tmax - m, A) > kBf16RescaleLog2) {
-            alpha = ex2_approx(__fmul_rn(m - tmax, A));
-            m = tmax;
-          }
           const float mc = m * A;
           float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          const uint32_t tp = lb + (buf ? Cf::TP1 : Cf::TP0) + 32 * half;
-          // P V of tile kv_it-2 has read this P buffer
-          if (kv_it >= 2 && !(ok = warp_wait(bar(Cf::PE0 + buf), ((kv_it >> 1) - 1) & 1, ctl))) break;
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {   // four chunks of 16 keys keep register pressure down
+          for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t pb[8];
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
@@ -552,16 +581,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
               acc[w & 3] += p0 + p1;
               pb[w] = pack_bf16x2(p0, p1);
             }
-            tmem_st8p(tp + 8 * c4, pb);
+            tmem_st8p(tp + 32 * h + 8 * c4, pb);
           }
-          l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-          if (j == nkv - 1) lfin_s[(buf * 2 + half) * 128 + row] = l;
+          rowsum += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
-        if (half == 0) alpha_s[buf * 128 + row] = alpha;
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(Cf::PF0 + buf));
       }
+      tc_fence_before();
+      mbar_arrive(bar(Cf::SC0 + grp));   // S buffer free for the tile after next
+      if (FP8) {
+        *sf_w = sfw;
+        fence_proxy_async_smem();   // the copy to TMEM reads it through the async proxy
+      } else {
+        // this group's partial row sum, kept relative to the newest max
+        l = l * ex2_approx(__fmul_rn(m_own - m, A)) + rowsum;
+        m_own = m;
+        if (t.j >= t.nkv - 2) {   // this group's last tile of the unit: hand over (l, m)
+          lfin_s[grp * 128 + row] = l;
+          xch_s[(2 + grp) * 128 + row] = m_own;
+        }
+      }
+      alpha_s[grp * 128 + row] = alpha;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(Cf::PF0 + grp));
     }
   } else {
     // ------------------------------------------------------------ correction warpgroup
@@ -572,12 +614,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     bool ok = true;
     while (ok && units.next(b, hkv, hq, qt)) {
       const int nkv = qt + 1;
-      float l_final = 1.0f;
+      // BF16: each softmax group hands over its partial row sum and the max it
+      // is relative to at its last tile of the unit (one of the last two)
+      float lg0 = 0.0f, lg1 = 0.0f, mg0 = 0.0f, mg1 = 0.0f;
       for (int j = 0; j < nkv; ++j, ++kv_it) {
         const uint32_t buf = kv_it & 1;
         if (!(ok = warp_wait(bar(Cf::PF0 + buf), (kv_it >> 1) & 1, ctl))) break;
         const float alpha = alpha_s[buf * 128 + row];
-        if (!FP8 && j == nkv - 1) l_final = lfin_s[(buf * 2) * 128 + row] + lfin_s[(buf * 2 + 1) * 128 + row];
+        if (!FP8 && j >= nkv - 2) {
+          const float lv = lfin_s[buf * 128 + row], mv = xch_s[(2 + buf) * 128 + row];
+          if (buf) { lg1 = lv; mg1 = mv; } else { lg0 = lv; mg0 = mv; }
+        }
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
           // O holds tiles 0..j-1: wait for P V of tile j-1, then scale the rows
           const uint32_t pg = kv_it - 1;
@@ -613,7 +660,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         tmem_wait_ld();
         inv = vsc / lv;
       } else {
-        inv = 1.0f / l_final;
+        // the group of the unit's last tile holds the final max
+        const bool last1 = ((kv_it - 1) & 1) != 0;
+        const float l_last = last1 ? lg1 : lg0, m_last = last1 ? mg1 : mg0;
+        const float l_oth = last1 ? lg0 : lg1, m_oth = last1 ? mg0 : mg1;
+        float lt = l_last;
+        if (nkv >= 2) lt += l_oth * ex2_approx(__fmul_rn(m_oth - m_last, a.C));
+        inv = 1.0f / lt;
       }
       const int grow = qt * 128 + row;
       __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.S + grow) * a.Hq + hq) * 128;

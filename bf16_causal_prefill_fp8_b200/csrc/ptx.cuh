@@ -52,16 +52,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// Test for completion of phase `parity`; a waiting thread is suspended in
-// hardware (it issues nothing) until the phase completes or about 0.5 ms pass.
+// Test for completion of phase `parity`; a waiting thread may be suspended
+// in hardware for a system-dependent time before the test gives up.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(500000u)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -90,11 +90,11 @@ struct WaitCtl {
 // kDevWaitTimeout in the device error word, raises the CTA's abort flag and
 // returns false.  Never traps and never spins without a limit.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
-  if (mbar_test_wait(bar, parity)) return true;   // fast path: phase already complete
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 3u) == 0u) {
+    if ((it & 63u) == 0u) {
       if (*ctl.abort_flag) return false;
       if (globaltimer_ns() - t0 > ctl.timeout_ns) {
         atomicExch(&g_device_status, kDevWaitTimeout);
