@@ -27,7 +27,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from bf16_causal_prefill_fp8_b200 import synth  # noqa: E402
+from bf16_causal_prefill_fp8_b200 import shard, synth  # noqa: E402
 
 METRIC = "causal prefill attn TFLOP/s (FP8 e4m3 & BF16, D=128, S=16K) and % of B200 peak"
 DEFAULT_WORKLOAD = "gqa32x8_s16k_outlier"
@@ -48,7 +48,7 @@ def load_peaks():
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
     FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -60,7 +60,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
@@ -224,7 +224,7 @@ def run_ours(args, wl):
     peaks, peak_src = load_peaks()
 
     # inputs: seeded per rank (each rank holds its own independent shard)
-    q, k, v = synth.make_qkv(args.seed + 1000 * rank, B, S, Hq, Hkv, Dqk, Dv, wl["kind"])
+    q, k, v = synth.make_qkv(shard.rank_seed(args.seed, rank), B, S, Hq, Hkv, Dqk, Dv, wl["kind"])
     qb, kb, vb = (torch.from_numpy(x).to(torch.bfloat16) for x in (q, k, v))
     dq, dk, dv = (t.to(dev) for t in (qb, kb, vb))
     cq = torch.empty(dq.shape, dtype=torch.uint8, device=dev)
@@ -269,11 +269,7 @@ def run_ours(args, wl):
         return per
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return shard.max_over_ranks(x, device=dev)
 
     # warm-up
     for _ in range(args.warmup):
@@ -400,13 +396,25 @@ def run_ours(args, wl):
     return 0
 
 
+KERNEL_SOURCES = ("attn_fwd.cuh", "leanp.cuh", "ptx.cuh")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "bf16_causal_prefill_fp8_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
 def load_traffic(workload):
-    """DRAM bytes per attention launch from the committed ncu summary, if any."""
+    """DRAM bytes per attention launch from the committed ncu summary; null
+    once the kernel sources differ from the ones the counters were taken on."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(p):
         d = json.load(open(p))
         e = d.get(workload)
-        if e and e.get("valid", True):
+        if e and e.get("source_sha256") == kernel_source_hash():
             return e.get("bytes_per_launch")
     return None
 
