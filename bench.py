@@ -142,6 +142,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--hadamard", action="store_true",
+                    help="rotate Q and K by the 128-point Hadamard transform in the prepass (D = 128)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = dict(synth.WORKLOADS[args.workload])
@@ -239,8 +241,8 @@ def run_ours(args, wl):
     stream = torch.cuda.current_stream()
 
     def prepass():
-        zyfa.quantize(dq, out=cq, scale=sq)
-        zyfa.quantize(dk, out=ck, scale=sk)
+        zyfa.quantize(dq, hadamard=args.hadamard, out=cq, scale=sq)
+        zyfa.quantize(dk, hadamard=args.hadamard, out=ck, scale=sk)
         zyfa.quantize(dv, out=cv, scale=sv)
 
     def attn8():
@@ -340,7 +342,7 @@ def run_ours(args, wl):
     if world == 1:
         from oracle import oracle as orc
         bfv = lambda t: t.float().numpy()
-        codes = oracle_inputs(wl, args.seed, bfv(qb), bfv(kb), bfv(vb))
+        codes = oracle_inputs(wl, args.seed, bfv(qb), bfv(kb), bfv(vb), hadamard=args.hadamard)
         gpu_codes_equal = all(np.array_equal(g.cpu().numpy(), c) for g, (c, _) in zip((cq, ck, cv), codes))
         rows = sample_rows(S, 96 if S >= 8192 else 256)
         o_ref, dt, cores = time_oracle_rows(wl, codes, rows)
@@ -365,7 +367,8 @@ def run_ours(args, wl):
         "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
         "config": {"workload": args.workload, "B": B, "S": S, "Hq": Hq, "Hkv": Hkv, "Dqk": Dqk, "Dv": Dv,
                    "inputs": wl["kind"] + ", seeded, bf16 in HBM", "global_batch": B * world, "seq_len": S,
-                   "step": "quantize Q,K,V (bf16 -> e4m3, per-head scale) + FP8 Lean-P causal attention",
+                   "step": "quantize Q,K,V (bf16 -> e4m3, per-head scale" + (", Hadamard Q/K" if args.hadamard else "")
+                           + ") + FP8 Lean-P causal attention",
                    "l2": "flushed before every timed step (256 MiB write, untimed)",
                    "parallelism": f"dp{world} (independent shards, no collective)"},
         "roofline": {"bound": "tensor", "achieved": ach8, "peak": fp8_peak, "unit": "TFLOP/s",

@@ -4,9 +4,11 @@
 // Method: kongchang.com "Zyphra ZYFA", section "ZYFA 的性能与精度数据" (per-head
 // scale factors map values into the e4m3 range) and spke.com "Zyphra ZYFA",
 // accuracy section (quantizing Q, K and V is the main FP8 error source; a
-// Hadamard rotation of Q and K roughly halves it).  HBM-bound: each kernel
-// streams the tensor once with 16-byte vector loads; a CTA covers whole
-// sequence rows of one batch.
+// Hadamard rotation of Q and K roughly halves it).
+//
+// HBM-bound streaming passes.  A CTA covers whole sequence rows of one batch;
+// every thread keeps kUnroll 16-byte loads in flight (the bytes in flight,
+// not arithmetic, bound these kernels).
 //
 // Steps (all on `stream`):
 //   1. memset(scale, 0)                         scale doubles as amax accumulator
@@ -24,6 +26,7 @@
 namespace zyfa {
 
 constexpr int kQuantThreads = 256;
+constexpr int kUnroll = 4;
 constexpr float kFwhtNorm = 0.08838834764831844055f;   // 2^-3.5 rounded to fp32
 
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
@@ -36,17 +39,36 @@ __device__ __forceinline__ float head_scale(float amax) {
   return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// Load 4 consecutive elements as fp32.
+// 16-byte vectors: 8 bf16 or 4 fp32 elements.
+template <typename T> struct Vec;
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void unpack(const uint4& t, float* v) {
+    v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xffff0000u);
+    v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xffff0000u);
+    v[4] = __uint_as_float(t.z << 16); v[5] = __uint_as_float(t.z & 0xffff0000u);
+    v[6] = __uint_as_float(t.w << 16); v[7] = __uint_as_float(t.w & 0xffff0000u);
+  }
+};
+template <> struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void unpack(const uint4& t, float* v) {
+    v[0] = __uint_as_float(t.x); v[1] = __uint_as_float(t.y);
+    v[2] = __uint_as_float(t.z); v[3] = __uint_as_float(t.w);
+  }
+};
+
+// Load 4 consecutive elements as fp32 (Hadamard path: lane l holds 4l .. 4l+3).
 template <typename T>
 __device__ __forceinline__ void load4(const T* p, float (&v)[4]);
 template <>
 __device__ __forceinline__ void load4<float>(const float* p, float (&v)[4]) {
-  const float4 t = *reinterpret_cast<const float4*>(p);
+  const float4 t = __ldg(reinterpret_cast<const float4*>(p));
   v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
 }
 template <>
 __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[4]) {
-  const uint2 t = *reinterpret_cast<const uint2*>(p);
+  const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
   v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xffff0000u);
   v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xffff0000u);
 }
@@ -90,28 +112,49 @@ __global__ void __launch_bounds__(kQuantThreads) quant_amax_kernel(QuantArgs a) 
   const int r0 = blockIdx.x * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
   for (int h = threadIdx.x; h < a.H; h += blockDim.x) s_amax[h] = 0u;
   __syncthreads();
-  const size_t HD = static_cast<size_t>(a.H) * a.D;
+  const uint32_t HD = static_cast<uint32_t>(a.H) * a.D;
   const T* base = static_cast<const T*>(a.x) + (static_cast<size_t>(b) * a.S + r0) * HD;
   if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int nvec = (r1 - r0) * a.H;          // 128-element rows
-    for (int vi = warp; vi < nvec; vi += nw) {
-      float x[4];
-      load4<T>(base + static_cast<size_t>(vi) * 128 + 4 * lane, x);
-      fwht128_warp(x, lane);
-      float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+    for (int v0 = warp * kUnroll; v0 < nvec; v0 += nw * kUnroll) {
+      float x[kUnroll][4];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (lane == 0) atomicMax(&s_amax[vi % a.H], __float_as_uint(mx));
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + u < nvec) load4<T>(base + static_cast<size_t>(v0 + u) * 128 + 4 * lane, x[u]);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + u >= nvec) break;
+        fwht128_warp(x[u], lane);
+        float mx = fmaxf(fmaxf(fabsf(x[u][0]), fabsf(x[u][1])), fmaxf(fabsf(x[u][2]), fabsf(x[u][3])));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) atomicMax(&s_amax[(v0 + u) % a.H], __float_as_uint(mx));
+      }
     }
   } else {
-    const size_t n4 = (static_cast<size_t>(r1 - r0) * HD) / 4;
-    for (size_t i = threadIdx.x; i < n4; i += blockDim.x) {
-      float x[4];
-      load4<T>(base + 4 * i, x);
-      const float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-      const int h = static_cast<int>(((4 * i) % HD) / a.D);
-      atomicMax(&s_amax[h], __float_as_uint(mx));
+    constexpr int N = Vec<T>::N;
+    const uint32_t vpr = HD / N, vph = a.D / N;        // 16-byte vectors per row / per head
+    const uint32_t nvec = static_cast<uint32_t>(r1 - r0) * vpr;
+    const uint4* src = reinterpret_cast<const uint4*>(base);
+    for (uint32_t v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * kUnroll) {
+      uint4 raw[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t vi = v0 + u * blockDim.x;
+        if (vi < nvec) raw[u] = __ldg(src + vi);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t vi = v0 + u * blockDim.x;
+        if (vi >= nvec) break;
+        float x[N];
+        Vec<T>::unpack(raw[u], x);
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < N; ++i) mx = fmaxf(mx, fabsf(x[i]));
+        atomicMax(&s_amax[(vi % vpr) / vph], __float_as_uint(mx));
+      }
     }
   }
   __syncthreads();
@@ -128,31 +171,55 @@ __global__ void __launch_bounds__(kQuantThreads) quant_codes_kernel(QuantArgs a)
   for (int h = threadIdx.x; h < a.H; h += blockDim.x)
     s_sc[h] = head_scale(a.scale[static_cast<size_t>(b) * a.H + h]);
   __syncthreads();
-  const size_t HD = static_cast<size_t>(a.H) * a.D;
+  const uint32_t HD = static_cast<uint32_t>(a.H) * a.D;
   const size_t off = (static_cast<size_t>(b) * a.S + r0) * HD;
   const T* base = static_cast<const T*>(a.x) + off;
   uint8_t* obase = a.out + off;
   if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int nvec = (r1 - r0) * a.H;
-    for (int vi = warp; vi < nvec; vi += nw) {
-      float x[4];
-      load4<T>(base + static_cast<size_t>(vi) * 128 + 4 * lane, x);
-      fwht128_warp(x, lane);
-      const float sc = s_sc[vi % a.H];
-      const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[0], sc), __fdiv_rn(x[1], sc));
-      const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[2], sc), __fdiv_rn(x[3], sc));
-      *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(vi) * 128 + 4 * lane) = lo | (hi << 16);
+    for (int v0 = warp * kUnroll; v0 < nvec; v0 += nw * kUnroll) {
+      float x[kUnroll][4];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + u < nvec) load4<T>(base + static_cast<size_t>(v0 + u) * 128 + 4 * lane, x[u]);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + u >= nvec) break;
+        fwht128_warp(x[u], lane);
+        const float sc = s_sc[(v0 + u) % a.H];
+        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[u][0], sc), __fdiv_rn(x[u][1], sc));
+        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[u][2], sc), __fdiv_rn(x[u][3], sc));
+        *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(v0 + u) * 128 + 4 * lane) = lo | (hi << 16);
+      }
     }
   } else {
-    const size_t n4 = (static_cast<size_t>(r1 - r0) * HD) / 4;
-    for (size_t i = threadIdx.x; i < n4; i += blockDim.x) {
-      float x[4];
-      load4<T>(base + 4 * i, x);
-      const float sc = s_sc[((4 * i) % HD) / a.D];
-      const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[0], sc), __fdiv_rn(x[1], sc));
-      const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[2], sc), __fdiv_rn(x[3], sc));
-      *reinterpret_cast<uint32_t*>(obase + 4 * i) = lo | (hi << 16);
+    constexpr int N = Vec<T>::N;
+    const uint32_t vpr = HD / N, vph = a.D / N;
+    const uint32_t nvec = static_cast<uint32_t>(r1 - r0) * vpr;
+    const uint4* src = reinterpret_cast<const uint4*>(base);
+    for (uint32_t v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * kUnroll) {
+      uint4 raw[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t vi = v0 + u * blockDim.x;
+        if (vi < nvec) raw[u] = __ldg(src + vi);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t vi = v0 + u * blockDim.x;
+        if (vi >= nvec) break;
+        float x[N];
+        Vec<T>::unpack(raw[u], x);
+        const float sc = s_sc[(vi % vpr) / vph];
+        uint32_t w[N / 4];
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i)
+          w[i] = cvt_e4m3x2(__fdiv_rn(x[4 * i], sc), __fdiv_rn(x[4 * i + 1], sc)) |
+                 (static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(x[4 * i + 2], sc), __fdiv_rn(x[4 * i + 3], sc))) << 16);
+        if constexpr (N == 8) *reinterpret_cast<uint2*>(obase + static_cast<size_t>(vi) * 8) = make_uint2(w[0], w[1]);
+        else *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(vi) * 4) = w[0];
+      }
     }
   }
 }
