@@ -36,7 +36,9 @@
  *       normal codes; largest code of a block in (112, 120].
  *   oracle_fp8_model_rows : with exact_p = 1 equals oracle_attention_rows on
  *       the dequantized inputs to 1e-6 (pins tile order, running max, the
- *       rescale factor and the row sum); Q = 0 gives prefix means exactly.
+ *       rescale factor and the row sum), also with the deferred reference max
+ *       on scores that grow by many binades across the keys; Q = 0 gives
+ *       prefix means exactly.
  * No function here is "parity unpinned".
  */
 #include <math.h>
@@ -289,9 +291,18 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 /*   s_j   = fl32(sum_d value(qcode) * value(kcode))   keys j <= i, j < S    */
 /*   bmax  = max s_j over each block (-inf if the block has no live key)    */
 /*   m'    = max(m, bmax_0, bmax_1)          running max after this tile    */
+/*           (rescale_log2 > 0: reference max instead -- m' = tile max on    */
+/*           tile 0; later m' = max(bmax_0, bmax_1) only when               */
+/*           fl32(fl32(that - m) * A) > 8 rescale_log2, i.e. when the tile  */
+/*           max is more than rescale_log2 binades above m, else m' = m.    */
+/*           The softmax is unchanged: O and l share the reference and the */
+/*           per-block shift j renormalises each block to its own max.)     */
 /*   w_j   = value(leanp code) * 2^-j_block  (exact_p: exp2((s_j-m')A/8))   */
 /*   alpha = exp2((m - m') A / 8)            (0 on the first tile)          */
 /*   O     = alpha O + sum_j w_j value(vcode_j);  l = alpha l + sum_j w_j   */
+/* Every block shift j must stay >= 0 (weights <= 448, E8M0 scale <= 1):   */
+/* true for the exact max (j >= 8) and for the deferred one (j >= 8 - r);   */
+/* a violation returns -2.                                                  */
 /* The row sum l comes from the rounded weights, like the extra matrix      */
 /* instruction per block on the pages.  Output o_i = O / l * v_s.           */
 /* q [B,S,Hq,Dqk], k [B,S,Hkv,Dqk], v [B,S,Hkv,Dv] codes; q_s [B*Hq],       */
@@ -300,9 +311,10 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *vc,
                           const float *q_s, const float *k_s, const float *v_s,
                           int B, int Hq, int Hkv, int S, int Dqk, int Dv,
-                          int exact_p, const int *rows, int nrows, double *o)
+                          int exact_p, float rescale_log2,
+                          const int *rows, int nrows, double *o)
 {
-    int b;
+    int b, shift_err = 0;
     if (!qc || !kc || !vc || !q_s || !k_s || !v_s || !o) return -1;
     if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Hq % Hkv != 0 || Dqk < 1 || Dv < 1) return -1;
     if (!rows) nrows = S;
@@ -339,9 +351,26 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
                         if (sj[n] > bmax[n / 64]) bmax[n / 64] = sj[n];
                     }
                 }
-                mnew = m;
-                if (bmax[0] > mnew) mnew = bmax[0];
-                if (bmax[1] > mnew) mnew = bmax[1];
+                if (rescale_log2 > 0.0f) {
+                    float tmax = bmax[0] > bmax[1] ? bmax[0] : bmax[1];
+                    float grow;
+                    if (t == 0) {
+                        mnew = tmax;
+                    } else {
+                        grow = tmax - m;
+                        grow = grow * A;
+                        mnew = (grow > 8.0f * rescale_log2) ? tmax : m;
+                    }
+                } else {
+                    mnew = m;
+                    if (bmax[0] > mnew) mnew = bmax[0];
+                    if (bmax[1] > mnew) mnew = bmax[1];
+                }
+                for (n = 0; n < 2; ++n)
+                    if (oracle_leanp_block_shift(mnew, bmax[n], A) < 0) {
+#pragma omp atomic write
+                        shift_err = 1;
+                    }
                 alpha = (t == 0) ? 0.0 : exp2(((double)m - (double)mnew) * (double)A / 8.0);
                 l *= alpha;
                 for (d = 0; d < Dv; ++d) acc[d] *= alpha;
@@ -370,7 +399,7 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
             free(acc);
         }
     }
-    return 0;
+    return shift_err ? -2 : 0;
 }
 
 /* Number of OpenMP threads the oracle runs with (1 without OpenMP). */

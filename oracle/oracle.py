@@ -42,7 +42,7 @@ def lib():
         L.oracle_leanp_batch.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i, c_p, c_p]
         L.oracle_fp8_model_rows.restype = c_i
         L.oracle_fp8_model_rows.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i,
-                                            c_i, c_i, c_i, c_p, c_i, c_p]
+                                            c_i, c_i, c_i, c_f, c_p, c_i, c_p]
         L.oracle_num_threads.restype = c_i
         L.oracle_num_threads.argtypes = []
         _lib = L
@@ -155,9 +155,11 @@ def leanp_batch(s, m, bmax, A, masked=None):
     return code, j
 
 
-def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None) -> np.ndarray:
+def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=0.0) -> np.ndarray:
     """The FP8 pipeline replayed on the CPU (see oracle.c).  Codes uint8 BSHD,
-    scales fp32 [B,H].  Returns o fp64 [B, S or len(rows), Hq, Dv]."""
+    scales fp32 [B,H].  rescale_log2 = 0: exact running max; > 0: the reference
+    max moves only when a tile max exceeds it by more than that many binades.
+    Returns o fp64 [B, S or len(rows), Hq, Dv]."""
     qc = _c(qc, np.uint8); kc = _c(kc, np.uint8); vc = _c(vc, np.uint8)
     q_s = _c(q_s, np.float32); k_s = _c(k_s, np.float32); v_s = _c(v_s, np.float32)
     B, S, Hq, Dqk = qc.shape
@@ -166,7 +168,9 @@ def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None) -> np.ndarray
     n = S if rows is None else len(r)
     o = np.empty((B, n, Hq, Dv), dtype=np.float64)
     rc = lib().oracle_fp8_model_rows(_ptr(qc), _ptr(kc), _ptr(vc), _ptr(q_s), _ptr(k_s), _ptr(v_s),
-                                     B, Hq, Hkv, S, Dqk, Dv, int(bool(exact_p)), _ptr(r), n, _ptr(o))
+                                     B, Hq, Hkv, S, Dqk, Dv, int(bool(exact_p)), ctypes.c_float(rescale_log2), _ptr(r), n, _ptr(o))
+    if rc == -2:
+        raise ArithmeticError("oracle_fp8_model_rows: a block shift fell below 0 (reference max too stale)")
     if rc != 0:
         raise ValueError("oracle_fp8_model_rows: bad arguments")
     return o

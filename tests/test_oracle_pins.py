@@ -271,6 +271,44 @@ def test_model_oracle_exact_p_equals_plain_definition():
     assert orc.rel_fro(o_model, o_ref) < 1e-6
 
 
+def _growing_score_case(seed):
+    """Q = 1.0 everywhere, K rows near a per-tile level, so the score of key j
+    for every query is about 128 * level(tile of j): levels chosen so that the
+    tile max jumps by ~20 binades, then ~4 (below an 8-binade threshold),
+    falls, then ~8.2 above the deferred reference (scores in binades:
+    s * 8 log2(e) / sqrt(128) / 8)."""
+    rng = np.random.default_rng(seed)
+    vals = orc.e4m3_values()
+    code_of = {float(vals[c]): c for c in range(0x00, 0x7F)}
+    levels = [0.5, 1.75, 2.0, 1.5, 2.25]
+    S, D = 128 * len(levels), 128
+    qc = np.full((1, S, 1, D), code_of[1.0], dtype=np.uint8)
+    kc = np.empty((1, S, 1, D), dtype=np.uint8)
+    for t, lv in enumerate(levels):
+        c = code_of[lv]
+        kc[0, 128 * t:128 * (t + 1), 0, :] = c - rng.integers(0, 2, size=(128, D))  # lv or next lower
+    vc = rng.integers(0x20, 0x50, size=(1, S, 1, D), dtype=np.uint8)
+    vc |= (rng.integers(0, 2, size=vc.shape) << 7).astype(np.uint8)              # random signs
+    one = np.ones((1, 1), dtype=np.float32)
+    return qc, kc, vc, one, one, one
+
+
+def test_model_oracle_deferred_max_equals_plain_definition():
+    """With exact probabilities the deferred reference max (8 binades) must give
+    the plain softmax: pins the deferral rule, its alpha and that O and l are
+    rescaled together, on scores that grow far beyond the fp32 exp2 range."""
+    qc, kc, vc, qs, ks, vs = _growing_score_case(21)
+    deq = tuple(orc.dequantize(x, sc) for x, sc in ((qc, qs), (kc, ks), (vc, vs)))
+    ref = orc.attention(*deq)
+    o_lazy = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True, rescale_log2=8.0)
+    assert orc.rel_fro(o_lazy, ref) < 1e-6
+    # the deferral changes the Lean-P codes (the reference moves), not the bar
+    o_exact = orc.fp8_model(qc, kc, vc, qs, ks, vs)
+    o_def = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=8.0)
+    assert not np.array_equal(o_exact, o_def)
+    assert orc.rel_fro(o_def, ref) < 3e-2 and orc.rel_fro(o_exact, ref) < 3e-2
+
+
 def test_model_oracle_zero_q_gives_prefix_means():
     codes, deq, _ = _quantized_case(13, 1, 200, 2, 2, 128)
     qc, kc, vc, qs, ks, vs = codes
