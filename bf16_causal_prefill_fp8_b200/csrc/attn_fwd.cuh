@@ -17,10 +17,11 @@
 // per SIMD, ping-pong).  Blackwell tracks MMA completion in hardware, so the
 // overlap here is warp specialisation with mbarrier hand-offs.  CTA = 480
 // threads, one per SM (persistent grid):
-//   warps 0-7   softmax: warp w owns rows 32(w%4) .. 32(w%4)+31 of the tile
-//               (TMEM lane quarter w%4) and the 64-key block w/4 of each key
-//               tile; running max (block maxima exchanged between the two
-//               warps of a quarter), P (Lean-P codes or bf16), rescale factor
+//   warps 0-7   softmax, two warpgroups taking alternate KV tiles
+//               (ping-pong): warp w owns rows 32(w%4) .. 32(w%4)+31 of the
+//               tile (TMEM lane quarter w%4), all 128 keys; reference max
+//               (handed from group to group), P (Lean-P codes or bf16),
+//               rescale factor
 //   warps 8-11  correction: rescales O (and the FP8 row sum) when the running
 //               max grew, then the epilogue O / l -> bf16 -> global
 //   warp 12     TMA producer (one elected thread): Q tile per unit, K/V ring
@@ -61,10 +62,14 @@ struct AttnArgs {
 };
 
 constexpr int kAttnThreads = 480;
-// BF16 only: the reference max of the exp2 is refreshed when the running max
-// exceeds it by more than this many binades (FlashAttention-4's lazy rescale;
-// the result is the same softmax, the O rescale becomes rare).
-constexpr float kBf16RescaleLog2 = 8.0f;
+// Deferred reference max (both paths): the max that the probabilities are
+// taken against moves only when a tile's max exceeds it by more than this
+// many binades (FlashAttention-4's lazy rescale).  O and the row sum always
+// share the reference, so the softmax is unchanged and the O rescale, which
+// serialises P V behind the previous tile, becomes rare.  FP8: the 64-key
+// block shift j renormalises every block to its own max, so the codes keep
+// their precision and j stays >= 8 - kRescaleLog2 >= 0.
+constexpr float kRescaleLog2 = 8.0f;
 
 template <bool FP8, int DQK>
 struct AttnCfg {
@@ -520,21 +525,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         if (!(ok = warp_wait(bar(Cf::MX0 + pb), ((g - 1) >> 1) & 1, ctl))) break;
         if (t.j > 0) m_prev = xch_s[pb * 128 + row];
       }
+      // reference max after this tile (FP8: A carries a factor 8)
       float m, alpha = 1.0f;
-      if (FP8) {
-        // Lean P against the running max after this tile
-        m = max3f(m_prev, bmx0, bmx1);
-        if (t.j > 0 && m > m_prev) alpha = ex2_approx(__fmul_rn(__fmul_rn(m_prev - m, A), 0.125f));
+      const float tmax = fmaxf(bmx0, bmx1);
+      if (t.j == 0) {
+        m = tmax;
+      } else if (__fmul_rn(tmax - m_prev, A) > (FP8 ? 8.0f * kRescaleLog2 : kRescaleLog2)) {
+        alpha = ex2_approx(FP8 ? __fmul_rn(__fmul_rn(m_prev - tmax, A), 0.125f)
+                               : __fmul_rn(m_prev - tmax, A));
+        m = tmax;
       } else {
-        const float tmax = fmaxf(bmx0, bmx1);
-        if (t.j == 0) {
-          m = tmax;
-        } else if (__fmul_rn(tmax - m_prev, A) > kBf16RescaleLog2) {
-          alpha = ex2_approx(__fmul_rn(m_prev - tmax, A));
-          m = tmax;
-        } else {
-          m = m_prev;
-        }
+        m = m_prev;
       }
       xch_s[grp * 128 + row] = m;
       mbar_arrive(bar(Cf::MX0 + grp));

@@ -19,6 +19,9 @@ TOL_FP8 = 3e-2
 # 4.0e-3 on the outlier-K case).  A layout or scale bug in the kernel moves
 # the error to >= 1e-1, far above this budget.
 TOL_FP8_MODEL = 8e-3
+# The kernel's deferred reference max: it moves when a tile's max exceeds it
+# by more than this many binades (the CPU replay takes the same rule).
+RESCALE_LOG2 = 8.0
 
 
 def bf16_round(x: np.ndarray) -> torch.Tensor:
@@ -69,5 +72,5 @@ def fp8_references(codes, rows=None):
     (qc, qs), (kc, ks), (vc, vs) = codes
     deq = (orc.dequantize(qc, qs), orc.dequantize(kc, ks), orc.dequantize(vc, vs))
     ref = orc.attention(*deq, rows=rows)
-    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rows=rows)
+    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rows=rows, rescale_log2=RESCALE_LOG2)
     return ref, model

@@ -69,6 +69,57 @@ def test_fp8_block_scales_engaged(q_gain, kind):
     assert e_ref <= TOL_FP8
 
 
+def test_deferred_reference_max_on_growing_scores():
+    """Scores that jump by ~20 binades, then ~4 (deferred), fall, then ~8.2
+    above the stale reference (rescaled): FP8 against fp64 attention and the
+    CPU replay with the same deferral rule; BF16 on the same values."""
+    from test_oracle_pins import _growing_score_case
+    qc, kc, vc, qs, ks, vs = _growing_score_case(21)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    o = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs))
+    torch.cuda.synchronize()
+    o = o.float().cpu().numpy().astype(np.float64)
+    ref, model = fp8_references(((qc, qs), (kc, ks), (vc, vs)))
+    e_ref, e_model = orc.rel_fro(o, ref), orc.rel_fro(o, model)
+    print(f"growing scores fp8: vs fp64 {e_ref:.3e}  vs model {e_model:.3e}")
+    assert e_ref <= TOL_FP8 and e_model <= TOL_FP8_MODEL
+    deq = [orc.dequantize(x, sc) for x, sc in ((qc, qs), (kc, ks), (vc, vs))]
+    ob = zyfa.attn_fwd(*[dev(x).to(torch.bfloat16) for x in deq])   # e4m3 values are exact in bf16
+    torch.cuda.synchronize()
+    e_b = orc.rel_fro(ob.float().cpu().numpy().astype(np.float64), ref)
+    print(f"growing scores bf16: vs fp64 {e_b:.3e}")
+    assert e_b <= TOL_BF16
+
+
+@pytest.mark.parametrize("kind,q_gain", [("outlier_k", 1.0), ("gaussian", 6.0)])
+def test_many_units_per_cta(kind, q_gain):
+    """512 work units on the persistent grid (several per CTA): unit hand-over
+    of O, the epilogue by either softmax group, Q double buffering and, with
+    peaked scores, frequent O rescales; sampled rows, FP8 and BF16, repeat
+    runs bit-identical."""
+    B, S, Hq, Hkv = 2, 2048, 16, 4
+    q, k, v = inputs(46, B, S, Hq, Hkv, 128, 128, kind=kind, q_gain=q_gain)
+    rows = np.unique(np.concatenate([np.arange(0, S, 37), np.arange(127, S, 128), np.arange(128, S, 128),
+                                     [S - 1]])).astype(np.int32)
+    o, codes = run_fp8(q, k, v)
+    ref, model = fp8_references(codes, rows=rows)
+    e_ref, e_model = orc.rel_fro(o[:, rows], ref), orc.rel_fro(o[:, rows], model)
+    print(f"many units fp8 {kind} gain={q_gain}: vs fp64 {e_ref:.3e}  vs model {e_model:.3e}")
+    assert e_ref <= TOL_FP8 and e_model <= TOL_FP8_MODEL
+    (qc, qs), (kc, ks), (vc, vs) = codes
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    o2 = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs))
+    torch.cuda.synchronize()
+    assert np.array_equal(o2.float().cpu().numpy().astype(np.float64), o)
+    ob, (qb, kb, vb) = run_bf16(q, k, v)
+    refb = orc.attention(qb, kb, vb, rows=rows)
+    e_b = orc.rel_fro(ob[:, rows], refb)
+    print(f"many units bf16 {kind} gain={q_gain}: vs fp64 {e_b:.3e}")
+    assert e_b <= TOL_BF16
+    ob2, _ = run_bf16(q, k, v)
+    assert np.array_equal(ob2, ob)
+
+
 def test_fp8_hadamard_prepass_path():
     q, k, v = inputs(44, 1, 513, 4, 4, 128, 128)
     o, codes = run_fp8(q, k, v, hadamard=True)
