@@ -83,30 +83,36 @@ struct AttnCfg {
   static constexpr int VB = 128 * 128 * EL;          // Dv = 128
   static constexpr int ST = FP8 ? 4 : 2;             // K/V ring stages
   static constexpr int QBUF = (!FP8 && DQK == 192) ? 1 : 2;   // Q tile buffers (units in flight)
+  static constexpr int NPB = FP8 ? 3 : 2;            // P buffers (tile g uses g % NPB)
   static constexpr int NK_QK = ROWB / 32;            // QK MMA K-steps of 32 bytes
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBUF * QB;
   static constexpr int OFF_V = OFF_K + ST * KB;
   static constexpr int OFF_ONES = OFF_V + ST * VB;   // FP8: 16 x 128 bytes of e4m3 1.0
-  static constexpr int OFF_SF = OFF_ONES + (FP8 ? 2048 : 0);   // FP8: 2 x 512 B scale factors
-  static constexpr int OFF_ALPHA = OFF_SF + (FP8 ? 1024 : 0);  // 2 x 128 fp32 rescale factors
-  static constexpr int OFF_LFIN = OFF_ALPHA + 1024;  // BF16 final partial row sums, per group (2 x 128 fp32, 1 KB used)
+  static constexpr int OFF_SF = OFF_ONES + (FP8 ? 2048 : 0);   // FP8: NPB x 512 B scale factors
+  static constexpr int OFF_ALPHA = OFF_SF + (FP8 ? NPB * 512 : 0);  // NPB x 128 fp32 rescale factors
+  static constexpr int OFF_LFIN = OFF_ALPHA + NPB * 512;  // BF16 final partial row sums, per group (2 x 128 fp32)
   static constexpr int OFF_XCH = OFF_LFIN + 2048;    // running max per group (2 x 128) + BF16 final max per group (2 x 128)
   static constexpr int OFF_BAR = OFF_XCH + 2048;
   // Barriers (phase bookkeeping: every waiter is at most one phase behind,
   // so a parity test cannot alias): Q full/empty per Q buffer; OF = O read
   // by the epilogue (per unit); OFIN = last P V of a unit done (per unit);
-  // per S buffer: SF = S full, SC = S read, PF = P/alpha written, PE = P V
-  // done (P buffer free, O updated), OR = O corrected, ready for P V.
-  enum { QF0 = 0, QF1, QE0, QE1, OF, OFIN, DRAIN, DRAIN2, SF0, SF1, SC0, SC1, PF0, PF1, PE0, PE1, OR0, OR1, MX0, MX1, KF };
+  // per S buffer: SF = S full, SC = S read, MX = running max published; per
+  // P buffer: PF = P/alpha written, PE = P V done (P buffer free, O
+  // updated), OR = O corrected, ready for P V.
+  enum { QF0 = 0, QF1, QE0, QE1, OF, OFIN, DRAIN, DRAIN2, SF0, SF1, SC0, SC1, PF0, PF1, PF2, PE0, PE1, PE2,
+         OR0, OR1, OR2, MX0, MX1, KF };
   static constexpr int KE = KF + ST, VF = KF + 2 * ST, VE = KF + 3 * ST;
   static constexpr int NBAR = KF + 4 * ST;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   // tensor-memory columns (512 allocated)
   static constexpr uint32_t TS0 = 0, TS1 = 128, TO = 256;
-  static constexpr uint32_t TL = 384, TSFB = 400, TSFA0 = 404, TSFA1 = 408;
-  static constexpr uint32_t TP0 = FP8 ? 448 : 384, TP1 = FP8 ? 480 : 448;
+  static constexpr uint32_t TL = 384, TSFB = 400;
+  // P buffer b: FP8 32 columns of packed codes at 416 + 32 b; BF16 64 columns
+  // of bf16 pairs at 384 + 64 b; FP8 scale factors of P buffer b at 404 + 4 b
+  static __device__ __forceinline__ uint32_t tp(uint32_t b) { return FP8 ? 416 + 32 * b : 384 + 64 * b; }
+  static __device__ __forceinline__ uint32_t tsfa(uint32_t b) { return 404 + 4 * b; }
   static constexpr uint32_t IDESC_QK = idesc_dense(FP8 ? 0 : 1, FP8 ? 0 : 1, 0, 0, 128, 128);
   static constexpr uint32_t IDESC_PV_BF16 = idesc_dense(1, 1, 0, 1, 128, 128);
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -256,8 +262,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(Cf::SF0 + i), 1);
       mbar_init(bar(Cf::SC0 + i), 128);
-      mbar_init(bar(Cf::PF0 + i), 128);
       mbar_init(bar(Cf::MX0 + i), 128);
+    }
+    for (int i = 0; i < Cf::NPB; ++i) {
+      mbar_init(bar(Cf::PF0 + i), 128);
       mbar_init(bar(Cf::PE0 + i), 1);
       mbar_init(bar(Cf::OR0 + i), 128);
     }
@@ -411,18 +419,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       return true;
     };
     auto issue_pv = [&](const TileStream& t) -> bool {
-      const uint32_t st = t.g % Cf::ST, buf = t.g & 1;
+      const uint32_t st = t.g % Cf::ST, buf = t.g % Cf::NPB, ph = (t.g / Cf::NPB) & 1;
       const bool first = t.j == 0;
       // O is free once the previous unit's epilogue has read it
       if (first && t.u > 0 && !wait1(bar(Cf::OF), (t.u - 1) & 1)) return false;
-      if (!wait1(bar(Cf::OR0 + buf), (t.g >> 1) & 1)) return false;   // P stored, O corrected
+      if (!wait1(bar(Cf::OR0 + buf), ph)) return false;   // P stored, O corrected
       if (!wait1(bar(Cf::VF + st), (t.g / Cf::ST) & 1)) return false;
       tc_fence_after();
       const uint64_t dvs = dv + ((st * Cf::VB) >> 4);
-      const uint32_t tp = tbase + (buf ? Cf::TP1 : Cf::TP0);
+      const uint32_t tp = tbase + Cf::tp(buf);
       if (leader) {
         if (FP8) {
-          const uint32_t sfa = tbase + (buf ? Cf::TSFA1 : Cf::TSFA0);
+          const uint32_t sfa = tbase + Cf::tsfa(buf);
           const uint32_t sfb = tbase + Cf::TSFB;
           // scale factors of P: 32 rows x 16 bytes in shared memory, copied to
           // all four lane quarters (the layout the block-scaled MMA reads)
@@ -478,9 +486,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       tmem_wait_st();
     }
     // scale-factor word of row r: bytes at (r % 32) * 16 + (r / 32) * 4
-    uint32_t* sf_w = sf_s + grp * 128 + ((row & 31) * 4 + (row >> 5));
+    const uint32_t sf_row = (row & 31) * 4 + (row >> 5);
     const uint32_t ts = lb + (grp ? Cf::TS1 : Cf::TS0);
-    const uint32_t tp = lb + (grp ? Cf::TP1 : Cf::TP0);
     TileStream t;
     t.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
     float A = a.C;
@@ -500,12 +507,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const bool diag = t.j == t.qt;
       if (!(ok = warp_wait(bar(Cf::SF0 + grp), (g >> 1) & 1, ctl))) break;
       tc_fence_after();
-      // pass 1: block maxima (loops over halves are kept rolled: a compact hot
-      // loop keeps the instruction cache warm for the 15 warps of the CTA)
+      // pass 1: block maxima (loops over the two 64-key blocks are kept rolled:
+      // a compact hot loop keeps the instruction cache warm for the 15 warps
+      // of the CTA).  Block 1 stays in registers for pass 2.
       float bmx0 = 0.0f, bmx1 = 0.0f;
+      uint32_t r[64];
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        uint32_t r[64];
         tmem_ld32p(ts + 64 * h, &r[0]);
         tmem_ld32p(ts + 64 * h + 32, &r[32]);
         tmem_wait_ld();
@@ -539,21 +547,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       }
       xch_s[grp * 128 + row] = m;
       mbar_arrive(bar(Cf::MX0 + grp));
-      // P V of tile g-2 has read this P buffer (and its scale factors)
-      if (g >= 2 && !(ok = warp_wait(bar(Cf::PE0 + grp), ((g >> 1) - 1) & 1, ctl))) break;
-      // pass 2: probabilities
+      // P V of tile g-NPB has read this P buffer (and its scale factors)
+      const uint32_t pbuf = g % Cf::NPB;
+      const uint32_t tp = lb + Cf::tp(pbuf);
+      if (g >= static_cast<uint32_t>(Cf::NPB) &&
+          !(ok = warp_wait(bar(Cf::PE0 + pbuf), ((g / Cf::NPB) - 1) & 1, ctl))) break;
+      // pass 2: probabilities, block 1 first (still in registers), then block
+      // 0 (read again; after that S is no longer needed and its buffer takes
+      // the tile after next)
       float rowsum = 0.0f;
       uint32_t sfw = 0;
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        uint32_t r[64];
-        tmem_ld32p(ts + 64 * h, &r[0]);
-        tmem_ld32p(ts + 64 * h + 32, &r[32]);
-        tmem_wait_ld();
-        if (diag) {
+      for (int h = 1; h >= 0; --h) {
+        if (h == 0) {
+          tmem_ld32p(ts, &r[0]);
+          tmem_ld32p(ts + 32, &r[32]);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(Cf::SC0 + grp));   // S buffer free for the tile after next
+          if (diag) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (64 * h + c > row) r[c] = 0xff800000u;
+            for (int c = 0; c < 64; ++c)
+              if (c > row) r[c] = 0xff800000u;
+          }
         }
         if (FP8) {
           const int jb = leanp_block_shift(m, h ? bmx1 : bmx0, A);
@@ -587,10 +603,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           rowsum += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(Cf::SC0 + grp));   // S buffer free for the tile after next
       if (FP8) {
-        *sf_w = sfw;
+        sf_s[pbuf * 128 + sf_row] = sfw;
         fence_proxy_async_smem();   // the copy to TMEM reads it through the async proxy
       } else {
         // this group's partial row sum, kept relative to the newest max
@@ -601,10 +615,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           xch_s[(2 + grp) * 128 + row] = m_own;
         }
       }
-      alpha_s[grp * 128 + row] = alpha;
+      alpha_s[pbuf * 128 + row] = alpha;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(Cf::PF0 + grp));
+      mbar_arrive(bar(Cf::PF0 + pbuf));
     }
   } else {
     // ------------------------------------------------------------ correction warpgroup
@@ -619,9 +633,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       // is relative to at its last tile of the unit (one of the last two)
       float lg0 = 0.0f, lg1 = 0.0f, mg0 = 0.0f, mg1 = 0.0f;
       for (int j = 0; j < nkv; ++j, ++kv_it) {
-        const uint32_t buf = kv_it & 1;
-        if (!(ok = warp_wait(bar(Cf::PF0 + buf), (kv_it >> 1) & 1, ctl))) break;
-        const float alpha = alpha_s[buf * 128 + row];
+        const uint32_t buf = kv_it & 1, pbuf = kv_it % Cf::NPB;
+        if (!(ok = warp_wait(bar(Cf::PF0 + pbuf), (kv_it / Cf::NPB) & 1, ctl))) break;
+        const float alpha = alpha_s[pbuf * 128 + row];
         if (!FP8 && j >= nkv - 2) {
           const float lv = lfin_s[buf * 128 + row], mv = xch_s[(2 + buf) * 128 + row];
           if (buf) { lg1 = lv; mg1 = mv; } else { lg0 = lv; mg0 = mv; }
@@ -629,7 +643,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
           // O holds tiles 0..j-1: wait for P V of tile j-1, then scale the rows
           const uint32_t pg = kv_it - 1;
-          if (!(ok = warp_wait(bar(Cf::PE0 + (pg & 1)), (pg >> 1) & 1, ctl))) break;
+          if (!(ok = warp_wait(bar(Cf::PE0 + pg % Cf::NPB), (pg / Cf::NPB) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -648,7 +662,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(bar(Cf::OR0 + buf));
+        mbar_arrive(bar(Cf::OR0 + pbuf));
       }
       if (!ok) break;
       // ---- epilogue: O / l (* v_scale) -> bf16, rows past S are not written
