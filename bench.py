@@ -241,9 +241,7 @@ def run_ours(args, wl):
     stream = torch.cuda.current_stream()
 
     def prepass():
-        zyfa.quantize(dq, hadamard=args.hadamard, out=cq, scale=sq)
-        zyfa.quantize(dk, hadamard=args.hadamard, out=ck, scale=sk)
-        zyfa.quantize(dv, out=cv, scale=sv)
+        zyfa.quantize_qkv(dq, dk, dv, hadamard_qk=args.hadamard, out=((cq, sq), (ck, sk), (cv, sv)))
 
     def attn8():
         zyfa.attn_fwd(cq, ck, cv, o=o8, q_scale=sq, k_scale=sk, v_scale=sv)
@@ -366,7 +364,7 @@ def run_ours(args, wl):
                "sample": f"{len(rows)} query rows x {B * Hq} heads (rows 0, S-1, tile edges, seeded random) of "
                          f"{args.workload}: fp64 causal attention on the dequantized e4m3 inputs, {dt:.1f} s"}
 
-    launches_per_fp8_step = 3 * 3 + 1      # per tensor: amax, codes, finalize; + attention
+    launches_per_fp8_step = 4 + 1          # prepass: zero, amax, codes, finalize (Q, K, V together); attention
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms8, "higher_is_better": True, "scaling": "weak",
@@ -392,7 +390,7 @@ def run_ours(args, wl):
         "fp8_breakdown_ms": {"prepass": ms8_pre, "attention": ms8_attn},
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-                "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize x3 -> zyfa_attn_fwd -> D2H O"},
+                "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize_qkv -> zyfa_attn_fwd -> D2H O"},
         "gpu_launches": args.steps * (launches_per_fp8_step + 1),
         "clocks": clk,
         "parity": parity,

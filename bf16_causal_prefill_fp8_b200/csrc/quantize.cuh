@@ -10,7 +10,8 @@
 // every thread keeps kUnroll 16-byte loads in flight (the bytes in flight,
 // not arithmetic, bound these kernels).
 //
-// Steps (all on `stream`):
+// Steps (all on `stream`; zyfa_quantize_qkv runs each step once for Q, K and
+// V together, splitting the grid among them in proportion to their bytes):
 //   1. memset(scale, 0)                         scale doubles as amax accumulator
 //   2. quant_amax_kernel:  scale[b,h] = max(scale[b,h], max |x'|)   (fp32 bits,
 //      atomicMax on the non-negative bit patterns, order-independent)
@@ -104,12 +105,10 @@ struct QuantArgs {
   int rows_per_cta;        // sequence rows of one batch per CTA
 };
 
-// Step 2.  grid = (ceil(S / rows_per_cta), B), block = kQuantThreads.
+// Step 2 for sequence-row chunk `chunk` of batch b (one CTA); s_amax: [H].
 template <typename T, bool HAD>
-__global__ void __launch_bounds__(kQuantThreads) quant_amax_kernel(QuantArgs a) {
-  extern __shared__ unsigned int s_amax[];   // [H]
-  const int b = blockIdx.y;
-  const int r0 = blockIdx.x * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
+__device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, int b, unsigned int* s_amax) {
+  const int r0 = chunk * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
   for (int h = threadIdx.x; h < a.H; h += blockDim.x) s_amax[h] = 0u;
   __syncthreads();
   const uint32_t HD = static_cast<uint32_t>(a.H) * a.D;
@@ -162,12 +161,10 @@ __global__ void __launch_bounds__(kQuantThreads) quant_amax_kernel(QuantArgs a) 
     atomicMax(reinterpret_cast<unsigned int*>(a.scale) + static_cast<size_t>(b) * a.H + h, s_amax[h]);
 }
 
-// Step 3.  Same grid; reads the finished amax of each (b, h).
+// Step 3 for one chunk; reads the finished amax of each (b, h); s_sc: [H].
 template <typename T, bool HAD>
-__global__ void __launch_bounds__(kQuantThreads) quant_codes_kernel(QuantArgs a) {
-  extern __shared__ float s_sc[];   // [H]
-  const int b = blockIdx.y;
-  const int r0 = blockIdx.x * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
+__device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, int b, float* s_sc) {
+  const int r0 = chunk * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
   for (int h = threadIdx.x; h < a.H; h += blockDim.x)
     s_sc[h] = head_scale(a.scale[static_cast<size_t>(b) * a.H + h]);
   __syncthreads();
@@ -224,10 +221,65 @@ __global__ void __launch_bounds__(kQuantThreads) quant_codes_kernel(QuantArgs a)
   }
 }
 
+// One tensor: grid = (ceil(S / rows_per_cta), B), block = kQuantThreads,
+// dynamic shared memory H * 4 bytes.
+template <typename T, bool HAD>
+__global__ void __launch_bounds__(kQuantThreads) quant_amax_kernel(QuantArgs a) {
+  extern __shared__ unsigned int s_amax[];
+  quant_amax_cta<T, HAD>(a, blockIdx.x, blockIdx.y, s_amax);
+}
+template <typename T, bool HAD>
+__global__ void __launch_bounds__(kQuantThreads) quant_codes_kernel(QuantArgs a) {
+  extern __shared__ float s_sc[];
+  quant_codes_cta<T, HAD>(a, blockIdx.x, blockIdx.y, s_sc);
+}
+
 // Step 4.
 __global__ void quant_finalize_kernel(float* scale, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) scale[i] = head_scale(scale[i]);
+}
+
+// Q, K and V in one launch per step: the CTAs of grid column x belong to
+// tensor i for first[i] <= x < first[i + 1] (chunk x - first[i]); had[i]
+// selects the rotated path.  Shared memory: max H * 4 bytes.
+struct Quant3Args {
+  QuantArgs t[3];
+  int had[3];
+  int first[4];
+};
+
+__device__ __forceinline__ int quant3_pick(const Quant3Args& a, int x) {
+  return x < a.first[1] ? 0 : (x < a.first[2] ? 1 : 2);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) quant3_amax_kernel(const __grid_constant__ Quant3Args a) {
+  extern __shared__ unsigned int s_amax[];
+  const int i = quant3_pick(a, blockIdx.x), chunk = blockIdx.x - a.first[i];
+  if (a.had[i]) quant_amax_cta<T, true>(a.t[i], chunk, blockIdx.y, s_amax);
+  else quant_amax_cta<T, false>(a.t[i], chunk, blockIdx.y, s_amax);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) quant3_codes_kernel(const __grid_constant__ Quant3Args a) {
+  extern __shared__ float s_sc[];
+  const int i = quant3_pick(a, blockIdx.x), chunk = blockIdx.x - a.first[i];
+  if (a.had[i]) quant_codes_cta<T, true>(a.t[i], chunk, blockIdx.y, s_sc);
+  else quant_codes_cta<T, false>(a.t[i], chunk, blockIdx.y, s_sc);
+}
+
+// Steps 1 and 4 for the three scale arrays (n[i] = B * H_i entries each).
+__global__ void quant3_zero_kernel(float* s0, float* s1, float* s2, int n0, int n1, int n2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n0) s0[i] = 0.0f;
+  else if (i < n0 + n1) s1[i - n0] = 0.0f;
+  else if (i < n0 + n1 + n2) s2[i - n0 - n1] = 0.0f;
+}
+__global__ void quant3_finalize_kernel(float* s0, float* s1, float* s2, int n0, int n1, int n2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  float* p = i < n0 ? s0 + i : (i < n0 + n1 ? s1 + (i - n0) : s2 + (i - n0 - n1));
+  if (i < n0 + n1 + n2) *p = head_scale(*p);
 }
 
 }  // namespace zyfa

@@ -259,6 +259,64 @@ extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* sc
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
+extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, int in_dtype, void* q_fp8,
+                                 void* k_fp8, void* v_fp8, float* q_scale, float* k_scale, float* v_scale,
+                                 int B, int S, int Hq, int Hkv, int Dqk, int Dv, int hadamard_qk, void* stream) {
+  if (!q || !k || !v || !q_fp8 || !k_fp8 || !v_fp8 || !q_scale || !k_scale || !v_scale) return ZYFA_ERR_NULL_PTR;
+  if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || B > 65535 || Hq > 4096 || Hkv > 4096) return ZYFA_ERR_BAD_SHAPE;
+  if (in_dtype != ZYFA_BF16 && in_dtype != ZYFA_FP32) return ZYFA_ERR_BAD_DTYPE;
+  if (hadamard_qk != 0 && hadamard_qk != 1) return ZYFA_ERR_BAD_DTYPE;
+  for (int d : {Dqk, Dv})
+    if (d < 8 || d > 1024 || d % 8 != 0) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (hadamard_qk && Dqk != 128) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  for (const void* t : {q, k, v, static_cast<const void*>(q_fp8), static_cast<const void*>(k_fp8),
+                        static_cast<const void*>(v_fp8)})
+    if (!aligned(t, 16)) return ZYFA_ERR_MISALIGNED;
+  if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4)) return ZYFA_ERR_MISALIGNED;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ZYFA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ZYFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Quant3Args a;
+  const void* xs[3] = {q, k, v};
+  void* outs[3] = {q_fp8, k_fp8, v_fp8};
+  float* scs[3] = {q_scale, k_scale, v_scale};
+  const int Hs[3] = {Hq, Hkv, Hkv}, Ds[3] = {Dqk, Dqk, Dv};
+  // CTAs per batch entry, split among the tensors in proportion to their bytes
+  const double want = static_cast<double>((4ll * sms + B - 1) / B);
+  double bytes[3], total = 0.0;
+  for (int i = 0; i < 3; ++i) { bytes[i] = static_cast<double>(Hs[i]) * Ds[i]; total += bytes[i]; }
+  a.first[0] = 0;
+  int max_h = 1;
+  for (int i = 0; i < 3; ++i) {
+    long long chunks = static_cast<long long>(want * bytes[i] / total + 0.5);
+    if (chunks < 1) chunks = 1;
+    if (chunks > S) chunks = S;
+    QuantArgs& t = a.t[i];
+    t.x = xs[i];
+    t.out = static_cast<uint8_t*>(outs[i]);
+    t.scale = scs[i];
+    t.S = S; t.H = Hs[i]; t.D = Ds[i];
+    t.rows_per_cta = static_cast<int>((S + chunks - 1) / chunks);
+    a.had[i] = (i < 2) ? hadamard_qk : 0;
+    a.first[i + 1] = a.first[i] + (S + t.rows_per_cta - 1) / t.rows_per_cta;
+    if (Hs[i] > max_h) max_h = Hs[i];
+  }
+  const dim3 grid(static_cast<unsigned>(a.first[3]), static_cast<unsigned>(B));
+  const size_t shm = static_cast<size_t>(max_h) * 4;
+  const int n0 = B * Hq, n1 = B * Hkv, n2 = B * Hkv, n = n0 + n1 + n2;
+  quant3_zero_kernel<<<(n + 255) / 256, 256, 0, st>>>(q_scale, k_scale, v_scale, n0, n1, n2);
+  if (in_dtype == ZYFA_BF16) {
+    quant3_amax_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
+    quant3_codes_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
+  } else {
+    quant3_amax_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
+    quant3_codes_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
+  }
+  quant3_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(q_scale, k_scale, v_scale, n0, n1, n2);
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
 extern "C" int zyfa_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZYFA_ERR_CUDA;
   int v = 0, zero = 0;

@@ -2,9 +2,9 @@
 
     python -m bf16_causal_prefill_fp8_b200.profile_case --workload gqa32x8_s16k_outlier --iters 3
 
-Each iteration launches, in order: zyfa_quantize for Q, K and V (amax, codes
-and finalize kernels each), the FP8 attention kernel, then the BF16 attention
-kernel on the same bf16 inputs.  Prints nothing but a completion line; timing
+Each iteration launches, in order: zyfa_quantize_qkv (zero, amax, codes and
+finalize kernels over Q, K and V together), the FP8 attention kernel, then the
+BF16 attention kernel on the same bf16 inputs.  Prints nothing but a completion line; timing
 numbers come from bench.py, never from a profiled run.
 """
 import argparse
@@ -26,9 +26,7 @@ def main():
     dq, dk, dv = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (q, k, v))
     for _ in range(args.iters):
         if args.only in ("all", "fp8"):
-            cq, sq = zyfa.quantize(dq, hadamard=args.hadamard)
-            ck, sk = zyfa.quantize(dk, hadamard=args.hadamard)
-            cv, sv = zyfa.quantize(dv)
+            (cq, sq), (ck, sk), (cv, sv) = zyfa.quantize_qkv(dq, dk, dv, hadamard_qk=args.hadamard)
             zyfa.attn_fwd(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv)
         if args.only in ("all", "bf16"):
             zyfa.attn_fwd(dq, dk, dv)

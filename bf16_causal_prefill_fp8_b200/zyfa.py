@@ -40,6 +40,8 @@ def lib() -> ctypes.CDLL:
         L.zyfa_attn_fwd.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, p, p, p]
         L.zyfa_quantize.restype = i
         L.zyfa_quantize.argtypes = [p, i, p, p, i, i, i, i, i, p]
+        L.zyfa_quantize_qkv.restype = i
+        L.zyfa_quantize_qkv.argtypes = [p, p, p, i, p, p, p, p, p, p, i, i, i, i, i, i, i, p]
         L.zyfa_status_string.restype = ctypes.c_char_p
         L.zyfa_status_string.argtypes = [i]
         L.zyfa_device_status.restype = i
@@ -132,6 +134,34 @@ def quantize(x, hadamard=False, out=None, scale=None, stream=None):
                              _stream(stream))
     _check(st, "zyfa_quantize")
     return out, scale
+
+
+def quantize_qkv(q, k, v, hadamard_qk=False, out=None, stream=None):
+    """Q, K, V [B,S,H,D] (same dtype: bf16 or fp32) -> ((q8, q_scale), (k8, k_scale), (v8, v_scale)),
+    identical to three quantize() calls (Hadamard on Q and K only), in four launches.  `out`: optional
+    ((q8, qs), (k8, ks), (v8, vs)) to write into."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k and v must share a dtype")
+    if q.dtype == torch.bfloat16:
+        dt = BF16
+    elif q.dtype == torch.float32:
+        dt = FP32
+    else:
+        raise ValueError(f"unsupported input dtype {q.dtype}")
+    B, S, Hq, Dqk = q.shape
+    Hkv, Dv = k.shape[2], v.shape[3]
+    if out is None:
+        out = tuple((torch.empty(t.shape, dtype=torch.uint8, device=t.device),
+                     torch.empty((B, t.shape[2]), dtype=torch.float32, device=t.device)) for t in (q, k, v))
+    for (c, sc), n in zip(out, "qkv"):
+        _dev(c, n + "_fp8"); _dev(sc, n + "_scale")
+    (q8, qs), (k8, ks), (v8, vs) = out
+    st = lib().zyfa_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs), _ptr(ks),
+                                 _ptr(vs), B, S, Hq, Hkv, Dqk, Dv, int(bool(hadamard_qk)), _stream(stream))
+    _check(st, "zyfa_quantize_qkv")
+    return out
 
 
 def leanp_codes(s, m, bmax, A, masked=None, stream=None):

@@ -123,6 +123,26 @@ int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
 int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* scale, int B, int S, int H,
                   int D, int hadamard, void* stream);
 
+/*
+ * zyfa_quantize_qkv -- the same prepass for Q, K and V at once (the sources
+ * above): byte for byte the result of
+ *   zyfa_quantize(q, in_dtype, q_fp8, q_scale, B, S, Hq, Dqk, hadamard_qk, s)
+ *   zyfa_quantize(k, in_dtype, k_fp8, k_scale, B, S, Hkv, Dqk, hadamard_qk, s)
+ *   zyfa_quantize(v, in_dtype, v_fp8, v_scale, B, S, Hkv, Dv, 0, s)
+ * in four kernel launches instead of twelve (each step of the prepass runs
+ * over the three tensors in one grid, shared in proportion to their bytes).
+ *   q [B, S, Hq, Dqk], k [B, S, Hkv, Dqk], v [B, S, Hkv, Dv]: in_dtype
+ *   *_fp8: e4m3 codes of the same shapes (outputs, caller-owned)
+ *   *_scale: fp32 [B*Hq], [B*Hkv], [B*Hkv] (outputs; used as amax
+ *   accumulators while the call's kernels run)
+ * Dqk and Dv: multiples of 8, at most 1024 (Dqk = 128 with hadamard_qk = 1).
+ * Alignment as for zyfa_quantize.  Errors as for zyfa_quantize; nothing is
+ * launched when an argument is rejected.
+ */
+int zyfa_quantize_qkv(const void* q, const void* k, const void* v, int in_dtype, void* q_fp8,
+                      void* k_fp8, void* v_fp8, float* q_scale, float* k_scale, float* v_scale,
+                      int B, int S, int Hq, int Hkv, int Dqk, int Dv, int hadamard_qk, void* stream);
+
 /* Human-readable text of a status code (static storage; never NULL). */
 const char* zyfa_status_string(int status);
 

@@ -15,7 +15,8 @@ def L():
 
 def test_every_declared_symbol_is_exported(L):
     names = zyfa.declared_symbols()
-    assert set(names) >= {"zyfa_attn_fwd", "zyfa_quantize", "zyfa_status_string", "zyfa_device_status",
+    assert set(names) >= {"zyfa_attn_fwd", "zyfa_quantize", "zyfa_quantize_qkv", "zyfa_status_string",
+                          "zyfa_device_status",
                           "zyfa_leanp_codes", "zyfa_selftest_wait_timeout", "zyfa_set_wait_timeout_ns"}
     for n in names:
         assert hasattr(L, n), n
@@ -68,6 +69,22 @@ def test_quantize_argument_errors(L):
     assert q(D=192, had=1) == -3
     assert q(x=FAKE + 4) == -5
     assert q(sc=FAKE + 2) == -5
+
+
+def test_quantize_qkv_argument_errors(L):
+    def q(q=FAKE, k=FAKE, v=FAKE, dt=0, q8=FAKE, k8=FAKE, v8=FAKE, qs=FAKE, ks=FAKE, vs=FAKE, B=1, S=16, Hq=4,
+          Hkv=2, Dqk=128, Dv=128, had=0):
+        return L.zyfa_quantize_qkv(q, k, v, dt, q8, k8, v8, qs, ks, vs, B, S, Hq, Hkv, Dqk, Dv, had, None)
+    assert q(v=None) == -1
+    assert q(ks=None) == -1
+    assert q(S=0) == -2
+    assert q(Hkv=0) == -2
+    assert q(dt=1) == -6
+    assert q(had=3) == -6
+    assert q(Dv=4) == -3
+    assert q(Dqk=192, had=1) == -3
+    assert q(k8=FAKE + 8) == -5
+    assert q(vs=FAKE + 1) == -5
 
 
 def test_leanp_and_selftest_argument_errors(L):

@@ -37,3 +37,26 @@ def test_quantize_outlier_channels_and_subnormals():
         rc, rs = orc.quantize(x, hadamard=had)
         assert np.array_equal(scale.cpu().numpy().view(np.uint32), rs.view(np.uint32))
         assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,Dqk,Dv,hadamard", [(1, 300, 8, 2, 128, 128, False),
+                                                        (2, 129, 4, 4, 128, 128, True),
+                                                        (1, 77, 6, 2, 192, 128, False),
+                                                        (1, 2048, 32, 8, 128, 128, True),
+                                                        (3, 5, 2, 1, 128, 128, False)])
+@pytest.mark.parametrize("as_bf16", [False, True])
+def test_quantize_qkv_equals_three_calls_and_oracle(B, S, Hq, Hkv, Dqk, Dv, hadamard, as_bf16):
+    """zyfa_quantize_qkv (one grid for Q, K and V per step) gives the oracle's
+    codes and scales, byte for byte, like three zyfa_quantize calls."""
+    import torch
+    from bf16_causal_prefill_fp8_b200 import zyfa
+    q, k, v = synth.make_qkv(31, B, S, Hq, Hkv, Dqk, Dv, "outlier_k")
+    q[0, :, 0, :] *= np.float32(40.0)
+    to = (lambda x: bf16_round(x).cuda()) if as_bf16 else (lambda x: torch.from_numpy(x).cuda())
+    got = zyfa.quantize_qkv(to(q), to(k), to(v), hadamard_qk=hadamard)
+    torch.cuda.synchronize()
+    for (c, sc), x, had in zip(got, (q, k, v), (hadamard, hadamard, False)):
+        xin = bf16_round(x).float().numpy() if as_bf16 else x
+        rc, rs = orc.quantize(xin, hadamard=had)
+        assert np.array_equal(sc.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+        assert np.array_equal(c.cpu().numpy(), rc)
