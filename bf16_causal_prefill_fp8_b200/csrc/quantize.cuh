@@ -15,7 +15,8 @@
 //   1. memset(scale, 0)                         scale doubles as amax accumulator
 //   2. quant_amax_kernel:  scale[b,h] = max(scale[b,h], max |x'|)   (fp32 bits,
 //      atomicMax on the non-negative bit patterns, order-independent)
-//   3. quant_codes_kernel: s = amax/448 (1 if amax == 0); code = e4m3(x'/s)
+//   3. quant_codes_kernel: s = amax/448 (1 if amax == 0); code = e4m3(x'/s),
+//      the quotient correctly rounded (div_by_scale)
 //   4. quant_finalize_kernel: scale[b,h] = s
 // x' is the row rotated by the orthonormal Sylvester transform when
 // hadamard != 0 (stages of stride 1, 2, ..., 64 in fp32, then one multiply by
@@ -38,6 +39,25 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
 
 __device__ __forceinline__ float head_scale(float amax) {
   return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+}
+
+// x / s rounded to nearest even, given rc = RN(1/s) (Markstein's correction,
+// P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also Muller et al.,
+// "Handbook of Floating-Point Arithmetic", division by FMA): q0 = RN(x rc) is
+// within one ulp of x/s, the residual x - s q0 is then exact in one FMA, and
+// RN(q0 + residual * rc) is the correctly rounded quotient.  rc == 0 marks a
+// scale too small or too large for the reciprocal to stay normal: plain
+// division.  The quotients here are at most 448 in magnitude.
+__device__ __forceinline__ float div_by_scale(float x, float s, float rc) {
+  if (rc == 0.0f) return __fdiv_rn(x, s);
+  const float q0 = __fmul_rn(x, rc);
+  const float r = __fmaf_rn(-q0, s, x);
+  return __fmaf_rn(r, rc, q0);
+}
+
+__device__ __forceinline__ float scale_reciprocal(float s) {
+  return (s >= 0x1p-120f && s <= 0x1p120f) ? __frcp_rn(s) : 0.0f;
 }
 
 // 16-byte vectors: 8 bf16 or 4 fp32 elements.
@@ -165,8 +185,12 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
 template <typename T, bool HAD>
 __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, int b, float* s_sc) {
   const int r0 = chunk * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
-  for (int h = threadIdx.x; h < a.H; h += blockDim.x)
-    s_sc[h] = head_scale(a.scale[static_cast<size_t>(b) * a.H + h]);
+  float* s_rc = s_sc + a.H;   // RN(1 / scale) per head
+  for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+    const float sc = head_scale(a.scale[static_cast<size_t>(b) * a.H + h]);
+    s_sc[h] = sc;
+    s_rc[h] = scale_reciprocal(sc);
+  }
   __syncthreads();
   const uint32_t HD = static_cast<uint32_t>(a.H) * a.D;
   const size_t off = (static_cast<size_t>(b) * a.S + r0) * HD;
@@ -184,9 +208,10 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
       for (int u = 0; u < kUnroll; ++u) {
         if (v0 + u >= nvec) break;
         fwht128_warp(x[u], lane);
-        const float sc = s_sc[(v0 + u) % a.H];
-        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[u][0], sc), __fdiv_rn(x[u][1], sc));
-        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[u][2], sc), __fdiv_rn(x[u][3], sc));
+        const int hh = (v0 + u) % a.H;
+        const float sc = s_sc[hh], rc = s_rc[hh];
+        const uint32_t lo = cvt_e4m3x2(div_by_scale(x[u][0], sc, rc), div_by_scale(x[u][1], sc, rc));
+        const uint32_t hi = cvt_e4m3x2(div_by_scale(x[u][2], sc, rc), div_by_scale(x[u][3], sc, rc));
         *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(v0 + u) * 128 + 4 * lane) = lo | (hi << 16);
       }
     }
@@ -208,12 +233,14 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
         if (vi >= nvec) break;
         float x[N];
         Vec<T>::unpack(raw[u], x);
-        const float sc = s_sc[(vi % vpr) / vph];
+        const uint32_t hh = (vi % vpr) / vph;
+        const float sc = s_sc[hh], rc = s_rc[hh];
         uint32_t w[N / 4];
 #pragma unroll
         for (int i = 0; i < N / 4; ++i)
-          w[i] = cvt_e4m3x2(__fdiv_rn(x[4 * i], sc), __fdiv_rn(x[4 * i + 1], sc)) |
-                 (static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(x[4 * i + 2], sc), __fdiv_rn(x[4 * i + 3], sc))) << 16);
+          w[i] = cvt_e4m3x2(div_by_scale(x[4 * i], sc, rc), div_by_scale(x[4 * i + 1], sc, rc)) |
+                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(x[4 * i + 2], sc, rc),
+                                                   div_by_scale(x[4 * i + 3], sc, rc))) << 16);
         if constexpr (N == 8) *reinterpret_cast<uint2*>(obase + static_cast<size_t>(vi) * 8) = make_uint2(w[0], w[1]);
         else *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(vi) * 4) = w[0];
       }
@@ -222,7 +249,7 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
 }
 
 // One tensor: grid = (ceil(S / rows_per_cta), B), block = kQuantThreads,
-// dynamic shared memory H * 4 bytes.
+// dynamic shared memory H * 8 bytes.
 template <typename T, bool HAD>
 __global__ void __launch_bounds__(kQuantThreads) quant_amax_kernel(QuantArgs a) {
   extern __shared__ unsigned int s_amax[];
@@ -242,7 +269,7 @@ __global__ void quant_finalize_kernel(float* scale, int n) {
 
 // Q, K and V in one launch per step: the CTAs of grid column x belong to
 // tensor i for first[i] <= x < first[i + 1] (chunk x - first[i]); had[i]
-// selects the rotated path.  Shared memory: max H * 4 bytes.
+// selects the rotated path.  Shared memory: max H * 8 bytes.
 struct Quant3Args {
   QuantArgs t[3];
   int had[3];

@@ -234,7 +234,7 @@ extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* sc
   a.S = S; a.H = H; a.D = D;
   a.rows_per_cta = static_cast<int>((S + chunks - 1) / chunks);
   const dim3 grid(static_cast<unsigned>((S + a.rows_per_cta - 1) / a.rows_per_cta), static_cast<unsigned>(B));
-  const size_t shm = static_cast<size_t>(H) * 4;
+  const size_t shm = static_cast<size_t>(H) * 8;   // amax, or scale and its reciprocal, per head
   if (cudaMemsetAsync(scale, 0, static_cast<size_t>(B) * H * sizeof(float), st) != cudaSuccess)
     return ZYFA_ERR_CUDA;
   if (in_dtype == ZYFA_BF16) {
@@ -283,7 +283,8 @@ extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, in
   float* scs[3] = {q_scale, k_scale, v_scale};
   const int Hs[3] = {Hq, Hkv, Hkv}, Ds[3] = {Dqk, Dqk, Dv};
   // CTAs per batch entry, split among the tensors in proportion to their bytes
-  const double want = static_cast<double>((4ll * sms + B - 1) / B);
+  // (the rotated path does more work per byte: twice as many CTAs)
+  const double want = static_cast<double>(((hadamard_qk ? 8ll : 4ll) * sms + B - 1) / B);
   double bytes[3], total = 0.0;
   for (int i = 0; i < 3; ++i) { bytes[i] = static_cast<double>(Hs[i]) * Ds[i]; total += bytes[i]; }
   a.first[0] = 0;
@@ -303,7 +304,7 @@ extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, in
     if (Hs[i] > max_h) max_h = Hs[i];
   }
   const dim3 grid(static_cast<unsigned>(a.first[3]), static_cast<unsigned>(B));
-  const size_t shm = static_cast<size_t>(max_h) * 4;
+  const size_t shm = static_cast<size_t>(max_h) * 8;   // amax, or scale and its reciprocal, per head
   const int n0 = B * Hq, n1 = B * Hkv, n2 = B * Hkv, n = n0 + n1 + n2;
   quant3_zero_kernel<<<(n + 255) / 256, 256, 0, st>>>(q_scale, k_scale, v_scale, n0, n1, n2);
   if (in_dtype == ZYFA_BF16) {

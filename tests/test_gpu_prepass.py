@@ -60,3 +60,28 @@ def test_quantize_qkv_equals_three_calls_and_oracle(B, S, Hq, Hkv, Dqk, Dv, hada
         rc, rs = orc.quantize(xin, hadamard=had)
         assert np.array_equal(sc.cpu().numpy().view(np.uint32), rs.view(np.uint32))
         assert np.array_equal(c.cpu().numpy(), rc)
+
+
+def test_quantize_quotients_at_e4m3_midpoints():
+    """Inputs whose quotient by the head scale lands exactly on, or one fp32 ulp
+    either side of, every rounding midpoint between adjacent e4m3 values: a
+    quotient off by one ulp flips the code here.  The scale is uneven
+    (amax = 448 * 1.3717), so the division is not exact."""
+    vals = np.sort(np.unique(np.abs(orc.e4m3_values()[np.isfinite(orc.e4m3_values())]))).astype(np.float64)
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)          # exact in fp32
+    amax = np.float32(448.0 * 1.3717)
+    s = np.float32(amax / np.float32(448.0))
+    xs = []
+    for m in mids:
+        x = np.float32(m * s)
+        xs += [np.nextafter(x, np.float32(-np.inf)), x, np.nextafter(x, np.float32(np.inf))]
+    xs = np.array(xs, dtype=np.float32)
+    xs = np.concatenate([xs, -xs, [amax]])
+    n = (len(xs) + 127) // 128 * 128
+    row = np.zeros(n, dtype=np.float32); row[:len(xs)] = xs
+    x = row.reshape(1, n // 128, 1, 128)
+    codes, scale = quantize_gpu(x)
+    rc, rs = orc.quantize(x)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    got = codes.cpu().numpy()
+    assert np.array_equal(got, rc), f"{np.count_nonzero(got != rc)} codes differ"
