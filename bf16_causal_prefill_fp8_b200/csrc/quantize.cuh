@@ -79,42 +79,42 @@ template <> struct Vec<float> {
   }
 };
 
-// Load 4 consecutive elements as fp32 (Hadamard path: lane l holds 4l .. 4l+3).
+// Rotated path, half a warp per row: lane l of a half holds elements
+// 8l .. 8l+7 (16-byte bf16 / 32-byte fp32 loads).  Butterflies of stride
+// 1, 2, 4 in registers and 8 .. 64 across the 16 lanes of the half, in that
+// order (the order the rotation is defined with), each stage the fp32 sum and
+// difference of its pair; four shuffles per element.
 template <typename T>
-__device__ __forceinline__ void load4(const T* p, float (&v)[4]);
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
 template <>
-__device__ __forceinline__ void load4<float>(const float* p, float (&v)[4]) {
-  const float4 t = __ldg(reinterpret_cast<const float4*>(p));
-  v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 template <>
-__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[4]) {
-  const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
-  v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xffff0000u);
-  v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xffff0000u);
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  Vec<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4*>(p)), v);
 }
 
-// In-warp 128-point transform: lane l holds elements 4l .. 4l+3.
-__device__ __forceinline__ void fwht128_warp(float (&x)[4], int lane) {
+__device__ __forceinline__ void fwht128_half(float (&x)[8], int li) {
   float a, b;
-  // stride 1
-  a = x[0]; b = x[1]; x[0] = a + b; x[1] = a - b;
-  a = x[2]; b = x[3]; x[2] = a + b; x[3] = a - b;
-  // stride 2
-  a = x[0]; b = x[2]; x[0] = a + b; x[2] = a - b;
-  a = x[1]; b = x[3]; x[1] = a + b; x[3] = a - b;
-  // strides 4 .. 64: partner lane differs in one bit
 #pragma unroll
-  for (int sh = 1; sh < 32; sh <<= 1) {
-    const bool upper = (lane & sh) != 0;
+  for (int st = 1; st < 8; st <<= 1)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i)
+      if ((i & st) == 0) { a = x[i]; b = x[i + st]; x[i] = a + b; x[i + st] = a - b; }
+#pragma unroll
+  for (int sh = 1; sh < 16; sh <<= 1) {   // strides 8, 16, 32, 64
+    const bool upper = (li & sh) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
       const float o = __shfl_xor_sync(0xffffffffu, x[i], sh);
       x[i] = upper ? (o - x[i]) : (x[i] + o);
     }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) x[i] = x[i] * kFwhtNorm;
+  for (int i = 0; i < 8; ++i) x[i] = x[i] * kFwhtNorm;
 }
 
 struct QuantArgs {
@@ -135,20 +135,29 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
   const T* base = static_cast<const T*>(a.x) + (static_cast<size_t>(b) * a.S + r0) * HD;
   if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int half = lane >> 4, li = lane & 15;
     const int nvec = (r1 - r0) * a.H;          // 128-element rows
-    for (int v0 = warp * kUnroll; v0 < nvec; v0 += nw * kUnroll) {
-      float x[kUnroll][4];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (v0 + u < nvec) load4<T>(base + static_cast<size_t>(v0 + u) * 128 + 4 * lane, x[u]);
+    for (int v0 = warp * 2 * kUnroll; v0 < nvec; v0 += nw * 2 * kUnroll) {
+      float x[kUnroll][8];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        if (v0 + u >= nvec) break;
-        fwht128_warp(x[u], lane);
-        float mx = fmaxf(fmaxf(fabsf(x[u][0]), fabsf(x[u][1])), fmaxf(fabsf(x[u][2]), fabsf(x[u][3])));
+        const int v = v0 + 2 * u + half;
+        if (v < nvec) load8<T>(base + static_cast<size_t>(v) * 128 + 8 * li, x[u]);
+        else
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) atomicMax(&s_amax[(v0 + u) % a.H], __float_as_uint(mx));
+          for (int i = 0; i < 8; ++i) x[u][i] = 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + 2 * u >= nvec) break;                  // both halves past the end
+        fwht128_half(x[u], li);
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[u][i]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const int v = v0 + 2 * u + half;
+        if (li == 0 && v < nvec) atomicMax(&s_amax[v % a.H], __float_as_uint(mx));
       }
     }
   } else {
@@ -198,21 +207,33 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
   uint8_t* obase = a.out + off;
   if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int half = lane >> 4, li = lane & 15;
     const int nvec = (r1 - r0) * a.H;
-    for (int v0 = warp * kUnroll; v0 < nvec; v0 += nw * kUnroll) {
-      float x[kUnroll][4];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (v0 + u < nvec) load4<T>(base + static_cast<size_t>(v0 + u) * 128 + 4 * lane, x[u]);
+    for (int v0 = warp * 2 * kUnroll; v0 < nvec; v0 += nw * 2 * kUnroll) {
+      float x[kUnroll][8];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        if (v0 + u >= nvec) break;
-        fwht128_warp(x[u], lane);
-        const int hh = (v0 + u) % a.H;
+        const int v = v0 + 2 * u + half;
+        if (v < nvec) load8<T>(base + static_cast<size_t>(v) * 128 + 8 * li, x[u]);
+        else
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[u][i] = 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + 2 * u >= nvec) break;
+        fwht128_half(x[u], li);
+        const int v = v0 + 2 * u + half;
+        if (v >= nvec) continue;
+        const int hh = v % a.H;
         const float sc = s_sc[hh], rc = s_rc[hh];
-        const uint32_t lo = cvt_e4m3x2(div_by_scale(x[u][0], sc, rc), div_by_scale(x[u][1], sc, rc));
-        const uint32_t hi = cvt_e4m3x2(div_by_scale(x[u][2], sc, rc), div_by_scale(x[u][3], sc, rc));
-        *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(v0 + u) * 128 + 4 * lane) = lo | (hi << 16);
+        uint32_t w[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          w[i] = cvt_e4m3x2(div_by_scale(x[u][4 * i], sc, rc), div_by_scale(x[u][4 * i + 1], sc, rc)) |
+                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(x[u][4 * i + 2], sc, rc),
+                                                   div_by_scale(x[u][4 * i + 3], sc, rc))) << 16);
+        *reinterpret_cast<uint2*>(obase + static_cast<size_t>(v) * 128 + 8 * li) = make_uint2(w[0], w[1]);
       }
     }
   } else {
