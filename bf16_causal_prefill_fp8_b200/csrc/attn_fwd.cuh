@@ -81,14 +81,19 @@ struct AttnCfg {
   static constexpr int QB = 128 * ROWB;
   static constexpr int KB = 128 * ROWB;
   static constexpr int VB = 128 * 128 * EL;          // Dv = 128
-  static constexpr int ST = FP8 ? 4 : 2;             // K/V ring stages
-  static constexpr int QBUF = (!FP8 && DQK == 192) ? 1 : 2;   // Q tile buffers (units in flight)
+  // ring stages: FP8 4 K + 4 V with two Q buffers; BF16 Dqk 128 trades its
+  // second Q buffer for a third K stage (S waits on K tiles, P V on V tiles a
+  // whole softmax pass later); BF16 Dqk 192 fits 2 + 2 with one Q buffer
+  static constexpr int STK = FP8 ? 4 : (DQK == 128 ? 3 : 2);
+  static constexpr int STV = FP8 ? 4 : 2;
+  static constexpr int QBUF = FP8 ? 2 : 1;           // Q tile buffers (units in flight)
+  static constexpr int KLEAD = STK - STV + 1;         // K tiles the producer keeps ahead of V
   static constexpr int NPB = FP8 ? 3 : 2;            // P buffers (tile g uses g % NPB)
   static constexpr int NK_QK = ROWB / 32;            // QK MMA K-steps of 32 bytes
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBUF * QB;
-  static constexpr int OFF_V = OFF_K + ST * KB;
-  static constexpr int OFF_ONES = OFF_V + ST * VB;   // FP8: 16 x 128 bytes of e4m3 1.0
+  static constexpr int OFF_V = OFF_K + STK * KB;
+  static constexpr int OFF_ONES = OFF_V + STV * VB;   // FP8: 16 x 128 bytes of e4m3 1.0
   static constexpr int OFF_SF = OFF_ONES + (FP8 ? 2048 : 0);   // FP8: NPB x 512 B scale factors
   static constexpr int OFF_ALPHA = OFF_SF + (FP8 ? NPB * 512 : 0);  // NPB x 128 fp32 rescale factors
   static constexpr int OFF_LFIN = OFF_ALPHA + NPB * 512;  // BF16 final partial row sums, per group (2 x 128 fp32)
@@ -102,8 +107,8 @@ struct AttnCfg {
   // updated), OR = O corrected, ready for P V.
   enum { QF0 = 0, QF1, QE0, QE1, OF, OFIN, DRAIN, DRAIN2, SF0, SF1, SC0, SC1, PF0, PF1, PF2, PE0, PE1, PE2,
          OR0, OR1, OR2, MX0, MX1, KF };
-  static constexpr int KE = KF + ST, VF = KF + 2 * ST, VE = KF + 3 * ST;
-  static constexpr int NBAR = KF + 4 * ST;
+  static constexpr int KE = KF + STK, VF = KF + 2 * STK, VE = VF + STV;
+  static constexpr int NBAR = VE + STV;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   // tensor-memory columns (512 allocated)
@@ -269,9 +274,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(bar(Cf::PE0 + i), 1);
       mbar_init(bar(Cf::OR0 + i), 128);
     }
-    for (int i = 0; i < Cf::ST; ++i) {
+    for (int i = 0; i < Cf::STK; ++i) {
       mbar_init(bar(Cf::KF + i), 1);
       mbar_init(bar(Cf::KE + i), 1);
+    }
+    for (int i = 0; i < Cf::STV; ++i) {
       mbar_init(bar(Cf::VF + i), 1);
       mbar_init(bar(Cf::VE + i), 1);
     }
@@ -314,7 +321,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
    };
    if (warp == 12) {
     // ------------------------------------------------------------ producer
-    // K runs one tile ahead of V, in the order the MMAs consume them.
+    // K runs KLEAD tiles ahead of V, in the order the MMAs consume them.
     const uint64_t pol_q = l2_policy_evict_first();
     const uint64_t pol_kv = l2_policy_evict_last();
     TileStream ks, vs;
@@ -338,7 +345,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
                     t.hq, t.qt * 128, t.b, pol_q);
         }
       }
-      const uint32_t st = t.g % Cf::ST, n = t.g / Cf::ST;
+      const uint32_t st = t.g % Cf::STK, n = t.g / Cf::STK;
       if (n > 0 && !wait1(bar(Cf::KE + st), (n - 1) & 1)) return false;
       if (leader) {
         mbar_arrive_expect_tx(bar(Cf::KF + st), Cf::KB);
@@ -349,7 +356,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       return true;
     };
     auto load_v = [&](const TileStream& t) -> bool {
-      const uint32_t st = t.g % Cf::ST, n = t.g / Cf::ST;
+      const uint32_t st = t.g % Cf::STV, n = t.g / Cf::STV;
       if (n > 0 && !wait1(bar(Cf::VE + st), (n - 1) & 1)) return false;
       if (leader) {
         mbar_arrive_expect_tx(bar(Cf::VF + st), Cf::VB);
@@ -361,7 +368,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       __syncwarp();
       return true;
     };
-    if (ks.next()) ok = load_k(ks);
+    for (int i = 0; i < Cf::KLEAD && ok && ks.next(); ++i) ok = load_k(ks);
     while (ok && vs.next()) {
       if (ks.next()) ok = load_k(ks);
       if (ok) ok = load_v(vs);
@@ -390,8 +397,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     auto issue_qk = [&](const TileStream& t) -> bool {
       const uint32_t slot = t.u % Cf::QBUF;
       if (t.j == 0 && !wait1(bar(Cf::QF0 + slot), (t.u / Cf::QBUF) & 1)) return false;
-      const uint32_t st = t.g % Cf::ST, buf = t.g & 1;
-      if (!wait1(bar(Cf::KF + st), (t.g / Cf::ST) & 1)) return false;
+      const uint32_t st = t.g % Cf::STK, buf = t.g & 1;
+      if (!wait1(bar(Cf::KF + st), (t.g / Cf::STK) & 1)) return false;
       if (t.g >= 2 && !wait1(bar(Cf::SC0 + buf), ((t.g >> 1) - 1) & 1)) return false;
       tc_fence_after();
       const uint64_t dqs = dq + ((slot * Cf::QB) >> 4), dqs_t = dq_t + ((slot * Cf::QB) >> 4);
@@ -419,12 +426,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       return true;
     };
     auto issue_pv = [&](const TileStream& t) -> bool {
-      const uint32_t st = t.g % Cf::ST, buf = t.g % Cf::NPB, ph = (t.g / Cf::NPB) & 1;
+      const uint32_t st = t.g % Cf::STV, buf = t.g % Cf::NPB, ph = (t.g / Cf::NPB) & 1;
       const bool first = t.j == 0;
       // O is free once the previous unit's epilogue has read it
       if (first && t.u > 0 && !wait1(bar(Cf::OF), (t.u - 1) & 1)) return false;
       if (!wait1(bar(Cf::OR0 + buf), ph)) return false;   // P stored, O corrected
-      if (!wait1(bar(Cf::VF + st), (t.g / Cf::ST) & 1)) return false;
+      if (!wait1(bar(Cf::VF + st), (t.g / Cf::STV) & 1)) return false;
       tc_fence_after();
       const uint64_t dvs = dv + ((st * Cf::VB) >> 4);
       const uint32_t tp = tbase + Cf::tp(buf);
