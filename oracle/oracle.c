@@ -34,7 +34,10 @@
  *   oracle_leanp_* : code == 8j + 56 when s == m == 0; monotone in s; decoded
  *       weight / exact weight inside Mitchell's band (2^-1/8, 1.0615] for
  *       normal codes; largest code of a block in (112, 120].
- *   oracle_fp8_model_rows : with exact_p = 1 equals oracle_attention_rows on
+ *   oracle_exactp_code : code 8j + 56 at s = m (a power of two: exact); monotone
+ *       in s; decoded weight within e4m3's half-ulp bound (2^-4 relative) of
+ *       the exact weight for normal codes.
+ *   oracle_fp8_model_rows : with p_mode = 1 equals oracle_attention_rows on
  *       the dequantized inputs to 1e-6 (pins tile order, running max, the
  *       rescale factor and the row sum), also with the deferred reference max
  *       on scores that grow by many binades across the keys; Q = 0 gives
@@ -270,6 +273,20 @@ unsigned oracle_leanp_code(float s, float m, float A, int j, int masked)
     return (unsigned)t;
 }
 
+/* The exact-P alternative (the pages' baseline that Lean P replaces, [NL]   */
+/* "Drie technieken", [JA] "Lean P": an exponential, then a conversion to   */
+/* e4m3): the same block shift j, then                                       */
+/*   code = e4m3 RNE-satfinite of fl32(exp2((s - m) A / 8 + j))             */
+/* (exp2 in fp64, rounded once to fp32); 0 for a masked key.  The weight is  */
+/* value(code) * 2^-j, as for Lean P.                                        */
+unsigned oracle_exactp_code(float s, float m, float A, int j, int masked)
+{
+    double x;
+    if (masked || (isinf(s) && s < 0.0f)) return 0u;
+    x = ((double)s - (double)m) * (double)A / 8.0 + (double)j;
+    return oracle_e4m3_from_f32((float)exp2(x));
+}
+
 /* Element-wise batch form used by the bit-exactness test. */
 void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
                         const float *A, const uint8_t *masked, int n,
@@ -297,7 +314,9 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 /*           max is more than rescale_log2 binades above m, else m' = m.    */
 /*           The softmax is unchanged: O and l share the reference and the */
 /*           per-block shift j renormalises each block to its own max.)     */
-/*   w_j   = value(leanp code) * 2^-j_block  (exact_p: exp2((s_j-m')A/8))   */
+/*   w_j   = value(leanp code) * 2^-j_block                                  */
+/*           p_mode 1: exp2((s_j-m')A/8) in fp64 (no rounding of P);          */
+/*           p_mode 2: value(exact-P e4m3 code) * 2^-j_block                 */
 /*   alpha = exp2((m - m') A / 8)            (0 on the first tile)          */
 /*   O     = alpha O + sum_j w_j value(vcode_j);  l = alpha l + sum_j w_j   */
 /* Every block shift j must stay >= 0 (weights <= 448, E8M0 scale <= 1):   */
@@ -311,7 +330,7 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *vc,
                           const float *q_s, const float *k_s, const float *v_s,
                           int B, int Hq, int Hkv, int S, int Dqk, int Dv,
-                          int exact_p, float rescale_log2,
+                          int p_mode, float rescale_log2,
                           const int *rows, int nrows, double *o)
 {
     int b, shift_err = 0;
@@ -379,8 +398,12 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
                     double w;
                     const uint8_t *vj;
                     if (!live[n]) continue;
-                    if (exact_p) {
+                    if (p_mode == 1) {
                         w = exp2(((double)sj[n] - (double)mnew) * (double)A / 8.0);
+                    } else if (p_mode == 2) {
+                        int sh = oracle_leanp_block_shift(mnew, bmax[n / 64], A);
+                        unsigned c = oracle_exactp_code(sj[n], mnew, A, sh, 0);
+                        w = ldexp(oracle_e4m3_value(c), -sh);
                     } else {
                         int sh = oracle_leanp_block_shift(mnew, bmax[n / 64], A);
                         unsigned c = oracle_leanp_code(sj[n], mnew, A, sh, 0);

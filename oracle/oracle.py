@@ -43,6 +43,8 @@ def lib():
         L.oracle_fp8_model_rows.restype = c_i
         L.oracle_fp8_model_rows.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i,
                                             c_i, c_i, c_i, c_f, c_p, c_i, c_p]
+        L.oracle_exactp_code.restype = ctypes.c_uint
+        L.oracle_exactp_code.argtypes = [c_f, c_f, c_f, c_i, c_i]
         L.oracle_num_threads.restype = c_i
         L.oracle_num_threads.argtypes = []
         _lib = L
@@ -144,6 +146,11 @@ def leanp_code(s, m, A, j, masked=False) -> int:
     return lib().oracle_leanp_code(float(s), float(m), float(A), int(j), int(bool(masked)))
 
 
+def exactp_code(s, m, A, j, masked=False) -> int:
+    """The exact-P ablation's code: e4m3 of fl32(exp2((s - m) A / 8 + j))."""
+    return lib().oracle_exactp_code(float(s), float(m), float(A), int(j), int(bool(masked)))
+
+
 def leanp_batch(s, m, bmax, A, masked=None):
     """Element-wise Lean-P codes and block shifts (fp32 inputs, same length)."""
     s = _c(s, np.float32); m = _c(m, np.float32); bmax = _c(bmax, np.float32); A = _c(A, np.float32)
@@ -155,11 +162,15 @@ def leanp_batch(s, m, bmax, A, masked=None):
     return code, j
 
 
-def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=0.0) -> np.ndarray:
+def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=0.0, p_mode=None) -> np.ndarray:
     """The FP8 pipeline replayed on the CPU (see oracle.c).  Codes uint8 BSHD,
     scales fp32 [B,H].  rescale_log2 = 0: exact running max; > 0: the reference
     max moves only when a tile max exceeds it by more than that many binades.
+    p_mode: 0 Lean-P codes (default), 1 exact fp64 weights (exact_p=True),
+    2 exact exp2 rounded to e4m3 (the exact-P ablation).
     Returns o fp64 [B, S or len(rows), Hq, Dv]."""
+    if p_mode is None:
+        p_mode = 1 if exact_p else 0
     qc = _c(qc, np.uint8); kc = _c(kc, np.uint8); vc = _c(vc, np.uint8)
     q_s = _c(q_s, np.float32); k_s = _c(k_s, np.float32); v_s = _c(v_s, np.float32)
     B, S, Hq, Dqk = qc.shape
@@ -168,7 +179,7 @@ def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=
     n = S if rows is None else len(r)
     o = np.empty((B, n, Hq, Dv), dtype=np.float64)
     rc = lib().oracle_fp8_model_rows(_ptr(qc), _ptr(kc), _ptr(vc), _ptr(q_s), _ptr(k_s), _ptr(v_s),
-                                     B, Hq, Hkv, S, Dqk, Dv, int(bool(exact_p)), ctypes.c_float(rescale_log2), _ptr(r), n, _ptr(o))
+                                     B, Hq, Hkv, S, Dqk, Dv, int(p_mode), ctypes.c_float(rescale_log2), _ptr(r), n, _ptr(o))
     if rc == -2:
         raise ArithmeticError("oracle_fp8_model_rows: a block shift fell below 0 (reference max too stale)")
     if rc != 0:

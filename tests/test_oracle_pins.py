@@ -326,3 +326,50 @@ def test_model_oracle_leanp_error_against_fp64_is_within_fp8_bar():
     ref = orc.attention(*deq)
     err = orc.rel_fro(o, ref)
     assert 1e-3 < err < 3e-2
+
+
+# --- exact-P ablation codes --------------------------------------------------------
+
+def test_exactp_code_power_of_two_ladder_and_masking():
+    # s == m: exp2(j) exactly, whose e4m3 code is 8j + 56 (the format's ladder)
+    A = orc.leanp_slope(np.float32(0.01), np.float32(0.02), 128)
+    for j in range(0, 9):
+        assert orc.exactp_code(3.0, 3.0, A, j) == 8 * j + 56
+    assert orc.exactp_code(-np.inf, 0.0, A, 8) == 0
+    assert orc.exactp_code(1.0, 2.0, A, 8, masked=True) == 0
+
+
+def test_exactp_code_monotone_and_within_half_ulp():
+    """Decoded weight / exact weight stays within e4m3's half-ulp bound for
+    normal codes (2^-4 relative), and codes never decrease with s."""
+    rng = np.random.default_rng(5)
+    vals = orc.e4m3_values()
+    A = np.float32(0.9)
+    m = np.float32(50.0)
+    s = np.sort(rng.uniform(-60.0, 50.0, 4000).astype(np.float32))
+    prev = -1
+    for si in s:
+        j = 8
+        c = orc.exactp_code(si, m, A, j)
+        assert c >= prev
+        prev = c
+        exact = 2.0 ** ((float(si) - float(m)) * float(A) / 8.0 + j)
+        if c >= 8:                                   # normal e4m3 codes
+            assert abs(vals[c] / exact - 1.0) <= 2.0 ** -4 + 1e-9
+    # Lean P on the same inputs is coarser: its worst ratio exceeds the exact-P bound
+    lean = [vals[orc.leanp_code(si, m, A, 8)] / 2.0 ** ((float(si) - float(m)) * float(A) / 8.0 + 8)
+            for si in s if orc.leanp_code(si, m, A, 8) >= 8]
+    assert max(abs(x - 1.0) for x in lean) > 2.0 ** -4
+
+
+def test_model_oracle_exactp_mode_prefix_means_and_bar():
+    codes, deq, _ = _quantized_case(15, 1, 512, 2, 2, 128)
+    qc, kc, vc, qs, ks, vs = codes
+    qz = np.zeros_like(qc)
+    o = orc.fp8_model(qz, kc, vc, qs, ks, vs, p_mode=2, rescale_log2=8.0)
+    pref = np.cumsum(deq[2], axis=1) / np.arange(1, 513)[None, :, None, None]
+    assert np.allclose(o, pref, atol=1e-12)           # equal weights: exact prefix means
+    ref = orc.attention(*deq)
+    e_exact = orc.rel_fro(orc.fp8_model(qc, kc, vc, qs, ks, vs, p_mode=2, rescale_log2=8.0), ref)
+    e_lean = orc.rel_fro(orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=8.0), ref)
+    assert 1e-4 < e_exact < 3e-2 and e_exact < e_lean
