@@ -166,6 +166,11 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--energy", type=float, default=0.0, metavar="SECONDS",
+                    help="also run each attention kernel back to back for SECONDS under NVML sampling and "
+                         "report sustained TFLOP/s, power, SM clock and TFLOP per joule")
+    ap.add_argument("--exact-p", action="store_true",
+                    help="also time the exact-P ablation (ex2 then e4m3 P) of the FP8 attention and report it")
     ap.add_argument("--hadamard", action="store_true",
                     help="rotate Q and K by the 128-point Hadamard transform in the prepass (D = 128)")
     args = ap.parse_args()
@@ -320,6 +325,45 @@ def run_ours(args, wl):
     if st != zyfa.OK:
         raise RuntimeError(f"device status {st} after timed region")
 
+    abl_ms = None
+    if args.exact_p:
+        o8x = torch.empty_like(o8)
+
+        def attn8x():
+            zyfa.attn_fwd(cq, ck, cv, o=o8x, q_scale=sq, k_scale=sk, v_scale=sv, exact_p=True)
+        for _ in range(args.warmup):
+            attn8x()
+        barrier()
+        perx = timed([attn8x], args.steps)
+        barrier()
+        abl_ms = max_over_ranks(sum(x[0] for x in perx) / args.steps)
+        if zyfa.device_status() != zyfa.OK:
+            raise RuntimeError("device wait timeout in the exact-P ablation")
+
+    energy = None
+    if args.energy > 0 and rank == 0 and bus is not None:
+        energy = {}
+        kernels = [("fp8_lean_p", attn8)] + ([("fp8_exact_p", attn8x)] if args.exact_p else []) + [("bf16", attnb)]
+        for name, fn in kernels:
+            fn(); torch.cuda.synchronize()
+            t0 = time.perf_counter(); fn(); torch.cuda.synchronize()
+            n = max(3, int(args.energy / max(time.perf_counter() - t0, 1e-4)))
+            smp = ClockSampler(bus); smp.start(); time.sleep(0.2)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            c = smp.stop() or {}
+            tf = flops / (e0.elapsed_time(e1) / n * 1e-3) / 1e12
+            w = c.get("power_w_median")
+            energy[name] = {"launches": n, "seconds": e0.elapsed_time(e1) * 1e-3, "tflops": tf,
+                            "power_w_median": w, "sm_mhz": c.get("sm_mhz"), "reasons": c.get("reasons"),
+                            "tflop_per_joule": (tf / w) if w else None}
+        if zyfa.device_status() != zyfa.OK:
+            raise RuntimeError("device wait timeout in the energy runs")
+
     ms8 = max_over_ranks(sum(a + b for a, b in per8) / args.steps)
     ms8_attn = max_over_ranks(sum(b for _, b in per8) / args.steps)
     ms8_pre = max_over_ranks(sum(a for a, _ in per8) / args.steps)
@@ -377,6 +421,10 @@ def run_ours(args, wl):
                   "fp8_vs_fp64_unquantized": orc.rel_fro(o_gpu, unq),
                   "bf16_vs_fp64": orc.rel_fro(ob_gpu, ob_ref), "prepass_codes_bit_exact": bool(gpu_codes_equal),
                   "tolerances": {"bf16": 5e-3, "fp8": 3e-2}}
+        if abl_ms is not None:
+            ox = o8x.float().cpu().numpy()[:, rows].astype(np.float64)
+            parity["exact_p_fp8_vs_fp64_dequantized"] = orc.rel_fro(ox, o_ref)
+            parity["exact_p_fp8_vs_fp64_unquantized"] = orc.rel_fro(ox, unq)
         bad = [k for k, tol in (("fp8_vs_fp64_dequantized", 3e-2), ("bf16_vs_fp64", 5e-3))
                if not parity[k] <= tol] + ([] if gpu_codes_equal else ["prepass_codes_bit_exact"])
         if bad:
@@ -412,6 +460,14 @@ def run_ours(args, wl):
                               "frac_of_datasheet": achb / DATASHEET["bf16"],
                               "frac_of_clock_scaled": (achb / clk_peak(8192)) if sm_mhz else None}},
         "fp8_breakdown_ms": {"prepass": ms8_pre, "attention": ms8_attn},
+        "energy": energy,
+        "ablation": None if abl_ms is None else {
+            "exact_p": {"kernel": f"attn_fwd_kernel<FP8,{Dqk},exact P>", "attention_ms": abl_ms,
+                        "attention_tflops": flops / (abl_ms * 1e-3) / 1e12,
+                        "frac": flops / (abl_ms * 1e-3) / 1e12 / fp8_peak,
+                        "lean_p_attention_tflops": ach8,
+                        "note": "same codes, scales, deferred max, block shift and row sum; P = e4m3(ex2(.)) "
+                                "instead of Lean P; errors under parity.exact_p_*"}},
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                 "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize_qkv -> zyfa_attn_fwd -> D2H O"},

@@ -200,6 +200,14 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// Two fp32 values -> two e4m3 codes (round to nearest even, saturating), the
+// first value's code in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
 // Two fp32 values -> bf16x2 (round to nearest even), first value in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t d;
@@ -238,7 +246,10 @@ __device__ __forceinline__ float max64(const uint32_t* s) {
   return max3f(fmaxf(a[0], a[1]), a[2], a[3]);
 }
 
-template <bool FP8, int DQK>
+// EXACTP (FP8 only): the ablation that writes P the conventional way, an
+// exponential (MUFU ex2) followed by a conversion to e4m3, with the same block
+// shift, scale factors and row sum as Lean P.
+template <bool FP8, int DQK, bool EXACTP = false>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnArgs a) {
   using Cf = AttnCfg<FP8, DQK>;
   extern __shared__ uint8_t smem_raw[];
@@ -580,15 +591,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         }
         if (FP8) {
           const int jb = leanp_block_shift(m, h ? bmx1 : bmx0, A);
-          const float Bb = leanp_row_offset(m, A, jb);
-          const float a256 = __fmul_rn(A, 0.00390625f), b256 = __fmul_rn(Bb, 0.00390625f);
           uint32_t p[16];
+          if (EXACTP) {
+            // p = exp2((s - m) A / 8 + j): one FMA, MUFU ex2, then e4m3
+            const float a8 = __fmul_rn(A, 0.125f);
+            const float b8 = __fmaf_rn(-m, a8, static_cast<float>(jb));
 #pragma unroll
-          for (int w = 0; w < 16; ++w)
-            p[w] = pack4_low_bytes(leanp_code_word(__uint_as_float(r[4 * w]), a256, b256),
-                                   leanp_code_word(__uint_as_float(r[4 * w + 1]), a256, b256),
-                                   leanp_code_word(__uint_as_float(r[4 * w + 2]), a256, b256),
-                                   leanp_code_word(__uint_as_float(r[4 * w + 3]), a256, b256));
+            for (int w = 0; w < 16; ++w) {
+              const float e0 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w]), a8, b8));
+              const float e1 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w + 1]), a8, b8));
+              const float e2 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w + 2]), a8, b8));
+              const float e3 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w + 3]), a8, b8));
+              p[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
+            }
+          } else {
+            const float Bb = leanp_row_offset(m, A, jb);
+            const float a256 = __fmul_rn(A, 0.00390625f), b256 = __fmul_rn(Bb, 0.00390625f);
+#pragma unroll
+            for (int w = 0; w < 16; ++w)
+              p[w] = pack4_low_bytes(leanp_code_word(__uint_as_float(r[4 * w]), a256, b256),
+                                     leanp_code_word(__uint_as_float(r[4 * w + 1]), a256, b256),
+                                     leanp_code_word(__uint_as_float(r[4 * w + 2]), a256, b256),
+                                     leanp_code_word(__uint_as_float(r[4 * w + 3]), a256, b256));
+          }
           tmem_st16p(tp + 16 * h, p);
           // E8M0 scale code 127 - j for both 32-key MX blocks of this 64-key block
           sfw |= static_cast<uint32_t>((127 - jb) * 0x0101) << (16 * h);

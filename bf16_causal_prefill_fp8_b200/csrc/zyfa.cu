@@ -59,7 +59,7 @@ EncodeTiledFn encode_fn() {
 
 struct DeviceInfo {
   int sms = 0;
-  bool attr_set[4] = {false, false, false, false};
+  bool attr_set[6] = {false, false, false, false, false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -79,7 +79,7 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int el, 
             swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool FP8, int DQK>
+template <bool FP8, int DQK, bool EXACTP = false>
 int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int S,
                 const float* qs, const float* ks, const float* vs, cudaStream_t stream, int dev,
                 int inst) {
@@ -121,7 +121,7 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int
     if (di.sms == 0 && cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return ZYFA_ERR_CUDA;
     if (!di.attr_set[inst]) {
-      if (cudaFuncSetAttribute(attn_fwd_kernel<FP8, DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(attn_fwd_kernel<FP8, DQK, EXACTP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cf::SMEM) != cudaSuccess)
         return ZYFA_ERR_CUDA;
       di.attr_set[inst] = true;
@@ -129,7 +129,7 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int
   }
   const long long units = static_cast<long long>(B) * Hq * a.Tq;
   const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
-  attn_fwd_kernel<FP8, DQK><<<grid, kAttnThreads, Cf::SMEM, stream>>>(a);
+  attn_fwd_kernel<FP8, DQK, EXACTP><<<grid, kAttnThreads, Cf::SMEM, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
@@ -185,9 +185,9 @@ extern "C" void zyfa_set_wait_timeout_ns(unsigned long long ns) {
   g_timeout_ns.store(ns, std::memory_order_relaxed);
 }
 
-extern "C" int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq,
-                             int Hkv, int S, int Dqk, int Dv, int dtype, const float* q_scale,
-                             const float* k_scale, const float* v_scale, void* stream) {
+static int attn_validate(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int S,
+                         int Dqk, int Dv, int dtype, const float* q_scale, const float* k_scale,
+                         const float* v_scale) {
   if (!q || !k || !v || !o) return ZYFA_ERR_NULL_PTR;
   if (B < 1 || S < 1 || Hq < 1 || Hkv < 1) return ZYFA_ERR_BAD_SHAPE;
   if (Hq % Hkv != 0) return ZYFA_ERR_BAD_GQA;
@@ -200,6 +200,14 @@ extern "C" int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* 
   if (dtype == ZYFA_FP8_E4M3 &&
       (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4)))
     return ZYFA_ERR_MISALIGNED;
+  return ZYFA_OK;
+}
+
+extern "C" int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq,
+                             int Hkv, int S, int Dqk, int Dv, int dtype, const float* q_scale,
+                             const float* k_scale, const float* v_scale, void* stream) {
+  const int bad = attn_validate(q, k, v, o, B, Hq, Hkv, S, Dqk, Dv, dtype, q_scale, k_scale, v_scale);
+  if (bad != ZYFA_OK) return bad;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -209,6 +217,18 @@ extern "C" int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* 
   }
   if (Dqk == 128) return launch_attn<false, 128>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 2);
   return launch_attn<false, 192>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 3);
+}
+
+extern "C" int zyfa_attn_fwd_fp8_exact_p(const void* q, const void* k, const void* v, void* o, int B, int Hq,
+                                         int Hkv, int S, int Dqk, int Dv, const float* q_scale,
+                                         const float* k_scale, const float* v_scale, void* stream) {
+  const int bad = attn_validate(q, k, v, o, B, Hq, Hkv, S, Dqk, Dv, ZYFA_FP8_E4M3, q_scale, k_scale, v_scale);
+  if (bad != ZYFA_OK) return bad;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (Dqk == 128) return launch_attn<true, 128, true>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 4);
+  return launch_attn<true, 192, true>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 5);
 }
 
 extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* scale, int B, int S, int H,

@@ -38,6 +38,8 @@ def lib() -> ctypes.CDLL:
         p, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.zyfa_attn_fwd.restype = i
         L.zyfa_attn_fwd.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, p, p, p]
+        L.zyfa_attn_fwd_fp8_exact_p.restype = i
+        L.zyfa_attn_fwd_fp8_exact_p.argtypes = [p, p, p, p, i, i, i, i, i, i, p, p, p, p]
         L.zyfa_quantize.restype = i
         L.zyfa_quantize.argtypes = [p, i, p, p, i, i, i, i, i, p]
         L.zyfa_quantize_qkv.restype = i
@@ -87,10 +89,11 @@ def _dev(t, name):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
-def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=None):
+def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=None, exact_p=False):
     """Causal attention forward.  q [B,S,Hq,Dqk], k [B,S,Hkv,Dqk], v [B,S,Hkv,Dv];
     bf16 tensors (BF16 path) or uint8 / float8_e4m3fn codes with fp32 scales
-    [B,H] (FP8 path).  Returns o [B,S,Hq,Dv] bf16."""
+    [B,H] (FP8 path).  exact_p (FP8 only): the exact-P ablation
+    (zyfa_attn_fwd_fp8_exact_p) instead of Lean P.  Returns o [B,S,Hq,Dv] bf16."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
     if q.dtype == torch.bfloat16:
@@ -109,6 +112,13 @@ def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=N
             _dev(t, n)
             if t.dtype != torch.float32:
                 raise ValueError(f"{n} must be fp32")
+    if exact_p:
+        if dt != FP8_E4M3:
+            raise ValueError("exact_p applies to the FP8 path only")
+        st = lib().zyfa_attn_fwd_fp8_exact_p(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, S, Dqk, Dv,
+                                             _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream(stream))
+        _check(st, "zyfa_attn_fwd_fp8_exact_p")
+        return o
     st = lib().zyfa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, S, Dqk, Dv, dt,
                              _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream(stream))
     _check(st, "zyfa_attn_fwd")

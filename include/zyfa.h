@@ -98,6 +98,23 @@ int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
                   const float* v_scale, void* stream);
 
 /*
+ * zyfa_attn_fwd_fp8_exact_p -- the exact-P ablation of the FP8 path: the
+ * pages' Lean P (the-ai.news "Zyphra presenteert ZYFA", section "Drie
+ * technieken om de bottleneck te omzeilen"; spke.com "Zyphra ZYFA", section
+ * "Lean P") replaces the conventional way of writing P in FP8, an
+ * exponential followed by a conversion to e4m3.  This entry runs that
+ * conventional way in the same kernel: each probability is
+ * e4m3 RNE-satfinite of ex2((s - m) A / 8 + j), with the same deferred
+ * reference max, the same 64-key block shift j and E8M0 scales, and the same
+ * row sum over the rounded P, so the two can be compared on speed and error.
+ * Arguments, layouts, ownership and errors as zyfa_attn_fwd with
+ * dtype = ZYFA_FP8_E4M3.
+ */
+int zyfa_attn_fwd_fp8_exact_p(const void* q, const void* k, const void* v, void* o, int B, int Hq,
+                              int Hkv, int S, int Dqk, int Dv, const float* q_scale,
+                              const float* k_scale, const float* v_scale, void* stream);
+
+/*
  * zyfa_quantize -- the prepass: per-(batch, head) FP8 e4m3 quantization, with
  * an optional Hadamard rotation for Q and K (spke.com "Zyphra ZYFA", accuracy
  * section: most FP8 error comes from quantizing Q, K and V, and a Hadamard

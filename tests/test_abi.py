@@ -15,7 +15,8 @@ def L():
 
 def test_every_declared_symbol_is_exported(L):
     names = zyfa.declared_symbols()
-    assert set(names) >= {"zyfa_attn_fwd", "zyfa_quantize", "zyfa_quantize_qkv", "zyfa_status_string",
+    assert set(names) >= {"zyfa_attn_fwd", "zyfa_attn_fwd_fp8_exact_p", "zyfa_quantize", "zyfa_quantize_qkv",
+                          "zyfa_status_string",
                           "zyfa_device_status",
                           "zyfa_leanp_codes", "zyfa_selftest_wait_timeout", "zyfa_set_wait_timeout_ns"}
     for n in names:
@@ -54,6 +55,17 @@ def test_attn_argument_errors(L):
     assert _attn(L, o=FAKE + 2) == -5
     assert _attn(L, dt=1, qs=FAKE + 1) == -5
     assert _attn(L, B=1 << 20, Hq=1 << 12, Hkv=1, S=1 << 16) == -2
+
+
+def test_exact_p_argument_errors(L):
+    def e(q=FAKE, o=FAKE, B=1, Hq=2, Hkv=2, S=128, Dqk=128, Dv=128, qs=None):
+        return L.zyfa_attn_fwd_fp8_exact_p(q, FAKE, FAKE, o, B, Hq, Hkv, S, Dqk, Dv, qs, None, None, None)
+    assert e(q=None) == -1
+    assert e(S=0) == -2
+    assert e(Hq=3) == -4
+    assert e(Dqk=64) == -3
+    assert e(o=FAKE + 4) == -5
+    assert e(qs=FAKE + 2) == -5
 
 
 def test_quantize_argument_errors(L):

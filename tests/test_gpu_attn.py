@@ -11,7 +11,7 @@ import torch
 from bf16_causal_prefill_fp8_b200 import zyfa
 from oracle import oracle as orc
 
-from helpers import (TOL_BF16, TOL_FP8, TOL_FP8_MODEL, fp8_references, inputs, run_bf16,
+from helpers import (RESCALE_LOG2, TOL_BF16, TOL_FP8, TOL_FP8_MODEL, fp8_references, inputs, run_bf16,
                      run_fp8)
 
 pytestmark = pytest.mark.gpu
@@ -118,6 +118,30 @@ def test_many_units_per_cta(kind, q_gain):
     assert e_b <= TOL_BF16
     ob2, _ = run_bf16(q, k, v)
     assert np.array_equal(ob2, ob)
+
+
+@pytest.mark.parametrize("shape", [(1, 512, 2, 2, 128, 128), (2, 700, 4, 2, 128, 128), (1, 300, 2, 2, 192, 128)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_fp8_exact_p_ablation(shape):
+    """Exact P (ex2 then e4m3) in the same kernel: within the FP8 bar of fp64
+    attention, close to the CPU replay of the same route, and no less accurate
+    than Lean P on the same codes."""
+    import torch
+    B, S, Hq, Hkv, Dqk, Dv = shape
+    q, k, v = inputs(47, B, S, Hq, Hkv, Dqk, Dv, kind="outlier_k" if Dqk == 128 else "mla")
+    o_lean, codes = run_fp8(q, k, v)
+    (qc, qs), (kc, ks), (vc, vs) = codes
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    o = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs), exact_p=True)
+    torch.cuda.synchronize()
+    o = o.float().cpu().numpy().astype(np.float64)
+    ref, _ = fp8_references(codes)
+    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, p_mode=2, rescale_log2=RESCALE_LOG2)
+    e_ref, e_model, e_lean = orc.rel_fro(o, ref), orc.rel_fro(o, model), orc.rel_fro(o_lean, ref)
+    print(f"exact-P {shape}: vs fp64 {e_ref:.3e}  vs exact-P model {e_model:.3e}  (Lean P vs fp64 {e_lean:.3e})")
+    assert e_ref <= TOL_FP8 and e_model <= TOL_FP8_MODEL
+    assert e_ref <= e_lean * 1.05
+    assert zyfa.device_status() == zyfa.OK
 
 
 def test_fp8_hadamard_prepass_path():
