@@ -25,6 +25,8 @@
  *       against torch's float8_e4m3fn and ml_dtypes decoders, the power-of-two
  *       ladder code(2^k) = 8k + 56 (tests/golden/e4m3_pow2_ladder.txt), RNE ties.
  *   oracle_fwht128 : against scipy.linalg.hadamard(128)/sqrt(128); H H^T = I.
+ *   oracle_fwht64 : against scipy.linalg.hadamard(64)/8; with the 128-point
+ *       block it keeps Q K^T of Dqk 192 rows (rotation invariance).
  *   oracle_quantize : amax/448 scale and codes against a brute-force nearest
  *       search over the 127 finite non-negative e4m3 values; rotation
  *       invariance of Q K^T in fp64.
@@ -124,6 +126,32 @@ void oracle_fwht128(float *x)
     for (i = 0; i < 128; ++i) x[i] = x[i] * norm;
 }
 
+/* The 64-point companion for the MLA shape (reading: Dqk 192 = 128 + 64 is */
+/* rotated block-diagonally, H128/sqrt(128) on dims 0..127 and              */
+/* H64/sqrt(64) on dims 128..191; orthonormal, so Q K^T is unchanged).      */
+/* Stages of stride 1, 2, ..., 32 in fp32, then one multiply by 2^-3.       */
+void oracle_fwht64(float *x)
+{
+    int h, i;
+    for (h = 1; h < 64; h <<= 1) {
+        for (i = 0; i < 64; ++i) {
+            if ((i & h) == 0) {
+                float a = x[i], b = x[i + h];
+                x[i] = a + b;
+                x[i + h] = a - b;
+            }
+        }
+    }
+    for (i = 0; i < 64; ++i) x[i] = x[i] * 0.125f;
+}
+
+/* The rotation the prepass applies to a row of D = 128 or 192 values. */
+static void oracle_rotate_row(float *row, int D)
+{
+    oracle_fwht128(row);
+    if (D == 192) oracle_fwht64(row + 128);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Per-(batch, head) FP8 quantization.  [ZH] "ZYFA 的性能与精度数据": FP8     */
 /* attention maps values into the e4m3 range with per-tensor or per-head    */
@@ -131,7 +159,8 @@ void oracle_fwht128(float *x)
 /* quantizing Q, K and V.                                                   */
 /*   x      : [B, S, H, D] fp32 (bf16 inputs are widened exactly by caller) */
 /*   amax   : max |x'| over (s, d) of one (b, h), x' = rotated row when     */
-/*            hadamard != 0 (D must be 128), else x' = x                    */
+/*            hadamard != 0 (D 128: H128; D 192: H128 on dims 0..127 and  */
+/*            H64 on dims 128..191), else x' = x                            */
 /*   scale  : amax / 448 in fp32 (IEEE division); 1 when amax == 0          */
 /*   code   : e4m3 RNE satfinite of fl32(x' / scale) (IEEE division)        */
 /* Returns 0, or -1 for bad arguments.                                      */
@@ -141,7 +170,7 @@ int oracle_quantize(const float *x, int B, int S, int H, int D, int hadamard,
 {
     int b, h;
     if (!x || !codes || !scale || B < 1 || S < 1 || H < 1 || D < 1) return -1;
-    if (hadamard && D != 128) return -1;
+    if (hadamard && D != 128 && D != 192) return -1;
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (b = 0; b < B; ++b) {
         for (h = 0; h < H; ++h) {
@@ -151,7 +180,7 @@ int oracle_quantize(const float *x, int B, int S, int H, int D, int hadamard,
             for (s = 0; s < S; ++s) {
                 const float *src = x + (((size_t)b * S + s) * H + h) * (size_t)D;
                 for (d = 0; d < D; ++d) row[d] = src[d];
-                if (hadamard) oracle_fwht128(row);
+                if (hadamard) oracle_rotate_row(row, D);
                 for (d = 0; d < D; ++d) {
                     float a = fabsf(row[d]);
                     if (a > amax) amax = a;
@@ -162,7 +191,7 @@ int oracle_quantize(const float *x, int B, int S, int H, int D, int hadamard,
             for (s = 0; s < S; ++s) {
                 size_t off = (((size_t)b * S + s) * H + h) * (size_t)D;
                 for (d = 0; d < D; ++d) row[d] = x[off + d];
-                if (hadamard) oracle_fwht128(row);
+                if (hadamard) oracle_rotate_row(row, D);
                 for (d = 0; d < D; ++d)
                     codes[off + d] = (uint8_t)oracle_e4m3_from_f32(row[d] / sc);
             }

@@ -25,6 +25,8 @@ def lib():
         L.oracle_e4m3_value.argtypes = [ctypes.c_uint]
         L.oracle_e4m3_from_f32.restype = ctypes.c_uint
         L.oracle_e4m3_from_f32.argtypes = [c_f]
+        L.oracle_fwht64.restype = None
+        L.oracle_fwht64.argtypes = [c_p]
         L.oracle_fwht128.restype = None
         L.oracle_fwht128.argtypes = [c_p]
         L.oracle_quantize.restype = c_i
@@ -88,6 +90,17 @@ def dequantize(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
 
 
 # --- Hadamard and quantizer --------------------------------------------------
+
+def fwht64(x) -> np.ndarray:
+    """Orthonormal 64-point transform of each row of x [..., 64] (fp32 steps)."""
+    x = _c(x, np.float32).copy()
+    flat = x.reshape(-1, 64)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        lib().oracle_fwht64(_ptr(row))
+        flat[r] = row
+    return flat.reshape(x.shape)
+
 
 def fwht128(x) -> np.ndarray:
     """Orthonormal 128-point transform of each row of x [..., 128] (fp32 steps)."""

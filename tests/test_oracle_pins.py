@@ -373,3 +373,31 @@ def test_model_oracle_exactp_mode_prefix_means_and_bar():
     e_exact = orc.rel_fro(orc.fp8_model(qc, kc, vc, qs, ks, vs, p_mode=2, rescale_log2=8.0), ref)
     e_lean = orc.rel_fro(orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=8.0), ref)
     assert 1e-4 < e_exact < 3e-2 and e_exact < e_lean
+
+
+# --- MLA rotation (H128 on the first 128 dims, H64 on the last 64) --------------------
+
+def test_fwht64_matches_scipy_and_is_orthonormal():
+    import scipy.linalg
+    x = synth.gaussian(31, 1, (5, 64))
+    ref = (x.astype(np.float64) @ scipy.linalg.hadamard(64).T) / 8.0
+    assert np.allclose(orc.fwht64(x), ref, rtol=0, atol=1e-5)
+    eye = orc.fwht64(np.eye(64, dtype=np.float32))
+    assert np.allclose(eye @ eye.T, np.eye(64), atol=1e-6)
+
+
+def test_quantize_192_rotation_is_block_diagonal_and_keeps_qk():
+    """Dqk 192 with hadamard: dims 0..127 by H128, 128..191 by H64 (pinned
+    through the codes: rotating first and quantizing without the flag gives the
+    same bytes), and the rotation leaves Q K^T unchanged in fp64."""
+    import scipy.linalg
+    q = synth.gaussian(32, 1, (1, 40, 2, 192)) * np.float32(2.0)
+    c_rot, s_rot = orc.quantize(q, hadamard=True)
+    pre = np.concatenate([orc.fwht128(q[..., :128]), orc.fwht64(q[..., 128:])], axis=-1)
+    c_pre, s_pre = orc.quantize(pre, hadamard=False)
+    assert np.array_equal(c_rot, c_pre) and np.array_equal(s_rot.view(np.uint32), s_pre.view(np.uint32))
+    H = np.zeros((192, 192))
+    H[:128, :128] = scipy.linalg.hadamard(128) / np.sqrt(128.0)
+    H[128:, 128:] = scipy.linalg.hadamard(64) / 8.0
+    a = q[0, :, 0].astype(np.float64); b = q[0, :, 1].astype(np.float64)
+    assert np.allclose((a @ H.T) @ (b @ H.T).T, a @ b.T, atol=1e-9)
