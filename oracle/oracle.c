@@ -252,6 +252,42 @@ int oracle_attention_rows(const double *q, const double *k, const double *v,
     return 0;
 }
 
+/* Log-sum-exp of each row's causal scores in fp64, the plain definition:   */
+/*   lse_i = max_j s_j + log(sum_j exp(s_j - max_j s_j)),  s_j as above.    */
+/* lse [B, Hq, nrows].                                                      */
+int oracle_attention_lse_rows(const double *q, const double *k, int B, int Hq, int Hkv, int S, int Dqk,
+                              double sm_scale, const int *rows, int nrows, double *lse)
+{
+    int b;
+    if (!q || !k || !lse || B < 1 || Hq < 1 || Hkv < 1 || S < 1) return -1;
+    if (Hq % Hkv != 0 || Dqk < 1) return -1;
+    if (!rows) nrows = S;
+    for (b = 0; b < B; ++b) {
+        int task;
+#pragma omp parallel for schedule(dynamic, 4)
+        for (task = 0; task < Hq * nrows; ++task) {
+            int hq = task / nrows, r = task % nrows;
+            int i = rows ? rows[r] : r;
+            int kvh = hq / (Hq / Hkv);
+            double *s = (double *)malloc(sizeof(double) * (size_t)(i + 1));
+            const double *qi = q + (((size_t)b * S + i) * Hq + hq) * (size_t)Dqk;
+            double mx = -INFINITY, den = 0.0;
+            int j, d;
+            for (j = 0; j <= i; ++j) {
+                const double *kj = k + (((size_t)b * S + j) * Hkv + kvh) * (size_t)Dqk;
+                double dot = 0.0;
+                for (d = 0; d < Dqk; ++d) dot += qi[d] * kj[d];
+                s[j] = dot * sm_scale;
+                if (s[j] > mx) mx = s[j];
+            }
+            for (j = 0; j <= i; ++j) den += exp(s[j] - mx);
+            lse[((size_t)b * Hq + hq) * (size_t)nrows + r] = mx + log(den);
+            free(s);
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Lean P, bit level ([NL] "Drie technieken om de bottleneck te omzeilen";  */
 /* [JA] "Lean P: 指数関数の代わりに1回の乗算加算" and "ブロックごとの       */
@@ -351,6 +387,7 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 /* Every block shift j must stay >= 0 (weights <= 448, E8M0 scale <= 1):   */
 /* true for the exact max (j >= 8) and for the deferred one (j >= 8 - r);   */
 /* a violation returns -2.                                                  */
+/* lse (may be NULL) [B, Hq, nrows]: ln 2 (m A/8 + log2 l) at the last tile. */
 /* The row sum l comes from the rounded weights, like the extra matrix      */
 /* instruction per block on the pages.  Output o_i = O / l * v_s.           */
 /* q [B,S,Hq,Dqk], k [B,S,Hkv,Dqk], v [B,S,Hkv,Dv] codes; q_s [B*Hq],       */
@@ -360,7 +397,7 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
                           const float *q_s, const float *k_s, const float *v_s,
                           int B, int Hq, int Hkv, int S, int Dqk, int Dv,
                           int p_mode, float rescale_log2,
-                          const int *rows, int nrows, double *o)
+                          const int *rows, int nrows, double *o, double *lse)
 {
     int b, shift_err = 0;
     if (!qc || !kc || !vc || !q_s || !k_s || !v_s || !o) return -1;
@@ -447,6 +484,11 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
             for (d = 0; d < Dv; ++d)
                 o[(((size_t)b * nrows + r) * Hq + hq) * (size_t)Dv + d] =
                     acc[d] / l * (double)v_s[(size_t)b * Hkv + kvh];
+            /* the weights are 2^((s - m) A / 8) relative to the reference m:  */
+            /* log-sum-exp of the scaled scores = ln 2 (m A / 8 + log2 l)      */
+            if (lse)
+                lse[((size_t)b * Hq + hq) * (size_t)nrows + r] =
+                    0.69314718055994530942 * ((double)m * (double)A / 8.0 + log2(l));
             free(qv);
             free(acc);
         }

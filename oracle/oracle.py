@@ -44,7 +44,9 @@ def lib():
         L.oracle_leanp_batch.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i, c_p, c_p]
         L.oracle_fp8_model_rows.restype = c_i
         L.oracle_fp8_model_rows.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i,
-                                            c_i, c_i, c_i, c_f, c_p, c_i, c_p]
+                                            c_i, c_i, c_i, c_f, c_p, c_i, c_p, c_p]
+        L.oracle_attention_lse_rows.restype = c_i
+        L.oracle_attention_lse_rows.argtypes = [c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_d, c_p, c_i, c_p]
         L.oracle_exactp_code.restype = ctypes.c_uint
         L.oracle_exactp_code.argtypes = [c_f, c_f, c_f, c_i, c_i]
         L.oracle_num_threads.restype = c_i
@@ -145,6 +147,23 @@ def attention(q, k, v, sm_scale=None, rows=None) -> np.ndarray:
     return o
 
 
+def attention_lse(q, k, sm_scale=None, rows=None) -> np.ndarray:
+    """Log-sum-exp of each row's causal scores in fp64: lse [B, Hq, S or len(rows)]."""
+    q = _c(q, np.float64); k = _c(k, np.float64)
+    B, S, Hq, Dqk = q.shape
+    Hkv = k.shape[2]
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(Dqk)
+    r = None if rows is None else _c(rows, np.int32)
+    n = S if rows is None else len(r)
+    lse = np.empty((B, Hq, n), dtype=np.float64)
+    rc = lib().oracle_attention_lse_rows(_ptr(q), _ptr(k), B, Hq, Hkv, S, Dqk, float(sm_scale), _ptr(r), n,
+                                         _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attention_lse_rows: bad arguments")
+    return lse
+
+
 # --- Lean P ------------------------------------------------------------------
 
 def leanp_slope(q_s: float, k_s: float, dqk: int) -> np.float32:
@@ -175,13 +194,15 @@ def leanp_batch(s, m, bmax, A, masked=None):
     return code, j
 
 
-def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=0.0, p_mode=None) -> np.ndarray:
+def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=0.0, p_mode=None,
+              return_lse=False):
     """The FP8 pipeline replayed on the CPU (see oracle.c).  Codes uint8 BSHD,
     scales fp32 [B,H].  rescale_log2 = 0: exact running max; > 0: the reference
     max moves only when a tile max exceeds it by more than that many binades.
     p_mode: 0 Lean-P codes (default), 1 exact fp64 weights (exact_p=True),
     2 exact exp2 rounded to e4m3 (the exact-P ablation).
-    Returns o fp64 [B, S or len(rows), Hq, Dv]."""
+    Returns o fp64 [B, S or len(rows), Hq, Dv] (and lse [B, Hq, rows] with
+    return_lse: ln 2 (m A/8 + log2 l) from the replay's own row sum)."""
     if p_mode is None:
         p_mode = 1 if exact_p else 0
     qc = _c(qc, np.uint8); kc = _c(kc, np.uint8); vc = _c(vc, np.uint8)
@@ -191,13 +212,15 @@ def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=
     r = None if rows is None else _c(rows, np.int32)
     n = S if rows is None else len(r)
     o = np.empty((B, n, Hq, Dv), dtype=np.float64)
+    lse = np.empty((B, Hq, n), dtype=np.float64) if return_lse else None
     rc = lib().oracle_fp8_model_rows(_ptr(qc), _ptr(kc), _ptr(vc), _ptr(q_s), _ptr(k_s), _ptr(v_s),
-                                     B, Hq, Hkv, S, Dqk, Dv, int(p_mode), ctypes.c_float(rescale_log2), _ptr(r), n, _ptr(o))
+                                     B, Hq, Hkv, S, Dqk, Dv, int(p_mode), ctypes.c_float(rescale_log2), _ptr(r), n, _ptr(o),
+                                     _ptr(lse))
     if rc == -2:
         raise ArithmeticError("oracle_fp8_model_rows: a block shift fell below 0 (reference max too stale)")
     if rc != 0:
         raise ValueError("oracle_fp8_model_rows: bad arguments")
-    return o
+    return (o, lse) if return_lse else o
 
 
 def rel_fro(a, b) -> float:

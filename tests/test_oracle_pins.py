@@ -401,3 +401,34 @@ def test_quantize_192_rotation_is_block_diagonal_and_keeps_qk():
     H[128:, 128:] = scipy.linalg.hadamard(64) / 8.0
     a = q[0, :, 0].astype(np.float64); b = q[0, :, 1].astype(np.float64)
     assert np.allclose((a @ H.T) @ (b @ H.T).T, a @ b.T, atol=1e-9)
+
+
+# --- log-sum-exp output --------------------------------------------------------------
+
+def test_attention_lse_closed_forms_and_torch():
+    import torch
+    q, k, _ = synth.make_qkv(33, 1, 150, 4, 2, 128, 128)
+    lse = orc.attention_lse(q, k)
+    sm = 1.0 / np.sqrt(128.0)
+    # row 0 has one key: lse = its scaled score
+    s00 = (q[0, 0].astype(np.float64) * k[0, 0, np.arange(4) // 2].astype(np.float64)).sum(-1) * sm
+    assert np.allclose(lse[0, :, 0], s00, atol=1e-12)
+    # Q = 0: every live score is 0, lse_i = ln(i + 1)
+    lz = orc.attention_lse(np.zeros_like(q), k)
+    assert np.allclose(lz[0], np.log(np.arange(1, 151))[None, :], atol=1e-12)
+    # torch's logsumexp over the masked scores (GQA by repeat)
+    qt = torch.from_numpy(q.astype(np.float64))[0].transpose(0, 1)                 # [H, S, D]
+    kt = torch.from_numpy(k.astype(np.float64))[0].transpose(0, 1).repeat_interleave(2, dim=0)
+    sc = qt @ kt.transpose(1, 2) * sm
+    sc = sc.masked_fill(torch.triu(torch.ones(150, 150, dtype=torch.bool), 1), float("-inf"))
+    assert np.allclose(lse[0], torch.logsumexp(sc, dim=-1).numpy(), atol=1e-10)
+
+
+def test_model_lse_with_exact_weights_equals_definition():
+    codes, deq, _ = _quantized_case(16, 1, 300, 2, 2, 128)
+    qc, kc, vc, qs, ks, vs = codes
+    for r in (0.0, 8.0):
+        _, lse = orc.fp8_model(qc, kc, vc, qs, ks, vs, p_mode=1, rescale_log2=r, return_lse=True)
+        assert np.allclose(lse, orc.attention_lse(deq[0], deq[1]), atol=1e-6)
+    _, lse_lean = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=8.0, return_lse=True)
+    assert np.abs(lse_lean - orc.attention_lse(deq[0], deq[1])).max() < 0.07   # Lean P weights: within ~6 %
