@@ -172,7 +172,7 @@ def main():
     ap.add_argument("--exact-p", action="store_true",
                     help="also time the exact-P ablation (ex2 then e4m3 P) of the FP8 attention and report it")
     ap.add_argument("--hadamard", action="store_true",
-                    help="rotate Q and K by the 128-point Hadamard transform in the prepass (D = 128)")
+                    help="rotate Q and K by the Hadamard transform in the prepass (H128; H128 + H64 for Dqk 192)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = dict(synth.WORKLOADS[args.workload])

@@ -51,6 +51,7 @@ struct AttnArgs {
   CUtensorMap map_k_tail;
   CUtensorMap map_v;
   __nv_bfloat16* o;
+  float* lse;              // [B, Hq, S] natural-log sum of exp(scaled scores) per row, or null
   const float* q_scale;    // [B*Hq] or null (1.0); FP8 only
   const float* k_scale;    // [B*Hkv] or null
   const float* v_scale;    // [B*Hkv] or null
@@ -96,7 +97,8 @@ struct AttnCfg {
   static constexpr int OFF_ONES = OFF_V + STV * VB;   // FP8: 16 x 128 bytes of e4m3 1.0
   static constexpr int OFF_SF = OFF_ONES + (FP8 ? 2048 : 0);   // FP8: NPB x 512 B scale factors
   static constexpr int OFF_ALPHA = OFF_SF + (FP8 ? NPB * 512 : 0);  // NPB x 128 fp32 rescale factors
-  static constexpr int OFF_LFIN = OFF_ALPHA + NPB * 512;  // BF16 final partial row sums, per group (2 x 128 fp32)
+  static constexpr int OFF_LFIN = OFF_ALPHA + NPB * 512;  // BF16: final partial row sums per group (2 x 128 fp32);
+                                                          // FP8: final reference max per unit (4 x 128 fp32)
   static constexpr int OFF_XCH = OFF_LFIN + 2048;    // running max per group (2 x 128) + BF16 final max per group (2 x 128)
   static constexpr int OFF_BAR = OFF_XCH + 2048;
   // Barriers (phase bookkeeping: every waiter is at most one phase behind,
@@ -638,6 +640,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       if (FP8) {
         sf_s[pbuf * 128 + sf_row] = sfw;
         fence_proxy_async_smem();   // the copy to TMEM reads it through the async proxy
+        // the unit's final reference max, for the log-sum-exp (slot per unit
+        // mod 4: unit u+4's last tile comes after P V of unit u+1's first
+        // tile, which waits for the epilogue of unit u that reads this slot)
+        if (t.j == t.nkv - 1) lfin_s[(t.u & 3) * 128 + row] = m;
       } else {
         // this group's partial row sum, kept relative to the newest max
         l = l * ex2_approx(__fmul_rn(m_own - m, A)) + rowsum;
@@ -700,12 +706,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       // ---- epilogue: O / l (* v_scale) -> bf16, rows past S are not written
       if (!(ok = warp_wait(bar(Cf::OFIN), u_it & 1, ctl))) break;
       tc_fence_after();
-      float inv;
+      float inv, lse_log2;   // lse_log2: log-sum-exp of the scaled scores, in binades
+      const int grow = qt * 128 + row;
       if (FP8) {
         const float vsc = a.v_scale ? a.v_scale[b * a.Hkv + hkv] : 1.0f;
         const float lv = __uint_as_float(tmem_ld1(lb + Cf::TL));
         tmem_wait_ld();
         inv = vsc / lv;
+        if (a.lse) {   // weights are 2^((s - m) A / 8) against the final reference m
+          const float qs = a.q_scale ? a.q_scale[b * a.Hq + hq] : 1.0f;
+          const float ks = a.k_scale ? a.k_scale[b * a.Hkv + hkv] : 1.0f;
+          const float A8 = __fmul_rn(leanp_slope(qs, ks, a.C), 0.125f);
+          lse_log2 = __fmaf_rn(lfin_s[(u_it & 3) * 128 + row], A8, log2f(lv));
+        }
       } else {
         // the group of the unit's last tile holds the final max
         const bool last1 = ((kv_it - 1) & 1) != 0;
@@ -714,8 +727,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         float lt = l_last;
         if (nkv >= 2) lt += l_oth * ex2_approx(__fmul_rn(m_oth - m_last, a.C));
         inv = 1.0f / lt;
+        if (a.lse) lse_log2 = __fmaf_rn(m_last, a.C, log2f(lt));
       }
-      const int grow = qt * 128 + row;
+      if (a.lse && grow < a.S)
+        a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.S + grow] = lse_log2 * 0.69314718055994530942f;
       __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.S + grow) * a.Hq + hq) * 128;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {

@@ -117,6 +117,34 @@ __device__ __forceinline__ void fwht128_half(float (&x)[8], int li) {
   for (int i = 0; i < 8; ++i) x[i] = x[i] * kFwhtNorm;
 }
 
+// Rotated rows of D = 192 (MLA: H128 on dims 0..127, H64 on 128..191), one
+// row per warp: lane l < 24 holds dims 8l .. 8l+7 (lanes 0-15 the 128-point
+// block, 16-23 the 64-point block), lanes 24-31 zeros so every shuffle is
+// full-mask.  Each block runs its own transform's stages in order (strides
+// 1, 2, 4 in registers, then 8, 16, 32 across lanes, and 64 for the 128-point
+// block only), then its own normalisation (2^-3.5, 2^-3).
+__device__ __forceinline__ void fwht192_warp(float (&x)[8], int lane) {
+  float a, b;
+#pragma unroll
+  for (int st = 1; st < 8; st <<= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((i & st) == 0) { a = x[i]; b = x[i + st]; x[i] = a + b; x[i + st] = a - b; }
+  const bool b128 = lane < 16;
+#pragma unroll
+  for (int sh = 1; sh < 16; sh <<= 1) {   // strides 8, 16, 32 (both blocks), 64 (128-point block)
+    const bool upper = (lane & sh) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[i], sh);
+      if (sh < 8 || b128) x[i] = upper ? (o - x[i]) : (x[i] + o);
+    }
+  }
+  const float norm = b128 ? kFwhtNorm : 0.125f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = x[i] * norm;
+}
+
 struct QuantArgs {
   const void* x;
   uint8_t* out;
@@ -133,7 +161,31 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
   __syncthreads();
   const uint32_t HD = static_cast<uint32_t>(a.H) * a.D;
   const T* base = static_cast<const T*>(a.x) + (static_cast<size_t>(b) * a.S + r0) * HD;
-  if (HAD) {
+  if (HAD && a.D == 192) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nrow = (r1 - r0) * a.H;
+    for (int v0 = warp * kUnroll; v0 < nrow; v0 += nw * kUnroll) {
+      float x[kUnroll][8];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + u < nrow && lane < 24) load8<T>(base + static_cast<size_t>(v0 + u) * 192 + 8 * lane, x[u]);
+        else
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[u][i] = 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + u >= nrow) break;
+        fwht192_warp(x[u], lane);
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[u][i]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) atomicMax(&s_amax[(v0 + u) % a.H], __float_as_uint(mx));
+      }
+    }
+  } else if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int half = lane >> 4, li = lane & 15;
     const int nvec = (r1 - r0) * a.H;          // 128-element rows
@@ -205,7 +257,35 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
   const size_t off = (static_cast<size_t>(b) * a.S + r0) * HD;
   const T* base = static_cast<const T*>(a.x) + off;
   uint8_t* obase = a.out + off;
-  if (HAD) {
+  if (HAD && a.D == 192) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nrow = (r1 - r0) * a.H;
+    for (int v0 = warp * kUnroll; v0 < nrow; v0 += nw * kUnroll) {
+      float x[kUnroll][8];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + u < nrow && lane < 24) load8<T>(base + static_cast<size_t>(v0 + u) * 192 + 8 * lane, x[u]);
+        else
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[u][i] = 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 + u >= nrow) break;
+        fwht192_warp(x[u], lane);
+        if (lane >= 24) continue;
+        const int hh = (v0 + u) % a.H;
+        const float sc = s_sc[hh], rc = s_rc[hh];
+        uint32_t w[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          w[i] = cvt_e4m3x2(div_by_scale(x[u][4 * i], sc, rc), div_by_scale(x[u][4 * i + 1], sc, rc)) |
+                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(x[u][4 * i + 2], sc, rc),
+                                                   div_by_scale(x[u][4 * i + 3], sc, rc))) << 16);
+        *reinterpret_cast<uint2*>(obase + static_cast<size_t>(v0 + u) * 192 + 8 * lane) = make_uint2(w[0], w[1]);
+      }
+    }
+  } else if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int half = lane >> 4, li = lane & 15;
     const int nvec = (r1 - r0) * a.H;

@@ -82,7 +82,7 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int el, 
 template <bool FP8, int DQK, bool EXACTP = false>
 int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int S,
                 const float* qs, const float* ks, const float* vs, cudaStream_t stream, int dev,
-                int inst) {
+                int inst, float* lse = nullptr) {
   using Cf = AttnCfg<FP8, DQK>;
   AttnArgs a;
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -100,6 +100,7 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int
   }
   if (!ok) return ZYFA_ERR_CUDA;
   a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
   a.q_scale = qs;
   a.k_scale = ks;
   a.v_scale = vs;
@@ -219,6 +220,24 @@ extern "C" int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* 
   return launch_attn<false, 192>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 3);
 }
 
+extern "C" int zyfa_attn_fwd_lse(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                 int Hq, int Hkv, int S, int Dqk, int Dv, int dtype, const float* q_scale,
+                                 const float* k_scale, const float* v_scale, void* stream) {
+  const int bad = attn_validate(q, k, v, o, B, Hq, Hkv, S, Dqk, Dv, dtype, q_scale, k_scale, v_scale);
+  if (bad != ZYFA_OK) return bad;
+  if (!lse) return ZYFA_ERR_NULL_PTR;
+  if (!aligned(lse, 4)) return ZYFA_ERR_MISALIGNED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == ZYFA_FP8_E4M3) {
+    if (Dqk == 128) return launch_attn<true, 128>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 0, lse);
+    return launch_attn<true, 192>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 1, lse);
+  }
+  if (Dqk == 128) return launch_attn<false, 128>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 2, lse);
+  return launch_attn<false, 192>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 3, lse);
+}
+
 extern "C" int zyfa_attn_fwd_fp8_exact_p(const void* q, const void* k, const void* v, void* o, int B, int Hq,
                                          int Hkv, int S, int Dqk, int Dv, const float* q_scale,
                                          const float* k_scale, const float* v_scale, void* stream) {
@@ -237,7 +256,7 @@ extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* sc
   if (B < 1 || S < 1 || H < 1 || B > 65535 || H > 4096) return ZYFA_ERR_BAD_SHAPE;
   if (in_dtype != ZYFA_BF16 && in_dtype != ZYFA_FP32) return ZYFA_ERR_BAD_DTYPE;
   if (hadamard != 0 && hadamard != 1) return ZYFA_ERR_BAD_DTYPE;
-  if (D < 8 || D > 1024 || D % 8 != 0 || (hadamard && D != 128)) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (D < 8 || D > 1024 || D % 8 != 0 || (hadamard && D != 128 && D != 192)) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
   if (!aligned(x, 16) || !aligned(x_fp8, 16) || !aligned(scale, 4)) return ZYFA_ERR_MISALIGNED;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return ZYFA_ERR_CUDA;
@@ -288,7 +307,7 @@ extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, in
   if (hadamard_qk != 0 && hadamard_qk != 1) return ZYFA_ERR_BAD_DTYPE;
   for (int d : {Dqk, Dv})
     if (d < 8 || d > 1024 || d % 8 != 0) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
-  if (hadamard_qk && Dqk != 128) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (hadamard_qk && Dqk != 128 && Dqk != 192) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
   for (const void* t : {q, k, v, static_cast<const void*>(q_fp8), static_cast<const void*>(k_fp8),
                         static_cast<const void*>(v_fp8)})
     if (!aligned(t, 16)) return ZYFA_ERR_MISALIGNED;

@@ -38,6 +38,8 @@ def lib() -> ctypes.CDLL:
         p, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.zyfa_attn_fwd.restype = i
         L.zyfa_attn_fwd.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, p, p, p]
+        L.zyfa_attn_fwd_lse.restype = i
+        L.zyfa_attn_fwd_lse.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, p, p, p, p]
         L.zyfa_attn_fwd_fp8_exact_p.restype = i
         L.zyfa_attn_fwd_fp8_exact_p.argtypes = [p, p, p, p, i, i, i, i, i, i, p, p, p, p]
         L.zyfa_quantize.restype = i
@@ -89,11 +91,13 @@ def _dev(t, name):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
-def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=None, exact_p=False):
+def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=None, exact_p=False, lse=False):
     """Causal attention forward.  q [B,S,Hq,Dqk], k [B,S,Hkv,Dqk], v [B,S,Hkv,Dv];
     bf16 tensors (BF16 path) or uint8 / float8_e4m3fn codes with fp32 scales
     [B,H] (FP8 path).  exact_p (FP8 only): the exact-P ablation
-    (zyfa_attn_fwd_fp8_exact_p) instead of Lean P.  Returns o [B,S,Hq,Dv] bf16."""
+    (zyfa_attn_fwd_fp8_exact_p) instead of Lean P.  Returns o [B,S,Hq,Dv] bf16;
+    with lse=True (or an fp32 [B,Hq,S] tensor) returns (o, lse) through
+    zyfa_attn_fwd_lse."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
     if q.dtype == torch.bfloat16:
@@ -112,6 +116,15 @@ def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=N
             _dev(t, n)
             if t.dtype != torch.float32:
                 raise ValueError(f"{n} must be fp32")
+    if lse is not False and lse is not None:
+        if exact_p:
+            raise ValueError("lse is not produced by the exact-P ablation")
+        out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device) if lse is True else lse
+        _dev(out, "lse")
+        st = lib().zyfa_attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(out), B, Hq, Hkv, S, Dqk, Dv, dt,
+                                     _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream(stream))
+        _check(st, "zyfa_attn_fwd_lse")
+        return o, out
     if exact_p:
         if dt != FP8_E4M3:
             raise ValueError("exact_p applies to the FP8 path only")

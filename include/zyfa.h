@@ -98,6 +98,24 @@ int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
                   const float* v_scale, void* stream);
 
 /*
+ * zyfa_attn_fwd_lse -- zyfa_attn_fwd plus each row's softmax log-sum-exp, for
+ * callers that combine partial attention results (the online softmax of
+ * kongchang.com "Zyphra ZYFA", FlashAttention tiling, keeps exactly the
+ * running max and row sum this is formed from):
+ *   lse [B, Hq, S] fp32 (caller-owned, 4-byte aligned), natural log of
+ *   sum over keys j <= i of exp(s_ij / sqrt(Dqk)), s_ij the dot product of
+ *   the values the kernel received (dequantized for FP8).  It is formed from
+ *   the kernel's final reference max m and row sum l: ln 2 (m c + log2 l)
+ *   with c = log2(e) q_s k_s / sqrt(Dqk); for FP8, l sums the rounded Lean-P
+ *   weights, so the FP8 value carries their error (a few 1e-2 absolute).
+ * Other arguments, layouts and errors as zyfa_attn_fwd; NULL lse is
+ * ZYFA_ERR_NULL_PTR.
+ */
+int zyfa_attn_fwd_lse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                      int Hkv, int S, int Dqk, int Dv, int dtype, const float* q_scale,
+                      const float* k_scale, const float* v_scale, void* stream);
+
+/*
  * zyfa_attn_fwd_fp8_exact_p -- the exact-P ablation of the FP8 path: the
  * pages' Lean P (the-ai.news "Zyphra presenteert ZYFA", section "Drie
  * technieken om de bottleneck te omzeilen"; spke.com "Zyphra ZYFA", section
@@ -126,12 +144,15 @@ int zyfa_attn_fwd_fp8_exact_p(const void* q, const void* k, const void* v, void*
  *   scale  [B*H]         fp32 (output), indexed b*H + h
  *   hadamard = 1: each D = 128 row is first rotated by the orthonormal
  *     128-point Sylvester Walsh-Hadamard transform (butterflies of stride
- *     1, 2, ..., 64 in fp32, then one multiply by fp32(2^-3.5)).  Apply it to
- *     Q and K only (the rotation cancels in Q K^T); never to V.
+ *     1, 2, ..., 64 in fp32, then one multiply by fp32(2^-3.5)).  A D = 192
+ *     row (the MLA shape) is rotated block-diagonally: dims 0..127 by that
+ *     transform, dims 128..191 by the 64-point one (strides 1 .. 32, then
+ *     times 2^-3).  Apply it to Q and K only (the rotation cancels in Q K^T);
+ *     never to V.
  *   For each (b, h): amax = max |x'| over (s, d); scale = amax / 448 (fp32,
  *   IEEE division; 1.0 when amax == 0); code = e4m3 round-to-nearest-even,
  *   saturating at +-448, of fp32(x' / scale) (IEEE division).
- * D must be a multiple of 8 and at most 1024 (128 with hadamard).
+ * D must be a multiple of 8 and at most 1024 (128 or 192 with hadamard).
  * Alignment: x and x_fp8 16-byte aligned; scale 4-byte aligned.  The scale
  * buffer is used as the amax accumulator while the prepass runs (four
  * stream-ordered steps); it holds the final scales once the stream reaches
@@ -152,7 +173,7 @@ int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* scale, int B,
  *   *_fp8: e4m3 codes of the same shapes (outputs, caller-owned)
  *   *_scale: fp32 [B*Hq], [B*Hkv], [B*Hkv] (outputs; used as amax
  *   accumulators while the call's kernels run)
- * Dqk and Dv: multiples of 8, at most 1024 (Dqk = 128 with hadamard_qk = 1).
+ * Dqk and Dv: multiples of 8, at most 1024 (Dqk = 128 or 192 with hadamard_qk = 1).
  * Alignment as for zyfa_quantize.  Errors as for zyfa_quantize; nothing is
  * launched when an argument is rejected.
  */

@@ -15,7 +15,8 @@ def L():
 
 def test_every_declared_symbol_is_exported(L):
     names = zyfa.declared_symbols()
-    assert set(names) >= {"zyfa_attn_fwd", "zyfa_attn_fwd_fp8_exact_p", "zyfa_quantize", "zyfa_quantize_qkv",
+    assert set(names) >= {"zyfa_attn_fwd", "zyfa_attn_fwd_lse", "zyfa_attn_fwd_fp8_exact_p", "zyfa_quantize",
+                          "zyfa_quantize_qkv",
                           "zyfa_status_string",
                           "zyfa_device_status",
                           "zyfa_leanp_codes", "zyfa_selftest_wait_timeout", "zyfa_set_wait_timeout_ns"}
@@ -57,6 +58,16 @@ def test_attn_argument_errors(L):
     assert _attn(L, B=1 << 20, Hq=1 << 12, Hkv=1, S=1 << 16) == -2
 
 
+def test_lse_argument_errors(L):
+    def e(lse=FAKE, q=FAKE, B=1, S=128, dt=0):
+        return L.zyfa_attn_fwd_lse(q, FAKE, FAKE, FAKE, lse, B, 2, 2, S, 128, 128, dt, None, None, None, None)
+    assert e(lse=None) == -1
+    assert e(q=None) == -1
+    assert e(lse=FAKE + 2) == -5
+    assert e(S=0) == -2
+    assert e(dt=3) == -6
+
+
 def test_exact_p_argument_errors(L):
     def e(q=FAKE, o=FAKE, B=1, Hq=2, Hkv=2, S=128, Dqk=128, Dv=128, qs=None):
         return L.zyfa_attn_fwd_fp8_exact_p(q, FAKE, FAKE, o, B, Hq, Hkv, S, Dqk, Dv, qs, None, None, None)
@@ -78,7 +89,8 @@ def test_quantize_argument_errors(L):
     assert q(dt=1) == -6
     assert q(had=2) == -6
     assert q(D=12) == -3
-    assert q(D=192, had=1) == -3
+    assert q(D=64, had=1) == -3
+    assert q(D=256, had=1) == -3
     assert q(x=FAKE + 4) == -5
     assert q(sc=FAKE + 2) == -5
 
@@ -94,7 +106,7 @@ def test_quantize_qkv_argument_errors(L):
     assert q(dt=1) == -6
     assert q(had=3) == -6
     assert q(Dv=4) == -3
-    assert q(Dqk=192, had=1) == -3
+    assert q(Dqk=64, had=1) == -3
     assert q(k8=FAKE + 8) == -5
     assert q(vs=FAKE + 1) == -5
 

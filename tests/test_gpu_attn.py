@@ -11,8 +11,8 @@ import torch
 from bf16_causal_prefill_fp8_b200 import zyfa
 from oracle import oracle as orc
 
-from helpers import (RESCALE_LOG2, TOL_BF16, TOL_FP8, TOL_FP8_MODEL, fp8_references, inputs, run_bf16,
-                     run_fp8)
+from helpers import (RESCALE_LOG2, TOL_BF16, TOL_FP8, TOL_FP8_MODEL, bf16_round, fp8_references, inputs,
+                     run_bf16, run_fp8)
 
 pytestmark = pytest.mark.gpu
 
@@ -142,6 +142,58 @@ def test_fp8_exact_p_ablation(shape):
     assert e_ref <= TOL_FP8 and e_model <= TOL_FP8_MODEL
     assert e_ref <= e_lean * 1.05
     assert zyfa.device_status() == zyfa.OK
+
+
+@pytest.mark.parametrize("shape", [(1, 300, 2, 2, 128, 128), (2, 700, 4, 2, 128, 128), (1, 260, 4, 4, 192, 128)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_lse_output(shape):
+    """zyfa_attn_fwd_lse: the same O as zyfa_attn_fwd (bit for bit) plus each
+    row's log-sum-exp.  BF16 against the fp64 definition on the bf16 inputs;
+    FP8 against the CPU replay's own value (same weights) and, within the Lean-P
+    weight error, against the fp64 definition on the dequantized inputs."""
+    import torch
+    B, S, Hq, Hkv, Dqk, Dv = shape
+    q, k, v = inputs(49, B, S, Hq, Hkv, Dqk, Dv, kind="outlier_k" if Dqk == 128 else "mla")
+    qb, kb, vb = (bf16_round(x).cuda() for x in (q, k, v))
+    o_plain = zyfa.attn_fwd(qb, kb, vb)
+    o, lse = zyfa.attn_fwd(qb, kb, vb, lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_plain)
+    ref = orc.attention_lse(qb.cpu().double().numpy(), kb.cpu().double().numpy())
+    e_b = np.abs(lse.cpu().numpy() - ref).max()
+    print(f"lse bf16 {shape}: max abs err {e_b:.2e}")
+    assert e_b < 2e-3
+    o8, codes = run_fp8(q, k, v)
+    (qc, qs), (kc, ks), (vc, vs) = codes
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    o8b, lse8 = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs), lse=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(o8b.float().cpu().numpy().astype(np.float64), o8)
+    _, lse_model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=RESCALE_LOG2, return_lse=True)
+    deq = [orc.dequantize(x, sc) for x, sc in codes]
+    lse_ref = orc.attention_lse(deq[0], deq[1])
+    g = lse8.cpu().numpy()
+    d = np.abs(g - lse_model)
+    print(f"lse fp8 {shape}: vs replay max {d.max():.2e} median {np.median(d):.1e} mean {d.mean():.1e}  "
+          f"vs fp64 {np.abs(g - lse_ref).max():.2e}")
+    # A score whose fp32 tensor-core sum and fp64 replay sum straddle an integer
+    # of u gets a code one step apart: that weight differs by 2^(1/8), so a row's
+    # row sum by at most that factor, its lse by ln 2^(1/8) = 0.0866; such rows
+    # are rare (the bulk of rows equals the replay's value).  Against fp64 add
+    # Lean P's own per-weight band (2^-1/8, 1.0615]: at most 2 x 0.0866.
+    assert d.max() <= 0.087 and np.median(d) <= 1e-5 and d.mean() <= 5e-3
+    assert np.abs(g - lse_ref).max() <= 0.18
+
+
+def test_fp8_hadamard_prepass_path_mla():
+    """MLA shape with Q and K rotated block-diagonally (H128 + H64): the same
+    bars as without the rotation, which cancels in Q K^T."""
+    q, k, v = inputs(48, 1, 400, 4, 4, 192, 128, kind="mla")
+    o, codes = run_fp8(q, k, v, hadamard=True)
+    ref, model = fp8_references(codes)
+    assert orc.rel_fro(o, ref) <= TOL_FP8
+    assert orc.rel_fro(o, model) <= TOL_FP8_MODEL
+    assert orc.rel_fro(o, orc.attention(q, k, v)) < 0.1
 
 
 def test_fp8_hadamard_prepass_path():

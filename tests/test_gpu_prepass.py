@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("shape,hadamard", [((1, 200, 3, 128), False), ((1, 200, 3, 128), True),
                                             ((2, 77, 4, 192), False), ((3, 1, 5, 128), True),
-                                            ((1, 1000, 8, 128), True), ((2, 129, 2, 64), False)])
+                                            ((1, 1000, 8, 128), True), ((2, 129, 2, 64), False),
+                                            ((2, 77, 4, 192), True), ((1, 300, 3, 192), True)])
 @pytest.mark.parametrize("as_bf16", [False, True])
 def test_quantize_bit_exact(shape, hadamard, as_bf16):
     x = synth.gaussian(21, 1, shape) * np.float32(3.0)
@@ -42,6 +43,7 @@ def test_quantize_outlier_channels_and_subnormals():
 @pytest.mark.parametrize("B,S,Hq,Hkv,Dqk,Dv,hadamard", [(1, 300, 8, 2, 128, 128, False),
                                                         (2, 129, 4, 4, 128, 128, True),
                                                         (1, 77, 6, 2, 192, 128, False),
+                                                        (1, 77, 6, 2, 192, 128, True),
                                                         (1, 2048, 32, 8, 128, 128, True),
                                                         (3, 5, 2, 1, 128, 128, False)])
 @pytest.mark.parametrize("as_bf16", [False, True])
