@@ -1,0 +1,277 @@
+"""A randomized model of the attention kernel's mbarrier protocol (test
+infrastructure; it shares no code with the kernel).
+
+Each role of the kernel (producer, S issuer, P V issuer, the two softmax
+groups, the correction warpgroup) is a generator that takes the same barrier
+waits and arrivals, in the same order, as its counterpart in
+csrc/attn_fwd.cuh; the tensor-core and TMA engines are queues that complete
+after random delays.  An mbarrier is a phase counter: a parity wait passes
+when the completed-phase count has the other parity.  The model checks that
+
+- every parity wait that passes has truly completed the phase it waits for
+  (no aliasing: the waiter is never two phases behind);
+- no wait is stuck on a phase that is already complete;
+- nothing deadlocks;
+- no buffer is overwritten before its reader is done (S, P, rescale factors,
+  the reference-max exchange, the row-sum hand-over slots, the O accumulator
+  across units).
+
+`mutation` plants a known mistake, for the tests that show the model catches it.
+"""
+import random
+from dataclasses import dataclass
+
+
+@dataclass(frozen=True)
+class Config:
+    stk: int      # K ring stages
+    stv: int      # V ring stages
+    qbuf: int     # Q tile buffers
+    npb: int      # P buffers
+    fp8: bool     # FP8 hands the final max over per unit; BF16 per group
+
+    @property
+    def klead(self):
+        return self.stk - self.stv + 1
+
+
+# the kernel's three instantiations
+FP8 = Config(stk=4, stv=4, qbuf=2, npb=3, fp8=True)
+BF16_D128 = Config(stk=3, stv=2, qbuf=1, npb=2, fp8=False)
+BF16_D192 = Config(stk=2, stv=2, qbuf=1, npb=2, fp8=False)
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+class _Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.pend, self.c = name, count, 0, 0
+
+    def arrive(self, n=1):
+        self.pend += n
+        if self.pend > self.count:
+            raise ProtocolError(f"{self.name}: more arrivals than expected")
+        if self.pend == self.count:
+            self.pend = 0
+            self.c += 1
+
+
+def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5):
+    """Simulate one CTA that processes `units` (KV-tile counts per unit)."""
+    rng = random.Random(seed)
+    bars = {}
+
+    def bar(n, cnt):
+        bars[n] = _Bar(n, cnt)
+
+    for i in range(2):
+        for n, c in (("QF", 1), ("QE", 1), ("SF", 1), ("SC", 128), ("MX", 128)):
+            bar(f"{n}{i}", c)
+    for i in range(cfg.npb):
+        for n, c in (("PF", 128), ("PE", 1), ("OR", 128)):
+            bar(f"{n}{i}", c)
+    bar("OF", 128)
+    bar("OFIN", 1)
+    for i in range(cfg.stk):
+        bar(f"KF{i}", 1); bar(f"KE{i}", 1)
+    for i in range(cfg.stv):
+        bar(f"VF{i}", 1); bar(f"VE{i}", 1)
+    tiles = [(u, j, nkv) for u, nkv in enumerate(units) for j in range(nkv)]
+    fifos = {"qk": [], "pv": []}
+    tma = []
+    st = {"P": {}, "alpha": {}, "O_unit": None, "pv_done": set(), "qk_done": set(), "Sread": {}, "xch": {}, "lfin": {},
+          "hand": {}}
+    lfin_slots = 3 if mutation == "lfin_mod3" else 4
+
+    def wait(name, parity, need):
+        b = bars[name]
+        while True:
+            passed = (b.c & 1) != parity
+            truly = b.c > need
+            if passed:
+                if not truly:
+                    raise ProtocolError(f"aliasing on {name}: parity {parity} passed at phase count {b.c}, "
+                                        f"needs more than {need}")
+                return
+            if truly:
+                raise ProtocolError(f"stuck on {name}: phase {need} complete but parity {parity} fails")
+            yield "wait"
+
+    def producer():
+        ks = vs = 0
+
+        def load_k(g):
+            u, j, nkv = tiles[g]
+            if j == 0:
+                slot, n = u % cfg.qbuf, u // cfg.qbuf
+                if n > 0:
+                    yield from wait(f"QE{slot}", (n - 1) & 1, n - 1)
+                tma.append([rng.randint(5, 40), f"QF{slot}"])
+            s, n = g % cfg.stk, g // cfg.stk
+            if n > 0:
+                yield from wait(f"KE{s}", (n - 1) & 1, n - 1)
+            tma.append([rng.randint(5, 40), f"KF{s}"])
+
+        def load_v(g):
+            s, n = g % cfg.stv, g // cfg.stv
+            if n > 0:
+                yield from wait(f"VE{s}", (n - 1) & 1, n - 1)
+            tma.append([rng.randint(5, 40), f"VF{s}"])
+
+        for _ in range(cfg.klead):
+            if ks < len(tiles):
+                yield from load_k(ks); ks += 1
+        while vs < len(tiles):
+            if ks < len(tiles):
+                yield from load_k(ks); ks += 1
+            yield from load_v(vs); vs += 1
+            yield "step"
+
+    def qk_issuer():
+        for g, (u, j, nkv) in enumerate(tiles):
+            slot = u % cfg.qbuf
+            if j == 0:
+                yield from wait(f"QF{slot}", (u // cfg.qbuf) & 1, u // cfg.qbuf)
+            s, buf = g % cfg.stk, g & 1
+            yield from wait(f"KF{s}", (g // cfg.stk) & 1, g // cfg.stk)
+            if g >= 2 and mutation != "no_sc_wait":
+                yield from wait(f"SC{buf}", ((g >> 1) - 1) & 1, (g >> 1) - 1)
+            if g >= 2 and st["Sread"].get(buf, -1) < g - 2:
+                raise ProtocolError(f"S buffer {buf} overwritten by tile {g} before tile {g - 2} read it")
+            fifos["qk"].append([rng.randint(5, 30), "qk", g])
+            fifos["qk"].append([0, "commit", [f"SF{buf}", f"KE{s}"] + ([f"QE{slot}"] if j == nkv - 1 else [])])
+            yield "step"
+
+    def pv_issuer():
+        for g, (u, j, nkv) in enumerate(tiles):
+            s, buf = g % cfg.stv, g % cfg.npb
+            if j == 0 and u > 0:
+                yield from wait("OF", (u - 1) & 1, u - 1)
+            yield from wait(f"OR{buf}", (g // cfg.npb) & 1, g // cfg.npb)
+            yield from wait(f"VF{s}", (g // cfg.stv) & 1, g // cfg.stv)
+            if st["P"].get(buf) != g:
+                raise ProtocolError(f"P buffer {buf} holds tile {st['P'].get(buf)} at P V of tile {g}")
+            if j == 0:
+                if st["O_unit"] not in (None, "free"):
+                    raise ProtocolError(f"O still in use by unit {st['O_unit']} at unit {u}")
+                st["O_unit"] = u
+            fifos["pv"].append([rng.randint(5, 30), "pv", g])
+            fifos["pv"].append([0, "commit", [f"VE{s}", f"PE{buf}"] + (["OFIN"] if j == nkv - 1 else [])])
+            yield "step"
+
+    def softmax_group(grp):
+        for g, (u, j, nkv) in enumerate(tiles):
+            if (g & 1) != grp:
+                continue
+            buf = grp
+            yield from wait(f"SF{buf}", (g >> 1) & 1, g >> 1)
+            if g not in st["qk_done"]:
+                raise ProtocolError(f"S of tile {g} read before its MMA finished")
+            yield "pass1"
+            if g >= 1:
+                pb = (g - 1) & 1
+                yield from wait(f"MX{pb}", ((g - 1) >> 1) & 1, (g - 1) >> 1)
+                if st["xch"].get(pb) != g - 1:
+                    raise ProtocolError(f"reference max of tile {g - 1} overwritten before tile {g} read it")
+            st["xch"][grp] = g
+            bars[f"MX{grp}"].arrive(128)
+            pbuf = g % cfg.npb
+            back = 2 if mutation == "pe_wait_two_back" else cfg.npb
+            if g >= back:
+                yield from wait(f"PE{pbuf}", ((g - back) // cfg.npb) & 1, (g - back) // cfg.npb)
+            if g >= cfg.npb and (g - cfg.npb) not in st["pv_done"]:
+                raise ProtocolError(f"P buffer {pbuf} rewritten by tile {g} before P V of tile {g - cfg.npb}")
+            for _ in range(rng.randint(0, 3)):
+                yield "codes"
+            st["Sread"][buf] = g
+            bars[f"SC{buf}"].arrive(128)
+            for _ in range(rng.randint(0, 3)):
+                yield "codes"
+            if cfg.fp8 and j == nkv - 1:
+                st["lfin"][u % lfin_slots] = u       # the unit's final reference max
+            if not cfg.fp8 and j >= nkv - 2:
+                st["hand"][grp] = g                  # this group's partial row sum and its max
+            st["P"][pbuf] = g
+            slot = (g & 1) if mutation == "alpha_by_group" else pbuf
+            st["alpha"][slot] = g
+            bars[f"PF{pbuf}"].arrive(128)
+
+    def correction():
+        for g, (u, j, nkv) in enumerate(tiles):
+            pbuf = g % cfg.npb
+            yield from wait(f"PF{pbuf}", (g // cfg.npb) & 1, g // cfg.npb)
+            slot = (g & 1) if mutation == "alpha_by_group" else pbuf
+            if st["alpha"].get(slot) != g:
+                raise ProtocolError(f"rescale factor of tile {g} overwritten before the correction read it")
+            if not cfg.fp8 and j >= nkv - 2 and st["hand"].get(g & 1) != g:
+                raise ProtocolError(f"row-sum hand-over of tile {g} overwritten before the correction read it")
+            if j > 0 and rng.random() < p_rescale:
+                pg = g - 1
+                yield from wait(f"PE{pg % cfg.npb}", (pg // cfg.npb) & 1, pg // cfg.npb)
+                if pg not in st["pv_done"]:
+                    raise ProtocolError(f"O rescaled for tile {g} before P V of tile {pg} finished")
+                yield "rescale"
+            bars[f"OR{pbuf}"].arrive(128)
+            if j == nkv - 1:
+                yield from wait("OFIN", u & 1, u)
+                if not all(t in st["pv_done"] for t in range(g - j, g + 1)):
+                    raise ProtocolError(f"epilogue of unit {u} before its last P V finished")
+                for _ in range(rng.randint(0, 3)):   # the row-sum load from TMEM comes first
+                    yield "epilogue"
+                if cfg.fp8 and st["lfin"].get(u % lfin_slots) != u:
+                    raise ProtocolError(f"final max of unit {u} overwritten before its epilogue read it")
+                for _ in range(rng.randint(1, 8)):
+                    yield "epilogue"
+                st["O_unit"] = "free"
+                bars["OF"].arrive(128)
+
+    roles = {"producer": producer(), "qk": qk_issuer(), "pv": pv_issuer(), "softmax0": softmax_group(0),
+             "softmax1": softmax_group(1), "correction": correction()}
+    done, idle = set(), 0
+    while len(done) < len(roles):
+        progressed = False
+        for fk in rng.sample(["qk", "pv"], 2):     # the tensor core completes each issuer's work in order
+            f = fifos[fk]
+            if not f:
+                continue
+            e = f[0]
+            if e[1] == "commit":
+                for n in e[2]:
+                    bars[n].arrive()
+                f.pop(0)
+            else:
+                e[0] -= 1
+                if e[0] <= 0:
+                    (st["qk_done"] if e[1] == "qk" else st["pv_done"]).add(e[2])
+                    f.pop(0)
+            progressed = True
+        for t in list(tma):
+            t[0] -= 1
+            if t[0] <= 0:
+                bars[t[1]].arrive()
+                tma.remove(t)
+            progressed = True
+        names = [n for n in roles if n not in done]
+        rng.shuffle(names)
+        for n in names:
+            try:
+                if next(roles[n]) != "wait":
+                    progressed = True
+            except StopIteration:
+                done.add(n)
+                progressed = True
+        idle = 0 if progressed else idle + 1
+        if idle >= 1000:
+            raise ProtocolError("deadlock: " + ", ".join(f"{k} {b.c}/{b.pend}" for k, b in bars.items() if b.pend))
+
+
+def random_units(rng):
+    """KV-tile counts of the units one CTA takes: random lengths, or (as the
+    heaviest-first queue hands them out) descending, ending in runs of
+    one-tile units."""
+    units = [rng.randint(1, 7) if rng.random() < 0.6 else 1 for _ in range(rng.randint(1, 12))]
+    if rng.random() < 0.5:
+        units.sort(reverse=True)
+    return units

@@ -1,0 +1,28 @@
+"""The attention kernel's barrier protocol, checked on a randomized model
+(tests/protocol_model.py) for the kernel's three ring / buffer
+configurations, and the model's power to catch planted mistakes."""
+import random
+
+import pytest
+
+from protocol_model import BF16_D128, BF16_D192, FP8, ProtocolError, random_units, run
+
+CONFIGS = {"fp8": FP8, "bf16_d128": BF16_D128, "bf16_d192": BF16_D192}
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_protocol_holds_on_random_schedules(name):
+    cfg = CONFIGS[name]
+    for seed in range(80):
+        rng = random.Random(seed)
+        run(random_units(rng), cfg, seed, p_rescale=(0.0, 0.3, 0.9)[seed % 3])
+
+
+@pytest.mark.parametrize("mutation,cfg", [("alpha_by_group", FP8), ("pe_wait_two_back", FP8),
+                                          ("no_sc_wait", FP8), ("no_sc_wait", BF16_D128),
+                                          ("lfin_mod3", FP8)])
+def test_model_catches_planted_mistakes(mutation, cfg):
+    with pytest.raises(ProtocolError):
+        for seed in range(200):
+            rng = random.Random(seed)
+            run(random_units(rng), cfg, seed, mutation=mutation)
