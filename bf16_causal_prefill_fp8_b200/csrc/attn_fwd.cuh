@@ -38,6 +38,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "leanp.cuh"
 #include "ptx.cuh"
@@ -125,25 +126,35 @@ struct AttnCfg {
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
+#define ZYFA_HD __host__ __device__
+
+ZYFA_HD __forceinline__ int imin(int x, int y) { return x < y ? x : y; }
+
 // Static causal-aware schedule.  Units are grouped by (batch, kv head) slots so
 // that one group's K/V stays resident in L2; inside a group the heaviest query
 // tiles (most KV tiles) come first, and consecutive units share a kv head.
 // Units are dealt round-robin to the persistent CTAs, reversing direction on
-// every round so per-CTA work evens out.
+// every round so per-CTA work evens out.  Host-callable, so the schedule a
+// launch will run can be enumerated on the CPU.
 struct UnitIter {
   int G, c, Tq, gq, Hkv, slots, Gk, ngroups;
   int g, k, slots_g, U_g;
-  __device__ void init(int grid, int cta, int Tq_, int Hq, int Hkv_, int B, int Gk_) {
+  ZYFA_HD void init(int grid, int cta, int Tq_, int Hq, int Hkv_, int B, int Gk_) {
     G = grid; c = cta; Tq = Tq_; Hkv = Hkv_; gq = Hq / Hkv_;
     slots = B * Hkv_; Gk = Gk_; ngroups = (slots + Gk - 1) / Gk;
     g = 0; k = 0;
-    slots_g = min(Gk, slots); U_g = slots_g * gq * Tq;
+    slots_g = imin(Gk, slots); U_g = slots_g * gq * Tq;
   }
-  __device__ bool next(int& b, int& hkv, int& hq, int& qt) {
+  // the variable-length signature, so both iterators take the same calls
+  ZYFA_HD bool next(int& b, int& hkv, int& hq, int& qt, int& r0, int& len) {
+    r0 = 0; len = 0;
+    return next(b, hkv, hq, qt);
+  }
+  ZYFA_HD bool next(int& b, int& hkv, int& hq, int& qt) {
     while (g < ngroups) {
       if (k * G >= U_g) {
         ++g; k = 0;
-        if (g < ngroups) { slots_g = min(Gk, slots - g * Gk); U_g = slots_g * gq * Tq; }
+        if (g < ngroups) { slots_g = imin(Gk, slots - g * Gk); U_g = slots_g * gq * Tq; }
         continue;
       }
       const int p = k * G + ((k & 1) ? (G - 1 - c) : c);
@@ -162,6 +173,86 @@ struct UnitIter {
   }
 };
 
+// Variable-length batch: sequences packed back to back along the row
+// dimension, sequence s holding rows cu[s] .. cu[s+1]-1 of every tensor.  The
+// host orders the sequences longest first; a (sequence, kv head) slot is
+// s_i * Hkv + hkv for the i-th sequence of that order.  The table travels as
+// a kernel parameter (with AttnArgs inside the 4 KiB parameter space).
+constexpr int kMaxVarlenSeqs = 384;
+struct VarlenSeqs {
+  int n;                          // sequences
+  int kv_row_bytes;               // bytes of one K row plus one V row of one kv head
+  long long group_bytes;          // K/V bytes a scheduling group may hold (L2 budget)
+  int order[kMaxVarlenSeqs];      // sequence ids, longest first (equal lengths by id)
+  int cu[kMaxVarlenSeqs + 1];     // first packed row of each sequence; cu[n] = total rows
+};
+
+// The same schedule over a variable-length batch.  Slots, in the order above,
+// are grouped greedily: a group takes slots while their K/V bytes fit the L2
+// budget (at least one slot).  Inside a group units are issued by query tile
+// index descending (level L = the tile index), a level holding every (slot,
+// query head) whose sequence has more than L tiles; slots are longest first,
+// so those are a prefix of the group and the prefix only grows as L falls.
+// With all lengths equal this is UnitIter's schedule, unit for unit.
+struct VarlenIter {
+  const VarlenSeqs* t;
+  int G, c, gq, Hkv, nslots;
+  int s0, s1;          // the group's slots [s0, s1)
+  int k, U;            // dealing round; units of the group
+  int L, base, act;    // current level, its first unit index, slots active at it
+  ZYFA_HD int seq_len(int slot) const {
+    const int s = t->order[slot / Hkv];
+    return t->cu[s + 1] - t->cu[s];
+  }
+  ZYFA_HD int tiles(int slot) const { return (seq_len(slot) + 127) / 128; }
+  ZYFA_HD void open(int from) {
+    s0 = from; s1 = from; U = 0; k = 0;
+    long long bytes = 0;
+    while (s1 < nslots) {
+      const long long sb = static_cast<long long>(seq_len(s1)) * t->kv_row_bytes;
+      if (s1 > s0 && bytes + sb > t->group_bytes) break;
+      bytes += sb;
+      U += tiles(s1);
+      ++s1;
+    }
+    U *= gq;
+    L = s0 < nslots ? tiles(s0) - 1 : -1;
+    base = 0; act = 0;
+    while (s0 + act < s1 && tiles(s0 + act) > L) ++act;
+  }
+  ZYFA_HD void init(int grid, int cta, const VarlenSeqs* seqs, int Hq, int Hkv_) {
+    t = seqs; G = grid; c = cta; Hkv = Hkv_; gq = Hq / Hkv_; nslots = seqs->n * Hkv_;
+    open(0);
+  }
+  ZYFA_HD bool next(int& b, int& hkv, int& hq, int& qt) {
+    int r0, len;
+    return next(b, hkv, hq, qt, r0, len);
+  }
+  // b: sequence id; r0, len: its first packed row and its length
+  ZYFA_HD bool next(int& b, int& hkv, int& hq, int& qt, int& r0, int& len) {
+    while (s0 < nslots) {
+      if (k * G >= U) { open(s1); continue; }
+      const int p = k * G + ((k & 1) ? (G - 1 - c) : c);
+      ++k;
+      if (p >= U) continue;
+      while (p >= base + act * gq) {   // p < U, so this stops at a level >= 0
+        base += act * gq;
+        --L;
+        while (s0 + act < s1 && tiles(s0 + act) > L) ++act;
+      }
+      const int rem = p - base, slot = s0 + rem / gq, i = slot / Hkv;
+      b = t->order[i];
+      hkv = slot - i * Hkv;
+      hq = hkv * gq + (rem - (rem / gq) * gq);
+      qt = L;
+      r0 = t->cu[b];
+      len = t->cu[b + 1] - r0;
+      return true;
+    }
+    return false;
+  }
+};
+
 // One lane of a converged warp (the same lane every time for the same mask).
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred;
@@ -173,18 +264,27 @@ __device__ __forceinline__ bool elect_one() {
 
 // The CTA's sequence of (unit, KV tile) pairs in issue order; g counts tiles
 // and u counts units across the whole sequence (ring stages and barrier phases
-// derive from them).
+// derive from them).  VARLEN: r0 and len are the unit's sequence's first
+// packed row and length.
+template <bool VARLEN>
 struct TileStream {
-  UnitIter units;
+  typename std::conditional<VARLEN, VarlenIter, UnitIter>::type units;
   int b, hkv, hq, qt, j, nkv;
+  int r0, len;
   uint32_t g, u;
-  __device__ void init(int grid, int cta, int Tq, int Hq, int Hkv, int B, int Gk) {
-    units.init(grid, cta, Tq, Hq, Hkv, B, Gk);
+  __device__ void init(int grid, int cta, const AttnArgs& a, const VarlenSeqs* vs) {
+    if constexpr (VARLEN) units.init(grid, cta, vs, a.Hq, a.Hkv);
+    else units.init(grid, cta, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
     j = 0; nkv = 0; g = 0xffffffffu; u = 0xffffffffu;
+    r0 = 0; len = 0;
   }
   __device__ bool next() {
     if (j + 1 < nkv) { ++j; ++g; return true; }
-    if (!units.next(b, hkv, hq, qt)) return false;
+    if constexpr (VARLEN) {
+      if (!units.next(b, hkv, hq, qt, r0, len)) return false;
+    } else {
+      if (!units.next(b, hkv, hq, qt)) return false;
+    }
     nkv = qt + 1; j = 0; ++g; ++u;
     return true;
   }
@@ -251,9 +351,18 @@ __device__ __forceinline__ float max64(const uint32_t* s) {
 // EXACTP (FP8 only): the ablation that writes P the conventional way, an
 // exponential (MUFU ex2) followed by a conversion to e4m3, with the same block
 // shift, scale factors and row sum as Lean P.
-template <bool FP8, int DQK, bool EXACTP = false>
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnArgs a) {
+//
+// VARLEN: the batch is packed (rows of sequence s at cu[s] .. cu[s+1]-1, one
+// tensor-map batch), and vs holds the sequences; otherwise vs is null.
+template <bool VARLEN> struct SeqTable {};
+template <> struct SeqTable<true> : VarlenSeqs {};
+template <bool FP8, int DQK, bool EXACTP = false, bool VARLEN = false>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ SeqTable<VARLEN> seqs) {
+  const VarlenSeqs* vs = nullptr;
+  if constexpr (VARLEN) vs = &seqs;
   using Cf = AttnCfg<FP8, DQK>;
+  using TS = TileStream<VARLEN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -317,8 +426,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
   const WaitCtl ctl{abort_flag, a.timeout_ns};
-  UnitIter units;
-  units.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+  typename std::conditional<VARLEN, VarlenIter, UnitIter>::type units;
+  if constexpr (VARLEN) units.init(gridDim.x, blockIdx.x, vs, a.Hq, a.Hkv);
+  else units.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
 
   if (warp >= 12) {
    // The producer and MMA warps run converged; one elected lane polls the
@@ -337,9 +447,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     // K runs KLEAD tiles ahead of V, in the order the MMAs consume them.
     const uint64_t pol_q = l2_policy_evict_first();
     const uint64_t pol_kv = l2_policy_evict_last();
-    TileStream ks, vs;
-    ks.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
-    vs.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    TS ks, vst;
+    ks.init(gridDim.x, blockIdx.x, a, vs);
+    vst.init(gridDim.x, blockIdx.x, a, vs);
     bool ok = true;
     auto load_rows = [&](uint32_t dst, const CUtensorMap* m, const CUtensorMap* mt, uint32_t br,
                          int h, int row, int bb, uint64_t pol) {
@@ -348,14 +458,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         tma_load_4d(dst + c * Cf::CHUNK, m, br, c * (128 / Cf::EL), h, row, bb, pol);
       if (Cf::TAIL) tma_load_4d(dst + Cf::NCH * Cf::CHUNK, mt, br, 128, h, row, bb, pol);
     };
-    auto load_k = [&](const TileStream& t) -> bool {
+    auto load_k = [&](const TS& t) -> bool {
+      // tensor-map row and batch coordinates of the unit's sequence
+      const int row0 = VARLEN ? t.r0 : 0, tb = VARLEN ? 0 : t.b;
       if (t.j == 0) {                      // first tile of a unit: its Q tile first
         const uint32_t slot = t.u % Cf::QBUF, n = t.u / Cf::QBUF;
         if (n > 0 && !wait1(bar(Cf::QE0 + slot), (n - 1) & 1)) return false;
         if (leader) {
           mbar_arrive_expect_tx(bar(Cf::QF0 + slot), Cf::QB);
           load_rows(sb + Cf::OFF_Q + slot * Cf::QB, &a.map_q, &a.map_q_tail, bar(Cf::QF0 + slot),
-                    t.hq, t.qt * 128, t.b, pol_q);
+                    t.hq, row0 + t.qt * 128, tb, pol_q);
         }
       }
       const uint32_t st = t.g % Cf::STK, n = t.g / Cf::STK;
@@ -363,12 +475,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       if (leader) {
         mbar_arrive_expect_tx(bar(Cf::KF + st), Cf::KB);
         load_rows(sb + Cf::OFF_K + st * Cf::KB, &a.map_k, &a.map_k_tail, bar(Cf::KF + st), t.hkv,
-                  t.j * 128, t.b, pol_kv);
+                  row0 + t.j * 128, tb, pol_kv);
       }
       __syncwarp();
       return true;
     };
-    auto load_v = [&](const TileStream& t) -> bool {
+    auto load_v = [&](const TS& t) -> bool {
+      const int row0 = VARLEN ? t.r0 : 0, tb = VARLEN ? 0 : t.b;
       const uint32_t st = t.g % Cf::STV, n = t.g / Cf::STV;
       if (n > 0 && !wait1(bar(Cf::VE + st), (n - 1) & 1)) return false;
       if (leader) {
@@ -376,15 +489,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
 #pragma unroll
         for (int c = 0; c < Cf::VB / Cf::CHUNK; ++c)
           tma_load_4d(sb + Cf::OFF_V + st * Cf::VB + c * Cf::CHUNK, &a.map_v, bar(Cf::VF + st),
-                      c * (128 / Cf::EL), t.hkv, t.j * 128, t.b, pol_kv);
+                      c * (128 / Cf::EL), t.hkv, row0 + t.j * 128, tb, pol_kv);
       }
       __syncwarp();
       return true;
     };
     for (int i = 0; i < Cf::KLEAD && ok && ks.next(); ++i) ok = load_k(ks);
-    while (ok && vs.next()) {
+    while (ok && vst.next()) {
       if (ks.next()) ok = load_k(ks);
-      if (ok) ok = load_v(vs);
+      if (ok) ok = load_v(vst);
     }
     if (!ok) {
       // let copies already in flight land before the CTA exits
@@ -396,8 +509,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     // warp 9: S for tile g is issued as soon as its K tile is loaded and the
     // softmax has read S of tile g-2 (two S buffers).  warp 10: P V of tile g
     // once the softmax has written P and the correction has rescaled O.
-    TileStream ts;
-    ts.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    TS ts;
+    ts.init(gridDim.x, blockIdx.x, a, vs);
     bool ok = true;
     // descriptor bases; per-step descriptors add (byte offset >> 4) to the low word
     const uint64_t dq = smem_desc(sb + Cf::OFF_Q, 16, 1024, kSw128);
@@ -407,7 +520,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const uint64_t dv = smem_desc(sb + Cf::OFF_V, 16384, 1024, kSw128);
     const uint64_t dones = smem_desc(sb + Cf::OFF_ONES, 16, 1024, kSw128);
     const uint64_t dsf = smem_desc(sb + Cf::OFF_SF, 16, 128, kSwNone);
-    auto issue_qk = [&](const TileStream& t) -> bool {
+    auto issue_qk = [&](const TS& t) -> bool {
       const uint32_t slot = t.u % Cf::QBUF;
       if (t.j == 0 && !wait1(bar(Cf::QF0 + slot), (t.u / Cf::QBUF) & 1)) return false;
       const uint32_t st = t.g % Cf::STK, buf = t.g & 1;
@@ -438,7 +551,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       __syncwarp();
       return true;
     };
-    auto issue_pv = [&](const TileStream& t) -> bool {
+    auto issue_pv = [&](const TS& t) -> bool {
       const uint32_t st = t.g % Cf::STV, buf = t.g % Cf::NPB, ph = (t.g / Cf::NPB) & 1;
       const bool first = t.j == 0;
       // O is free once the previous unit's epilogue has read it
@@ -508,8 +621,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     // scale-factor word of row r: bytes at (r % 32) * 16 + (r / 32) * 4
     const uint32_t sf_row = (row & 31) * 4 + (row >> 5);
     const uint32_t ts = lb + (grp ? Cf::TS1 : Cf::TS0);
-    TileStream t;
-    t.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    TS t;
+    t.init(gridDim.x, blockIdx.x, a, vs);
     float A = a.C;
     float l = 0.0f, m_own = __int_as_float(0xff800000);   // BF16: this group's row sum and its max
     while (ok && t.next()) {
@@ -664,8 +777,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const uint32_t lb = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     uint32_t kv_it = 0, u_it = 0;
     int b, hkv, hq, qt;
+    int r0 = 0, len = 0;   // VARLEN: the unit's sequence's first packed row and length
     bool ok = true;
-    while (ok && units.next(b, hkv, hq, qt)) {
+    while (ok && (VARLEN ? units.next(b, hkv, hq, qt, r0, len) : units.next(b, hkv, hq, qt))) {
       const int nkv = qt + 1;
       // BF16: each softmax group hands over its partial row sum and the max it
       // is relative to at its last tile of the unit (one of the last two)
@@ -729,9 +843,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         inv = 1.0f / lt;
         if (a.lse) lse_log2 = __fmaf_rn(m_last, a.C, log2f(lt));
       }
-      if (a.lse && grow < a.S)
-        a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.S + grow] = lse_log2 * 0.69314718055994530942f;
-      __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.S + grow) * a.Hq + hq) * 128;
+      // output row: (b, grow) of [B, S, Hq, 128], or packed row r0 + grow of
+      // [T, Hq, 128]; lse [B, Hq, S] or [Hq, T]
+      __nv_bfloat16* orow;
+      if constexpr (VARLEN) {
+        if (a.lse && grow < len)
+          a.lse[static_cast<size_t>(hq) * a.S + r0 + grow] = lse_log2 * 0.69314718055994530942f;
+        orow = a.o + ((static_cast<size_t>(r0) + grow) * a.Hq + hq) * 128;
+      } else {
+        if (a.lse && grow < a.S)
+          a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.S + grow] = lse_log2 * 0.69314718055994530942f;
+        orow = a.o + ((static_cast<size_t>(b) * a.S + grow) * a.Hq + hq) * 128;
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
@@ -741,7 +864,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (grow < a.S) {
+        if (grow < (VARLEN ? len : a.S)) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
@@ -758,5 +881,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tbase, 512);
 }
+
+static_assert(sizeof(AttnArgs) + sizeof(VarlenSeqs) <= 4096, "kernel parameter space");
 
 }  // namespace zyfa

@@ -397,6 +397,52 @@ __global__ void __launch_bounds__(kQuantThreads) quant3_codes_kernel(const __gri
   else quant_codes_cta<T, false>(a.t[i], chunk, blockIdx.y, s_sc);
 }
 
+// Variable-length batch: tensors packed [T, H, D], sequence s at rows
+// cu[s] .. cu[s+1]-1 with its own scale per head ([nseq, H] per tensor).
+// Grid = (sum of chunk columns, nseq): CTA (x, s) runs the fixed-length step
+// on sequence s alone (base and scale pointers moved to it, S = its length);
+// chunks past the sequence's end have no rows and return at once.
+constexpr int kMaxQuantSeqs = 384;
+struct Quant3VarArgs {
+  Quant3Args q;                  // t[i].S unused; rows_per_cta per tensor
+  int cu[kMaxQuantSeqs + 1];
+};
+
+template <typename T>
+__device__ __forceinline__ bool quant3v_select(const Quant3VarArgs& a, QuantArgs& t, int& i, int& chunk) {
+  i = quant3_pick(a.q, blockIdx.x);
+  chunk = blockIdx.x - a.q.first[i];
+  const int s = blockIdx.y, r0 = a.cu[s], len = a.cu[s + 1] - r0;
+  t = a.q.t[i];
+  if (static_cast<long long>(chunk) * t.rows_per_cta >= len) return false;
+  const size_t off = static_cast<size_t>(r0) * t.H * t.D;
+  t.x = static_cast<const T*>(t.x) + off;
+  t.out += off;
+  t.scale += static_cast<size_t>(s) * t.H;
+  t.S = len;
+  return true;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) quant3v_amax_kernel(const __grid_constant__ Quant3VarArgs a) {
+  extern __shared__ unsigned int s_amax[];
+  QuantArgs t;
+  int i, chunk;
+  if (!quant3v_select<T>(a, t, i, chunk)) return;
+  if (a.q.had[i]) quant_amax_cta<T, true>(t, chunk, 0, s_amax);
+  else quant_amax_cta<T, false>(t, chunk, 0, s_amax);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads) quant3v_codes_kernel(const __grid_constant__ Quant3VarArgs a) {
+  extern __shared__ float s_sc[];
+  QuantArgs t;
+  int i, chunk;
+  if (!quant3v_select<T>(a, t, i, chunk)) return;
+  if (a.q.had[i]) quant_codes_cta<T, true>(t, chunk, 0, s_sc);
+  else quant_codes_cta<T, false>(t, chunk, 0, s_sc);
+}
+
 // Steps 1 and 4 for the three scale arrays (n[i] = B * H_i entries each).
 __global__ void quant3_zero_kernel(float* s0, float* s1, float* s2, int n0, int n1, int n2) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

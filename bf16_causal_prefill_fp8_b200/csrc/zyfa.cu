@@ -4,11 +4,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
+#include <numeric>
+#include <vector>
 
 #include "../../include/zyfa.h"
 #include "attn_fwd.cuh"
@@ -59,7 +62,7 @@ EncodeTiledFn encode_fn() {
 
 struct DeviceInfo {
   int sms = 0;
-  bool attr_set[6] = {false, false, false, false, false, false};
+  bool attr_set[10] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -79,12 +82,46 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int el, 
             swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool FP8, int DQK, bool EXACTP = false>
-int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int S,
-                const float* qs, const float* ks, const float* vs, cudaStream_t stream, int dev,
-                int inst, float* lse = nullptr) {
+// K/V bytes one scheduling group may hold: its tiles stay resident in L2
+// (126 MB on B200) while the group's query tiles stream through.
+constexpr long long kGroupBytes = 48ll * 1024 * 1024;
+
+// (batch, kv head) slots per scheduling group of a fixed-length launch
+int group_slots_for(int B, int Hkv, int S, int dqk, int el) {
+  const double kv_slot_bytes = static_cast<double>(S) * (dqk + 128) * el;
+  long long gk = static_cast<long long>(static_cast<double>(kGroupBytes) / kv_slot_bytes);
+  const long long slots = static_cast<long long>(B) * Hkv;
+  if (gk < 1) gk = 1;
+  if (gk > slots) gk = slots;
+  return static_cast<int>(gk);
+}
+
+// The sequence table of a variable-length launch: ids ordered longest first
+// (a stable sort, so equal lengths keep their order), offsets as given.
+void fill_varlen_table(VarlenSeqs& t, const int* cu, int nseq, int dqk, int el) {
+  t.n = nseq;
+  t.kv_row_bytes = (dqk + 128) * el;
+  t.group_bytes = kGroupBytes;
+  for (int i = 0; i <= nseq; ++i) t.cu[i] = cu[i];
+  std::vector<int> ids(nseq);
+  std::iota(ids.begin(), ids.end(), 0);
+  std::stable_sort(ids.begin(), ids.end(),
+                   [&](int x, int y) { return cu[x + 1] - cu[x] > cu[y + 1] - cu[y]; });
+  for (int i = 0; i < nseq; ++i) t.order[i] = ids[i];
+}
+
+long long varlen_units(const int* cu, int nseq, int Hq) {
+  long long u = 0;
+  for (int i = 0; i < nseq; ++i) u += static_cast<long long>(Hq) * ((cu[i + 1] - cu[i] + 127) / 128);
+  return u;
+}
+
+// Tensor maps and scalar arguments shared by both launch forms.  B, S are the
+// tensor-map batch and row extents (a packed batch: 1, total rows).
+template <bool FP8, int DQK>
+bool fill_attn_args(AttnArgs& a, const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv,
+                    int S, const float* qs, const float* ks, const float* vs, float* lse) {
   using Cf = AttnCfg<FP8, DQK>;
-  AttnArgs a;
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int el = FP8 ? 1 : 2;
   const int box = 128 / el;   // 128 bytes of one row
@@ -98,39 +135,71 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int
     a.map_q_tail = a.map_q;
     a.map_k_tail = a.map_k;
   }
-  if (!ok) return ZYFA_ERR_CUDA;
+  if (!ok) return false;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.q_scale = qs;
   a.k_scale = ks;
   a.v_scale = vs;
-  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.S = S;
-  a.Tq = (S + 127) / 128;
-  const double kv_slot_bytes = static_cast<double>(S) * (DQK + 128) * el;
-  long long gk = static_cast<long long>((48.0 * 1024 * 1024) / kv_slot_bytes);
-  const long long slots = static_cast<long long>(B) * Hkv;
-  if (gk < 1) gk = 1;
-  if (gk > slots) gk = slots;
-  a.group_slots = static_cast<int>(gk);
+  a.Hq = Hq; a.Hkv = Hkv;
   a.C = FP8 ? static_cast<float>(8.0 * 1.4426950408889634074 / std::sqrt(static_cast<double>(DQK)))
             : static_cast<float>(1.4426950408889634074 / std::sqrt(static_cast<double>(DQK)));
   a.timeout_ns = wait_timeout_ns();
+  return true;
+}
 
-  {
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    DeviceInfo& di = g_dev[dev];
-    if (di.sms == 0 && cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return ZYFA_ERR_CUDA;
-    if (!di.attr_set[inst]) {
-      if (cudaFuncSetAttribute(attn_fwd_kernel<FP8, DQK, EXACTP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cf::SMEM) != cudaSuccess)
-        return ZYFA_ERR_CUDA;
-      di.attr_set[inst] = true;
-    }
+// SM count of the device, and the kernel instance's shared-memory opt-in (once)
+template <bool FP8, int DQK, bool EXACTP, bool VARLEN>
+bool prepare_device(int dev, int inst) {
+  using Cf = AttnCfg<FP8, DQK>;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (di.sms == 0 && cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return false;
+  if (!di.attr_set[inst]) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<FP8, DQK, EXACTP, VARLEN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM) != cudaSuccess)
+      return false;
+    di.attr_set[inst] = true;
   }
+  return true;
+}
+
+template <bool FP8, int DQK, bool EXACTP = false>
+int launch_attn(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int S,
+                const float* qs, const float* ks, const float* vs, cudaStream_t stream, int dev,
+                int inst, float* lse = nullptr) {
+  using Cf = AttnCfg<FP8, DQK>;
+  AttnArgs a;
+  if (!fill_attn_args<FP8, DQK>(a, q, k, v, o, B, Hq, Hkv, S, qs, ks, vs, lse)) return ZYFA_ERR_CUDA;
+  a.B = B; a.S = S;
+  a.Tq = (S + 127) / 128;
+  a.group_slots = group_slots_for(B, Hkv, S, DQK, FP8 ? 1 : 2);
+  if (!prepare_device<FP8, DQK, EXACTP, false>(dev, inst)) return ZYFA_ERR_CUDA;
   const long long units = static_cast<long long>(B) * Hq * a.Tq;
   const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
-  attn_fwd_kernel<FP8, DQK, EXACTP><<<grid, kAttnThreads, Cf::SMEM, stream>>>(a);
+  attn_fwd_kernel<FP8, DQK, EXACTP><<<grid, kAttnThreads, Cf::SMEM, stream>>>(a, SeqTable<false>{});
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+// Variable-length batch: q/k/v/o packed [T, H, D] with T = cu[nseq].
+template <bool FP8, int DQK>
+int launch_attn_varlen(const void* q, const void* k, const void* v, void* o, const int* cu, int nseq, int Hq,
+                       int Hkv, const float* qs, const float* ks, const float* vs, cudaStream_t stream, int dev,
+                       int inst, float* lse) {
+  using Cf = AttnCfg<FP8, DQK>;
+  const long long units = varlen_units(cu, nseq, Hq);
+  if (units == 0) return ZYFA_OK;   // every sequence empty: nothing to write
+  const int T = cu[nseq];
+  AttnArgs a;
+  if (!fill_attn_args<FP8, DQK>(a, q, k, v, o, 1, Hq, Hkv, T, qs, ks, vs, lse)) return ZYFA_ERR_CUDA;
+  a.B = nseq; a.S = T;
+  a.Tq = 0; a.group_slots = 0;   // the sequence table drives the schedule
+  SeqTable<true> t;
+  fill_varlen_table(t, cu, nseq, DQK, FP8 ? 1 : 2);
+  if (!prepare_device<FP8, DQK, false, true>(dev, inst)) return ZYFA_ERR_CUDA;
+  const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
+  attn_fwd_kernel<FP8, DQK, false, true><<<grid, kAttnThreads, Cf::SMEM, stream>>>(a, t);
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
@@ -355,6 +424,198 @@ extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, in
   }
   quant3_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(q_scale, k_scale, v_scale, n0, n1, n2);
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- variable-length batches
+
+// cu: host array of nseq + 1 packed-row offsets, cu[0] = 0, non-decreasing
+static int cu_validate(const int* cu, int nseq, int max_seqs) {
+  if (!cu) return ZYFA_ERR_NULL_PTR;
+  if (nseq < 1 || nseq > max_seqs) return ZYFA_ERR_BAD_SHAPE;
+  if (cu[0] != 0) return ZYFA_ERR_BAD_SHAPE;
+  for (int i = 0; i < nseq; ++i)
+    if (cu[i + 1] < cu[i]) return ZYFA_ERR_BAD_SHAPE;
+  return ZYFA_OK;
+}
+
+extern "C" int zyfa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                                    const int* cu_seqlens, int nseq, int Hq, int Hkv, int Dqk, int Dv, int dtype,
+                                    const float* q_scale, const float* k_scale, const float* v_scale,
+                                    void* stream) {
+  const int badc = cu_validate(cu_seqlens, nseq, kMaxVarlenSeqs);
+  if (badc != ZYFA_OK) return badc;
+  const int T = cu_seqlens[nseq];
+  if (T == 0) {   // every sequence empty: tensors may be NULL, nothing is launched
+    if (Hq < 1 || Hkv < 1) return ZYFA_ERR_BAD_SHAPE;
+    if (Hq % Hkv != 0) return ZYFA_ERR_BAD_GQA;
+    if (!((Dqk == 128 || Dqk == 192) && Dv == 128)) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+    if (dtype != ZYFA_BF16 && dtype != ZYFA_FP8_E4M3) return ZYFA_ERR_BAD_DTYPE;
+    return ZYFA_OK;
+  }
+  // the checks of the fixed-length form, on one batch of T rows
+  const int bad = attn_validate(q, k, v, o, 1, Hq, Hkv, T, Dqk, Dv, dtype, q_scale, k_scale, v_scale);
+  if (bad != ZYFA_OK) return bad;
+  const long long units = varlen_units(cu_seqlens, nseq, Hq);
+  if (units > (1ll << 31) - 1) return ZYFA_ERR_BAD_SHAPE;
+  if (lse && !aligned(lse, 4)) return ZYFA_ERR_MISALIGNED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == ZYFA_FP8_E4M3) {
+    if (Dqk == 128)
+      return launch_attn_varlen<true, 128>(q, k, v, o, cu_seqlens, nseq, Hq, Hkv, q_scale, k_scale, v_scale, st,
+                                           dev, 6, lse);
+    return launch_attn_varlen<true, 192>(q, k, v, o, cu_seqlens, nseq, Hq, Hkv, q_scale, k_scale, v_scale, st,
+                                         dev, 7, lse);
+  }
+  if (Dqk == 128)
+    return launch_attn_varlen<false, 128>(q, k, v, o, cu_seqlens, nseq, Hq, Hkv, nullptr, nullptr, nullptr, st,
+                                          dev, 8, lse);
+  return launch_attn_varlen<false, 192>(q, k, v, o, cu_seqlens, nseq, Hq, Hkv, nullptr, nullptr, nullptr, st,
+                                        dev, 9, lse);
+}
+
+// The prepass over a packed batch for n (1 or 3) tensors sharing cu.
+static int quantize_varlen_n(int n, const void* const* xs, void* const* outs, float* const* scs, const int* Hs,
+                             const int* Ds, const int* had, int in_dtype, const int* cu, int nseq, void* stream) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ZYFA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ZYFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int max_len = 0;
+  for (int i = 0; i < nseq; ++i) max_len = std::max(max_len, cu[i + 1] - cu[i]);
+  const int T = cu[nseq];
+  // CTAs per average sequence as in the fixed-length prepass, split among
+  // the tensors in proportion to their bytes; a longer sequence gets
+  // proportionally more chunks of the same height
+  const long long mean_len = std::max(1ll, (static_cast<long long>(T) + nseq - 1) / nseq);
+  bool any_had = false;
+  double bytes[3] = {0.0, 0.0, 0.0}, total = 0.0;
+  for (int i = 0; i < n; ++i) {
+    bytes[i] = static_cast<double>(Hs[i]) * Ds[i];
+    total += bytes[i];
+    any_had = any_had || had[i];
+  }
+  const double want = static_cast<double>(((any_had ? 8ll : 4ll) * sms + nseq - 1) / nseq);
+  Quant3VarArgs a;
+  Quant3Args& q3 = a.q;
+  q3.first[0] = 0;
+  int max_h = 1;
+  for (int i = 0; i < 3; ++i) {
+    QuantArgs& t = q3.t[i];
+    if (i >= n) {   // unused slots: no CTA columns
+      t = q3.t[0];
+      q3.had[i] = 0;
+      q3.first[i + 1] = q3.first[i];
+      continue;
+    }
+    long long chunks = static_cast<long long>(want * bytes[i] / total + 0.5);
+    if (chunks < 1) chunks = 1;
+    if (chunks > mean_len) chunks = mean_len;
+    t.x = xs[i];
+    t.out = static_cast<uint8_t*>(outs[i]);
+    t.scale = scs[i];
+    t.S = 0;
+    t.H = Hs[i]; t.D = Ds[i];
+    t.rows_per_cta = static_cast<int>((mean_len + chunks - 1) / chunks);
+    q3.had[i] = had[i];
+    q3.first[i + 1] = q3.first[i] + (max_len + t.rows_per_cta - 1) / t.rows_per_cta;
+    max_h = std::max(max_h, Hs[i]);
+  }
+  for (int i = 0; i <= nseq; ++i) a.cu[i] = cu[i];
+  const int n0 = nseq * Hs[0], n1 = n > 1 ? nseq * Hs[1] : 0, n2 = n > 2 ? nseq * Hs[2] : 0;
+  const int nn = n0 + n1 + n2;
+  float* s1 = n > 1 ? scs[1] : scs[0];
+  float* s2 = n > 2 ? scs[2] : scs[0];
+  quant3_zero_kernel<<<(nn + 255) / 256, 256, 0, st>>>(scs[0], s1, s2, n0, n1, n2);
+  if (q3.first[3] > 0) {   // some sequence has rows
+    const dim3 grid(static_cast<unsigned>(q3.first[3]), static_cast<unsigned>(nseq));
+    const size_t shm = static_cast<size_t>(max_h) * 8;   // amax, or scale and its reciprocal, per head
+    if (in_dtype == ZYFA_BF16) {
+      quant3v_amax_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
+      quant3v_codes_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
+    } else {
+      quant3v_amax_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
+      quant3v_codes_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
+    }
+  }
+  quant3_finalize_kernel<<<(nn + 255) / 256, 256, 0, st>>>(scs[0], s1, s2, n0, n1, n2);
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+extern "C" int zyfa_quantize_varlen(const void* x, int in_dtype, void* x_fp8, float* scale, const int* cu_seqlens,
+                                    int nseq, int H, int D, int hadamard, void* stream) {
+  const int badc = cu_validate(cu_seqlens, nseq, kMaxQuantSeqs);
+  if (badc != ZYFA_OK) return badc;
+  if (!scale || (cu_seqlens[nseq] > 0 && (!x || !x_fp8))) return ZYFA_ERR_NULL_PTR;
+  if (H < 1 || H > 4096) return ZYFA_ERR_BAD_SHAPE;
+  if (in_dtype != ZYFA_BF16 && in_dtype != ZYFA_FP32) return ZYFA_ERR_BAD_DTYPE;
+  if (hadamard != 0 && hadamard != 1) return ZYFA_ERR_BAD_DTYPE;
+  if (D < 8 || D > 1024 || D % 8 != 0 || (hadamard && D != 128 && D != 192)) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (!aligned(x, 16) || !aligned(x_fp8, 16) || !aligned(scale, 4)) return ZYFA_ERR_MISALIGNED;
+  const void* xs[1] = {x};
+  void* outs[1] = {x_fp8};
+  float* scs[1] = {scale};
+  const int Hs[1] = {H}, Ds[1] = {D}, had[1] = {hadamard};
+  return quantize_varlen_n(1, xs, outs, scs, Hs, Ds, had, in_dtype, cu_seqlens, nseq, stream);
+}
+
+extern "C" int zyfa_quantize_qkv_varlen(const void* q, const void* k, const void* v, int in_dtype, void* q_fp8,
+                                        void* k_fp8, void* v_fp8, float* q_scale, float* k_scale, float* v_scale,
+                                        const int* cu_seqlens, int nseq, int Hq, int Hkv, int Dqk, int Dv,
+                                        int hadamard_qk, void* stream) {
+  const int badc = cu_validate(cu_seqlens, nseq, kMaxQuantSeqs);
+  if (badc != ZYFA_OK) return badc;
+  if (!q_scale || !k_scale || !v_scale) return ZYFA_ERR_NULL_PTR;
+  if (cu_seqlens[nseq] > 0 && (!q || !k || !v || !q_fp8 || !k_fp8 || !v_fp8)) return ZYFA_ERR_NULL_PTR;
+  if (Hq < 1 || Hkv < 1 || Hq > 4096 || Hkv > 4096) return ZYFA_ERR_BAD_SHAPE;
+  if (in_dtype != ZYFA_BF16 && in_dtype != ZYFA_FP32) return ZYFA_ERR_BAD_DTYPE;
+  if (hadamard_qk != 0 && hadamard_qk != 1) return ZYFA_ERR_BAD_DTYPE;
+  for (int d : {Dqk, Dv})
+    if (d < 8 || d > 1024 || d % 8 != 0) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (hadamard_qk && Dqk != 128 && Dqk != 192) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  for (const void* t : {q, k, v, static_cast<const void*>(q_fp8), static_cast<const void*>(k_fp8),
+                        static_cast<const void*>(v_fp8)})
+    if (!aligned(t, 16)) return ZYFA_ERR_MISALIGNED;
+  if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4)) return ZYFA_ERR_MISALIGNED;
+  const void* xs[3] = {q, k, v};
+  void* outs[3] = {q_fp8, k_fp8, v_fp8};
+  float* scs[3] = {q_scale, k_scale, v_scale};
+  const int Hs[3] = {Hq, Hkv, Hkv}, Ds[3] = {Dqk, Dqk, Dv}, had[3] = {hadamard_qk, hadamard_qk, 0};
+  return quantize_varlen_n(3, xs, outs, scs, Hs, Ds, had, in_dtype, cu_seqlens, nseq, stream);
+}
+
+extern "C" int zyfa_attn_schedule(int B, int S, const int* cu_seqlens, int Hq, int Hkv, int Dqk, int dtype,
+                                  int grid, int cta, int* units, int cap) {
+  if (Hq < 1 || Hkv < 1 || grid < 1 || cta < 0 || cta >= grid || cap < 0) return ZYFA_ERR_BAD_SHAPE;
+  if (Hq % Hkv != 0) return ZYFA_ERR_BAD_GQA;
+  if (Dqk != 128 && Dqk != 192) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  if (dtype != ZYFA_BF16 && dtype != ZYFA_FP8_E4M3) return ZYFA_ERR_BAD_DTYPE;
+  if (cap > 0 && !units) return ZYFA_ERR_NULL_PTR;
+  const int el = dtype == ZYFA_FP8_E4M3 ? 1 : 2;
+  int n = 0, b, hkv, hq, qt, r0, len;
+  auto put = [&]() {
+    if (n < cap) { units[3 * n] = b; units[3 * n + 1] = hq; units[3 * n + 2] = qt; }
+    ++n;
+  };
+  if (cu_seqlens) {
+    const int badc = cu_validate(cu_seqlens, B, kMaxVarlenSeqs);
+    if (badc != ZYFA_OK) return badc;
+    if (varlen_units(cu_seqlens, B, Hq) > (1ll << 31) - 1) return ZYFA_ERR_BAD_SHAPE;
+    VarlenSeqs t;
+    fill_varlen_table(t, cu_seqlens, B, Dqk, el);
+    VarlenIter it;
+    it.init(grid, cta, &t, Hq, Hkv);
+    while (it.next(b, hkv, hq, qt, r0, len)) put();
+  } else {
+    if (B < 1 || S < 1) return ZYFA_ERR_BAD_SHAPE;
+    const long long tq = (static_cast<long long>(S) + 127) / 128;
+    if (static_cast<long long>(B) * Hq * tq > (1ll << 31) - 1) return ZYFA_ERR_BAD_SHAPE;
+    UnitIter it;
+    it.init(grid, cta, static_cast<int>(tq), Hq, Hkv, B, group_slots_for(B, Hkv, S, Dqk, el));
+    while (it.next(b, hkv, hq, qt)) put();
+  }
+  return n;
 }
 
 extern "C" int zyfa_device_status(void* stream) {

@@ -46,6 +46,14 @@ def lib() -> ctypes.CDLL:
         L.zyfa_quantize.argtypes = [p, i, p, p, i, i, i, i, i, p]
         L.zyfa_quantize_qkv.restype = i
         L.zyfa_quantize_qkv.argtypes = [p, p, p, i, p, p, p, p, p, p, i, i, i, i, i, i, i, p]
+        L.zyfa_attn_fwd_varlen.restype = i
+        L.zyfa_attn_fwd_varlen.argtypes = [p, p, p, p, p, p, i, i, i, i, i, i, p, p, p, p]
+        L.zyfa_quantize_varlen.restype = i
+        L.zyfa_quantize_varlen.argtypes = [p, i, p, p, p, i, i, i, i, p]
+        L.zyfa_quantize_qkv_varlen.restype = i
+        L.zyfa_quantize_qkv_varlen.argtypes = [p, p, p, i, p, p, p, p, p, p, p, i, i, i, i, i, i, p]
+        L.zyfa_attn_schedule.restype = i
+        L.zyfa_attn_schedule.argtypes = [i, i, p, i, i, i, i, i, i, p, i]
         L.zyfa_status_string.restype = ctypes.c_char_p
         L.zyfa_status_string.argtypes = [i]
         L.zyfa_device_status.restype = i
@@ -185,6 +193,134 @@ def quantize_qkv(q, k, v, hadamard_qk=False, out=None, stream=None):
                                  _ptr(vs), B, S, Hq, Hkv, Dqk, Dv, int(bool(hadamard_qk)), _stream(stream))
     _check(st, "zyfa_quantize_qkv")
     return out
+
+
+def _cu_host(cu_seqlens, rows=None):
+    """cu_seqlens (list, numpy array or CPU tensor of nseq + 1 ints) -> (ctypes int array, nseq).
+    rows: the packed tensors' row count, which must equal cu_seqlens[-1]."""
+    if isinstance(cu_seqlens, torch.Tensor):
+        if cu_seqlens.is_cuda:
+            raise ValueError("cu_seqlens must be host memory (a CPU tensor or a list)")
+        cu_seqlens = cu_seqlens.tolist()
+    vals = [int(x) for x in cu_seqlens]
+    if len(vals) < 2:
+        raise ValueError("cu_seqlens needs nseq + 1 >= 2 entries")
+    if rows is not None and vals[-1] != rows:
+        raise ValueError(f"cu_seqlens[-1] = {vals[-1]} but the packed tensors hold {rows} rows")
+    return (ctypes.c_int * len(vals))(*vals), len(vals) - 1
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens, o=None, q_scale=None, k_scale=None, v_scale=None, lse=False,
+                    stream=None):
+    """Causal attention over a packed batch (zyfa_attn_fwd_varlen).  q [T,Hq,Dqk], k [T,Hkv,Dqk],
+    v [T,Hkv,Dv] with sequence s at rows cu_seqlens[s] .. cu_seqlens[s+1]-1; bf16, or e4m3 codes
+    with fp32 scales [nseq,H].  Returns o [T,Hq,Dv] bf16, or (o, lse [Hq,T] fp32) with lse=True
+    (or an fp32 [Hq,T] tensor)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if q.dtype == torch.bfloat16:
+        dt = BF16
+    elif q.dtype in (torch.uint8, torch.float8_e4m3fn):
+        dt = FP8_E4M3
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    T, Hq, Dqk = q.shape
+    Hkv, Dv = k.shape[1], v.shape[2]
+    for t, n in ((k, "k"), (v, "v")):
+        if t.shape[0] != T:
+            raise ValueError(f"{n} holds {t.shape[0]} rows, q holds {T}")
+    cu, nseq = _cu_host(cu_seqlens, T)
+    if o is None:
+        o = torch.empty((T, Hq, Dv), dtype=torch.bfloat16, device=q.device)
+    if o.shape[0] != T:
+        raise ValueError(f"o holds {o.shape[0]} rows, q holds {T}")
+    _dev(o, "o")
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        if t is not None:
+            _dev(t, n)
+            if t.dtype != torch.float32:
+                raise ValueError(f"{n} must be fp32")
+    out = None
+    if lse is not False and lse is not None:
+        out = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if lse is True else lse
+        _dev(out, "lse")
+        if tuple(out.shape) != (Hq, T):
+            raise ValueError("lse must be [Hq, T]")
+    st = lib().zyfa_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(out), cu, nseq, Hq, Hkv, Dqk, Dv,
+                                    dt, _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream(stream))
+    _check(st, "zyfa_attn_fwd_varlen")
+    return o if out is None else (o, out)
+
+
+def _in_dtype(x):
+    if x.dtype == torch.bfloat16:
+        return BF16
+    if x.dtype == torch.float32:
+        return FP32
+    raise ValueError(f"unsupported input dtype {x.dtype}")
+
+
+def quantize_varlen(x, cu_seqlens, hadamard=False, out=None, scale=None, stream=None):
+    """x [T,H,D] bf16 or fp32, packed -> (codes uint8 [T,H,D], scale fp32 [nseq,H])."""
+    _dev(x, "x")
+    dt = _in_dtype(x)
+    T, H, D = x.shape
+    cu, nseq = _cu_host(cu_seqlens, T)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((nseq, H), dtype=torch.float32, device=x.device)
+    _dev(out, "out"); _dev(scale, "scale")
+    st = lib().zyfa_quantize_varlen(_ptr(x), dt, _ptr(out), _ptr(scale), cu, nseq, H, D, int(bool(hadamard)),
+                                    _stream(stream))
+    _check(st, "zyfa_quantize_varlen")
+    return out, scale
+
+
+def quantize_qkv_varlen(q, k, v, cu_seqlens, hadamard_qk=False, out=None, stream=None):
+    """Packed Q, K, V [T,H,D] (same dtype) -> ((q8, q_scale), (k8, k_scale), (v8, v_scale)), scales
+    [nseq,H]; identical to three quantize_varlen() calls, in four launches."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k and v must share a dtype")
+    dt = _in_dtype(q)
+    T, Hq, Dqk = q.shape
+    Hkv, Dv = k.shape[1], v.shape[2]
+    for t, n in ((k, "k"), (v, "v")):
+        if t.shape[0] != T:
+            raise ValueError(f"{n} holds {t.shape[0]} rows, q holds {T}")
+    cu, nseq = _cu_host(cu_seqlens, T)
+    if out is None:
+        out = tuple((torch.empty(t.shape, dtype=torch.uint8, device=t.device),
+                     torch.empty((nseq, t.shape[1]), dtype=torch.float32, device=t.device)) for t in (q, k, v))
+    for (c, sc), n in zip(out, "qkv"):
+        _dev(c, n + "_fp8"); _dev(sc, n + "_scale")
+    (q8, qs), (k8, ks), (v8, vs) = out
+    st = lib().zyfa_quantize_qkv_varlen(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
+                                        _ptr(ks), _ptr(vs), cu, nseq, Hq, Hkv, Dqk, Dv, int(bool(hadamard_qk)),
+                                        _stream(stream))
+    _check(st, "zyfa_quantize_qkv_varlen")
+    return out
+
+
+def attn_schedule(Hq, Hkv, Dqk, dtype, grid, cta, B=None, S=None, cu_seqlens=None):
+    """Host-only: the (b, hq, qt) units CTA `cta` of a `grid`-CTA launch runs, in order (a list of
+    tuples).  Fixed length: B and S; packed batch: cu_seqlens."""
+    if cu_seqlens is not None:
+        cu, nseq = _cu_host(cu_seqlens)
+        B, S = nseq, 0
+    else:
+        cu = None
+    L = lib()
+    n = L.zyfa_attn_schedule(B, S, cu, Hq, Hkv, Dqk, dtype, grid, cta, None, 0)
+    if n < 0:
+        raise ZyfaError(n, "zyfa_attn_schedule")
+    buf = (ctypes.c_int * max(1, 3 * n))()
+    m = L.zyfa_attn_schedule(B, S, cu, Hq, Hkv, Dqk, dtype, grid, cta, buf, n)
+    if m != n:
+        raise ZyfaError(m if m < 0 else -2, "zyfa_attn_schedule")
+    return [(buf[3 * i], buf[3 * i + 1], buf[3 * i + 2]) for i in range(n)]
 
 
 def leanp_codes(s, m, bmax, A, masked=None, stream=None):

@@ -11,8 +11,9 @@
  *   spke.com, "Zyphra ZYFA: AMD MI355X向けFP8 FlashAttention、最大1.76倍高速化"
  *
  * Conventions for every entry point:
- *  - Pointers named q, k, v, o, x, x_fp8, scale, *_scale and the Lean-P test
- *    arrays are DEVICE pointers (CUDA global memory of the current device).
+ *  - Pointers named q, k, v, o, lse, x, x_fp8, scale, *_scale and the Lean-P
+ *    test arrays are DEVICE pointers (CUDA global memory of the current
+ *    device); cu_seqlens and the schedule query's units are HOST arrays.
  *    The caller allocates and owns every buffer; the library allocates no
  *    memory and keeps no state between calls other than one device error
  *    word (see zyfa_device_status) and per-device launch attributes.
@@ -180,6 +181,79 @@ int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* scale, int B,
 int zyfa_quantize_qkv(const void* q, const void* k, const void* v, int in_dtype, void* q_fp8,
                       void* k_fp8, void* v_fp8, float* q_scale, float* k_scale, float* v_scale,
                       int B, int S, int Hq, int Hkv, int Dqk, int Dv, int hadamard_qk, void* stream);
+
+/*
+ * Variable-length batches.  The pages list them as future work for the
+ * method (ai-daily-news.org "Zyphra ZYFA", "Qué cubren los kernels": no
+ * decode, no paged KV caches, no variable-length batches); these entries
+ * extend the same computation to a packed batch of independent sequences.
+ *
+ * Packing: sequence s (0 <= s < nseq) holds rows cu_seqlens[s] ..
+ * cu_seqlens[s+1]-1 of every tensor; T = cu_seqlens[nseq] rows in all.
+ * cu_seqlens is a HOST array of nseq + 1 ints (read during the call, not
+ * kept): cu_seqlens[0] = 0, non-decreasing (empty sequences allowed).
+ * 1 <= nseq <= 384 per call.  Every sequence is causal on its own: row i of
+ * sequence s attends to rows 0..i of s only, and its output does not depend
+ * on the other sequences of the batch (FP8: each sequence has its own
+ * scales).  Precondition: the inputs are finite (a non-finite value could
+ * reach a neighbouring sequence through a masked, zero weight).
+ */
+
+/*
+ * zyfa_attn_fwd_varlen -- zyfa_attn_fwd over a packed batch.
+ *   q  [T, Hq,  Dqk], k [T, Hkv, Dqk], v [T, Hkv, Dv]   dtype elements
+ *   o  [T, Hq,  Dv ]  bfloat16 (every row of every sequence written)
+ *   lse [Hq, T] fp32, or NULL: each row's log-sum-exp as in zyfa_attn_fwd_lse
+ *   q_scale [nseq*Hq], k_scale [nseq*Hkv], v_scale [nseq*Hkv] (FP8; device;
+ *     NULL = 1.0), indexed s*H + h: one scale per (sequence, head).
+ * Each row's output is bit-identical to zyfa_attn_fwd (B = 1) on its
+ * sequence alone.  Scheduling: sequences longest first, heaviest query tiles
+ * first, K/V of a group of (sequence, kv head) slots kept in L2.
+ * Errors: NULL_PTR (a tensor or cu_seqlens NULL), BAD_SHAPE (nseq out of
+ * range, cu_seqlens not as above), BAD_GQA, UNSUPPORTED_HEADDIM, BAD_DTYPE,
+ * MISALIGNED (tensors 16-byte, scales and lse 4-byte), CUDA.  T = 0 is valid
+ * and launches nothing (the tensor pointers may then be NULL).  The library
+ * cannot see tensor sizes: each tensor must hold T rows.
+ */
+int zyfa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const int* cu_seqlens, int nseq, int Hq, int Hkv, int Dqk, int Dv, int dtype,
+                         const float* q_scale, const float* k_scale, const float* v_scale, void* stream);
+
+/*
+ * zyfa_quantize_varlen -- zyfa_quantize over a packed batch: x and x_fp8
+ * [T, H, D], scale [nseq*H] (output), one scale per (sequence, head), so the
+ * codes and scale of sequence s equal zyfa_quantize (B = 1) on its rows
+ * alone (an empty sequence gets scale 1.0).  Other arguments and errors as
+ * zyfa_quantize, plus the cu_seqlens rules above; with T = 0, x and x_fp8
+ * may be NULL (only the scales are written).
+ */
+int zyfa_quantize_varlen(const void* x, int in_dtype, void* x_fp8, float* scale, const int* cu_seqlens,
+                         int nseq, int H, int D, int hadamard, void* stream);
+
+/*
+ * zyfa_quantize_qkv_varlen -- zyfa_quantize_qkv over a packed batch: byte for
+ * byte zyfa_quantize_varlen on Q and K (hadamard_qk) and on V (no rotation),
+ * in four launches.  q [T, Hq, Dqk], k [T, Hkv, Dqk], v [T, Hkv, Dv];
+ * scales [nseq*Hq], [nseq*Hkv], [nseq*Hkv].
+ */
+int zyfa_quantize_qkv_varlen(const void* q, const void* k, const void* v, int in_dtype, void* q_fp8,
+                             void* k_fp8, void* v_fp8, float* q_scale, float* k_scale, float* v_scale,
+                             const int* cu_seqlens, int nseq, int Hq, int Hkv, int Dqk, int Dv,
+                             int hadamard_qk, void* stream);
+
+/*
+ * zyfa_attn_schedule -- host only (no device call): the work units that CTA
+ * `cta` of a `grid`-CTA attention launch processes, in order, as the kernel
+ * enumerates them.  A unit is (b, hq, qt): query tile qt (rows 128 qt ..
+ * 128 qt + 127) of query head hq of batch entry / sequence b, which takes
+ * key tiles 0..qt.  Fixed length: cu_seqlens = NULL, B entries of S rows.
+ * Packed: cu_seqlens as above with nseq = B (S ignored).  The launch itself
+ * uses grid = min(units, SM count).  Writes min(count, cap) units as int
+ * triples to `units` (host memory) and returns the count, or a negative
+ * status (BAD_SHAPE, BAD_GQA, UNSUPPORTED_HEADDIM, BAD_DTYPE, NULL_PTR).
+ */
+int zyfa_attn_schedule(int B, int S, const int* cu_seqlens, int Hq, int Hkv, int Dqk, int dtype, int grid,
+                       int cta, int* units, int cap);
 
 /* Human-readable text of a status code (static storage; never NULL). */
 const char* zyfa_status_string(int status);

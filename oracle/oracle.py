@@ -223,6 +223,73 @@ def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=
     return (o, lse) if return_lse else o
 
 
+# --- variable-length (packed) batches ------------------------------------------
+# A packed batch holds independent sequences back to back: sequence s is rows
+# cu[s] .. cu[s+1]-1 of every [T, H, D] tensor.  Each function below is its
+# fixed-length counterpart applied to every sequence alone (a batch of one),
+# results placed at the sequence's rows; nothing else is computed.
+
+def _spans(cu):
+    cu = [int(x) for x in cu]
+    return [(cu[s], cu[s + 1]) for s in range(len(cu) - 1)]
+
+
+def attention_varlen(q, k, v, cu, sm_scale=None) -> np.ndarray:
+    """q [T,Hq,Dqk], k [T,Hkv,Dqk], v [T,Hkv,Dv] -> o [T,Hq,Dv] fp64, causal per sequence."""
+    T, Hq = q.shape[0], q.shape[1]
+    o = np.zeros((T, Hq, v.shape[2]), dtype=np.float64)
+    for r0, r1 in _spans(cu):
+        if r1 > r0:
+            o[r0:r1] = attention(q[None, r0:r1], k[None, r0:r1], v[None, r0:r1], sm_scale=sm_scale)[0]
+    return o
+
+
+def attention_lse_varlen(q, k, cu, sm_scale=None) -> np.ndarray:
+    """Log-sum-exp of each row's causal scores within its sequence: lse [Hq, T] fp64."""
+    T, Hq = q.shape[0], q.shape[1]
+    lse = np.zeros((Hq, T), dtype=np.float64)
+    for r0, r1 in _spans(cu):
+        if r1 > r0:
+            lse[:, r0:r1] = attention_lse(q[None, r0:r1], k[None, r0:r1], sm_scale=sm_scale)[0]
+    return lse
+
+
+def quantize_varlen(x, cu, hadamard: bool = False):
+    """x [T,H,D] -> (codes uint8 [T,H,D], scale fp32 [nseq,H]): each sequence quantized alone; an
+    empty sequence gets the scale of an all-zero input."""
+    x = _c(x, np.float32)
+    T, H, D = x.shape
+    spans = _spans(cu)
+    codes = np.zeros((T, H, D), dtype=np.uint8)
+    scale = np.empty((len(spans), H), dtype=np.float32)
+    for s, (r0, r1) in enumerate(spans):
+        part = x[None, r0:r1] if r1 > r0 else np.zeros((1, 1, H, D), dtype=np.float32)
+        c, sc = quantize(part, hadamard=hadamard)
+        if r1 > r0:
+            codes[r0:r1] = c[0]
+        scale[s] = sc[0]
+    return codes, scale
+
+
+def fp8_model_varlen(qc, kc, vc, q_s, k_s, v_s, cu, rescale_log2=0.0, p_mode=0, return_lse=False):
+    """fp8_model over a packed batch: codes [T,H,D], scales [nseq,H].  Returns o [T,Hq,Dv] (and
+    lse [Hq,T] with return_lse)."""
+    T, Hq = qc.shape[0], qc.shape[1]
+    o = np.zeros((T, Hq, vc.shape[2]), dtype=np.float64)
+    lse = np.zeros((Hq, T), dtype=np.float64)
+    for s, (r0, r1) in enumerate(_spans(cu)):
+        if r1 == r0:
+            continue
+        res = fp8_model(qc[None, r0:r1], kc[None, r0:r1], vc[None, r0:r1], q_s[s:s + 1], k_s[s:s + 1],
+                        v_s[s:s + 1], rescale_log2=rescale_log2, p_mode=p_mode, return_lse=return_lse)
+        if return_lse:
+            o[r0:r1] = res[0][0]
+            lse[:, r0:r1] = res[1][0]
+        else:
+            o[r0:r1] = res[0]
+    return (o, lse) if return_lse else o
+
+
 def rel_fro(a, b) -> float:
     """||a - b||_F / ||b||_F in fp64."""
     a = np.asarray(a, dtype=np.float64); b = np.asarray(b, dtype=np.float64)

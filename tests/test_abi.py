@@ -16,7 +16,8 @@ def L():
 def test_every_declared_symbol_is_exported(L):
     names = zyfa.declared_symbols()
     assert set(names) >= {"zyfa_attn_fwd", "zyfa_attn_fwd_lse", "zyfa_attn_fwd_fp8_exact_p", "zyfa_quantize",
-                          "zyfa_quantize_qkv",
+                          "zyfa_quantize_qkv", "zyfa_attn_fwd_varlen", "zyfa_quantize_varlen",
+                          "zyfa_quantize_qkv_varlen", "zyfa_attn_schedule",
                           "zyfa_status_string",
                           "zyfa_device_status",
                           "zyfa_leanp_codes", "zyfa_selftest_wait_timeout", "zyfa_set_wait_timeout_ns"}
@@ -116,3 +117,58 @@ def test_leanp_and_selftest_argument_errors(L):
     assert L.zyfa_leanp_codes(None, None, None, None, None, 0, None, None, None) == 0
     assert L.zyfa_leanp_codes(None, FAKE, FAKE, FAKE, None, 4, FAKE, None, None) == -1
     assert L.zyfa_selftest_wait_timeout(ctypes.c_ulonglong(2_000_000_000), None) == -2
+
+
+def _cu(vals):
+    return (ctypes.c_int * len(vals))(*vals)
+
+
+def test_varlen_argument_errors(L):
+    def e(cu=(0, 100, 300), nseq=None, q=FAKE, o=FAKE, lse=None, Hq=2, Hkv=2, Dqk=128, Dv=128, dt=0, qs=None):
+        c = None if cu is None else _cu(cu)
+        n = (len(cu) - 1) if nseq is None else nseq
+        return L.zyfa_attn_fwd_varlen(q, FAKE, FAKE, o, lse, c, n, Hq, Hkv, Dqk, Dv, dt, qs, None, None, None)
+    assert e(cu=None, nseq=2) == -1
+    assert e(q=None) == -1
+    assert e(nseq=0) == -2
+    assert e(cu=[0] * 386) == -2                      # more than 384 sequences
+    assert e(cu=(1, 100, 300)) == -2                  # cu[0] != 0
+    assert e(cu=(0, 300, 100)) == -2                  # decreasing
+    assert e(Hq=3) == -4
+    assert e(Dqk=64) == -3
+    assert e(dt=2) == -6
+    assert e(q=FAKE + 8) == -5
+    assert e(lse=FAKE + 2) == -5
+    assert e(dt=1, qs=FAKE + 1) == -5
+    assert e(cu=(0, 0, 0)) == 0                       # every sequence empty: nothing to launch
+    assert e(cu=[0] * 385) == 0                       # 384 empty sequences
+    assert e(cu=(0, 0), q=None, o=None) == 0          # nothing to read or write
+    assert e(cu=(0, 0), Hq=3) == -4
+
+
+def test_quantize_varlen_argument_errors(L):
+    def e(cu=(0, 10, 30), nseq=None, x=FAKE, H=2, D=128, had=0, dt=0):
+        c = None if cu is None else _cu(cu)
+        n = (len(cu) - 1) if nseq is None else nseq
+        return L.zyfa_quantize_varlen(x, dt, FAKE, FAKE, c, n, H, D, had, None)
+    assert e(x=None) == -1
+    assert e(cu=None, nseq=2) == -1
+    assert e(nseq=0) == -2
+    assert e(cu=(0, 5, 4)) == -2
+    assert e(cu=[0] * 386) == -2
+    assert e(H=0) == -2
+    assert e(D=100) == -3
+    assert e(D=64, had=1) == -3
+    assert e(dt=1) == -6
+    assert e(had=2) == -6
+    assert e(x=FAKE + 4) == -5
+
+    def e3(cu=(0, 10, 30), Hq=4, Hkv=2, Dqk=192, Dv=128, had=1):
+        c = _cu(cu)
+        return L.zyfa_quantize_qkv_varlen(FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, c, len(cu) - 1,
+                                          Hq, Hkv, Dqk, Dv, had, None)
+    assert e3(cu=(0, 10, 3)) == -2
+    assert e3(Hkv=0) == -2
+    assert e3(Dqk=64) == -3
+    assert e3(Dv=12) == -3
+    assert e3(had=3) == -6
