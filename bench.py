@@ -163,7 +163,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.VARLEN_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--energy", type=float, default=0.0, metavar="SECONDS",
@@ -175,6 +176,11 @@ def main():
                     help="rotate Q and K by the Hadamard transform in the prepass (H128; H128 + H64 for Dqk 192)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.workload in synth.VARLEN_WORKLOADS:
+        wl = varlen_workload(args.workload, args.seed)
+        if args.impl == "reference":
+            return run_reference(args, wl)
+        return run_varlen(args, wl)
     wl = dict(synth.WORKLOADS[args.workload])
     if args.impl == "reference":
         return run_reference(args, wl)
@@ -229,7 +235,7 @@ def run_reference(args, wl):
         times.append(time.perf_counter() - t0)
     tot = sum(times)
     val = fl * args.steps / tot / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC_VARLEN if "lens" in wl else METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
@@ -472,6 +478,220 @@ def run_ours(args, wl):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                 "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize_qkv -> zyfa_attn_fwd -> D2H O"},
         "gpu_launches": args.steps * (launches_per_fp8_step + 1),
+        "clocks": clk,
+        "parity": parity,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+# ----------------------------------------------------------------- packed batches
+
+METRIC_VARLEN = "causal prefill attn TFLOP/s, packed variable-length batch (FP8 e4m3 & BF16, D=128)"
+
+
+def varlen_workload(name, seed):
+    """The packed workload: its lengths and offsets, and (for the reference arm
+    and the CPU baseline) the longest sequence as a one-sequence workload."""
+    wl = dict(synth.VARLEN_WORKLOADS[name])
+    lens = synth.varlen_lengths(seed, wl["nseq"], wl["lo"], wl["hi"])
+    wl["lens"] = lens
+    wl["cu"] = [0] + [int(x) for x in np.cumsum(lens)]
+    wl["B"], wl["S"] = 1, max(lens)
+    return wl
+
+
+def varlen_flops(lens, Hq, Dqk, Dv):
+    return sum(synth.causal_flops(1, n, Hq, Dqk, Dv) for n in lens)
+
+
+def varlen_parity_sequences(lens):
+    """Indices of the sequences the sampled parity check covers: the longest,
+    the shortest non-empty one and the median."""
+    order = sorted((n, s) for s, n in enumerate(lens) if n > 0)
+    pick = [order[-1][1], order[0][1], order[len(order) // 2][1]]
+    return sorted(set(pick))
+
+
+def run_varlen(args, wl):
+    """One packed batch per step: zyfa_quantize_qkv_varlen + zyfa_attn_fwd_varlen
+    (FP8), and the BF16 varlen attention on the same inputs, timed as in
+    run_ours; parity on sampled rows of three sequences against the oracle."""
+    import torch
+    import torch.distributed as dist
+
+    from bf16_causal_prefill_fp8_b200 import zyfa
+
+    rank, world, local = _dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lens, cu = wl["lens"], wl["cu"]
+    T, Hq, Hkv, Dqk, Dv = cu[-1], wl["Hq"], wl["Hkv"], wl["Dqk"], wl["Dv"]
+    nseq = len(lens)
+    flops = varlen_flops(lens, Hq, Dqk, Dv)
+    peaks, peak_src = load_peaks()
+    q, k, v = synth.make_qkv(shard.rank_seed(args.seed, rank), 1, T, Hq, Hkv, Dqk, Dv, wl["kind"])
+    qb, kb, vb = (torch.from_numpy(x[0]).to(torch.bfloat16) for x in (q, k, v))
+    dq, dk, dv = (t.to(dev) for t in (qb, kb, vb))
+    cq, ck, cv = (torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in (dq, dk, dv))
+    sq = torch.empty((nseq, Hq), dtype=torch.float32, device=dev)
+    sk = torch.empty((nseq, Hkv), dtype=torch.float32, device=dev)
+    sv = torch.empty((nseq, Hkv), dtype=torch.float32, device=dev)
+    o8 = torch.empty((T, Hq, Dv), dtype=torch.bfloat16, device=dev)
+    ob = torch.empty_like(o8)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def prepass():
+        zyfa.quantize_qkv_varlen(dq, dk, dv, cu, hadamard_qk=args.hadamard, out=((cq, sq), (ck, sk), (cv, sv)))
+
+    def attn8():
+        zyfa.attn_fwd_varlen(cq, ck, cv, cu, o=o8, q_scale=sq, k_scale=sk, v_scale=sv)
+
+    def attnb():
+        zyfa.attn_fwd_varlen(dq, dk, dv, cu, o=ob)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fns, steps):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)] for _ in range(steps)]
+        for st in range(steps):
+            flush.zero_()
+            ev[st][0].record(stream)
+            for i, f in enumerate(fns):
+                f()
+                ev[st][i + 1].record(stream)
+        torch.cuda.synchronize()
+        return [[ev[st][i].elapsed_time(ev[st][i + 1]) for i in range(len(fns))] for st in range(steps)]
+
+    for _ in range(args.warmup):
+        prepass(); attn8(); attnb()
+    barrier()
+    if zyfa.device_status() != zyfa.OK:
+        raise RuntimeError("device wait timeout during warm-up")
+    props = torch.cuda.get_device_properties(dev)
+    bus = None
+    if all(hasattr(props, a) for a in ("pci_domain_id", "pci_bus_id", "pci_device_id")):
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    clocks = ClockSampler(bus) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    per8 = timed([prepass, attn8], args.steps)
+    barrier()
+    perb = timed([attnb], args.steps)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if zyfa.device_status() != zyfa.OK:
+        raise RuntimeError("device wait timeout in the timed region")
+    mx = lambda x: shard.max_over_ranks(x, device=dev)
+    ms8 = mx(sum(a + b for a, b in per8) / args.steps)
+    ms8_attn = mx(sum(b for _, b in per8) / args.steps)
+    ms8_pre = mx(sum(a for a, _ in per8) / args.steps)
+    msb = mx(sum(x[0] for x in perb) / args.steps)
+
+    pin = [t.pin_memory() for t in (qb, kb, vb)]
+    host_o = torch.empty(o8.shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(pin[0], non_blocking=True); dk.copy_(pin[1], non_blocking=True); dv.copy_(pin[2], non_blocking=True)
+        prepass(); attn8()
+        host_o.copy_(o8, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = mx(e0.elapsed_time(e1) / e2e_steps)
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    bf16_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    fp8_peak = bf16_sus * FP8_PER_BF16
+    ach8 = flops / (ms8_attn * 1e-3) / 1e12
+    achb = flops / (msb * 1e-3) / 1e12
+    parity, cpu = None, None
+    if world == 1:
+        from oracle import oracle as orc
+        xq, xk, xv = (t.float().numpy() for t in (qb, kb, vb))
+        codes = [orc.quantize_varlen(xq, cu, args.hadamard), orc.quantize_varlen(xk, cu, args.hadamard),
+                 orc.quantize_varlen(xv, cu, False)]
+        codes_equal = all(np.array_equal(g.cpu().numpy(), c) and np.array_equal(gs.cpu().numpy(), cs)
+                          for (g, gs), (c, cs) in zip(((cq, sq), (ck, sk), (cv, sv)), codes))
+        o8h, obh = o8.float().cpu().numpy(), ob.float().cpu().numpy()
+        err8, errb, err_unq, rows_total = [], [], [], 0
+        deq_long = None
+        t_orc, fl_orc = 0.0, 0.0
+        for s in varlen_parity_sequences(lens):
+            r0, r1 = cu[s], cu[s + 1]
+            rows = sample_rows(r1 - r0, 48)
+            deq = tuple(orc.dequantize(c[None, r0:r1], sc[s:s + 1]) for c, sc in codes)
+            t0 = time.perf_counter()
+            ref = orc.attention(*deq, rows=rows)[0]
+            t_orc += time.perf_counter() - t0
+            fl_orc += row_flops(rows, Hq, Dqk, Dv, 1)
+            refb = orc.attention(*(x[None, r0:r1].astype(np.float64) for x in (xq, xk, xv)), rows=rows)[0]
+            unq = orc.attention(*(x[0, r0:r1][None] for x in (q, k, v)), rows=rows)[0]
+            err8.append(orc.rel_fro(o8h[r0:r1][rows], ref))
+            errb.append(orc.rel_fro(obh[r0:r1][rows], refb))
+            err_unq.append(orc.rel_fro(o8h[r0:r1][rows], unq))
+            rows_total += len(rows)
+            if r1 - r0 == max(lens):
+                deq_long = deq
+        parity = {"sequences_sampled": varlen_parity_sequences(lens), "rows_sampled": rows_total,
+                  "fp8_vs_fp64_dequantized": max(err8), "fp8_vs_fp64_unquantized": max(err_unq),
+                  "bf16_vs_fp64": max(errb), "prepass_codes_bit_exact": bool(codes_equal),
+                  "tolerances": {"bf16": 5e-3, "fp8": 3e-2}}
+        bad = [k2 for k2, tol in (("fp8_vs_fp64_dequantized", 3e-2), ("bf16_vs_fp64", 5e-3))
+               if not parity[k2] <= tol] + ([] if codes_equal else ["prepass_codes_bit_exact"])
+        if bad:
+            print(f"bench: parity failed ({', '.join(bad)}): {json.dumps(parity)}", file=sys.stderr)
+            return 1
+        S_long = max(lens)
+        rows_long = sample_rows(S_long, 48)
+        t0 = time.perf_counter()
+        orc.attention(*deq_long, rows=rows_long)
+        dt_long = time.perf_counter() - t0
+        cpu_val, cpu_rows, cpu_dt = time_oracle_baseline(deq_long, S_long, rows_long, dt_long, Hq, Dqk, Dv, 1)
+        cpu = {"value": cpu_val, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+               "sample": f"{cpu_rows} query rows x {Hq} heads of the longest sequence ({S_long} rows) of "
+                         f"{args.workload}: fp64 causal attention on the dequantized e4m3 inputs, {cpu_dt:.1f} s"}
+
+    line = {
+        "metric": METRIC_VARLEN, "value": world * flops / (ms8 * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms8,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "nseq": nseq, "tokens": T, "lens": lens, "Hq": Hq, "Hkv": Hkv,
+                   "Dqk": Dqk, "Dv": Dv, "inputs": wl["kind"] + ", seeded, bf16 in HBM, packed [T, H, D]",
+                   "lengths": f"{wl['nseq']} log-uniform in [{wl['lo']}, {wl['hi']}]",
+                   "step": "quantize Q,K,V per (sequence, head) + FP8 Lean-P causal attention, packed batch",
+                   "l2": "flushed before every timed step (256 MiB write, untimed)",
+                   "parallelism": f"dp{world} (independent shards, no collective)"},
+        "roofline": {"bound": "tensor", "achieved": ach8, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": ach8 / fp8_peak, "traffic": None,
+                     "kernel": f"attn_fwd_kernel<FP8,{Dqk},varlen>",
+                     "peak_source": f"{peak_src} bf16 sustained {bf16_sus} x nominal FP8/BF16 ratio 2"},
+        "bf16": {"value": world * flops / (msb * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": msb,
+                 "roofline": {"bound": "tensor", "achieved": achb, "peak": bf16_sus, "unit": "TFLOP/s",
+                              "frac": achb / bf16_sus, "kernel": f"attn_fwd_kernel<BF16,{Dqk},varlen>"}},
+        "fp8_breakdown_ms": {"prepass": ms8_pre, "attention": ms8_attn},
+        "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
+                "d2h_bytes_per_step": host_o.numel() * host_o.element_size(), "ms_per_step": ms_e2e,
+                "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize_qkv_varlen -> zyfa_attn_fwd_varlen -> D2H O"},
+        "gpu_launches": args.steps * (4 + 1 + 1),
         "clocks": clk,
         "parity": parity,
         "cpu_baseline": cpu,

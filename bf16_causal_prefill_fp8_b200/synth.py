@@ -117,6 +117,19 @@ for _s in (1024, 2048, 4096, 8192, 16384, 32768, 65536):
                                              Dv=128, kind="gaussian")
 
 
+# Packed (variable-length) batches: the pages measure fixed lengths only, so
+# this mix is a stand-in for serving traffic: n lengths drawn log-uniform in
+# [lo, hi] (stream 9), packed in draw order.
+VARLEN_WORKLOADS = {
+    "varlen_gqa32x8_mix32": dict(Hq=32, Hkv=8, Dqk=128, Dv=128, kind="outlier_k", nseq=32, lo=512, hi=16384),
+}
+
+
+def varlen_lengths(seed: int, n: int, lo: int, hi: int) -> list:
+    u = uniform64(seed, 9, 0, n)
+    return [int(round(lo * (hi / lo) ** float(x))) for x in u]
+
+
 def causal_flops(B: int, S: int, Hq: int, Dqk: int, Dv: int) -> float:
     """FLOP count of causal attention, FlashAttention convention 2*B*Hq*(S^2/2)*(Dqk+Dv)."""
     return 2.0 * B * Hq * (S * S / 2.0) * (Dqk + Dv)

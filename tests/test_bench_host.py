@@ -62,3 +62,30 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"] == "tiny_s512"
+
+
+def test_varlen_workload_recipe():
+    wl = bench.varlen_workload("varlen_gqa32x8_mix32", 0)
+    lens = wl["lens"]
+    assert len(lens) == wl["nseq"] == 32
+    assert all(wl["lo"] <= n <= wl["hi"] for n in lens)
+    assert wl["cu"][0] == 0 and wl["cu"][-1] == sum(lens)
+    assert all(b - a == n for a, b, n in zip(wl["cu"], wl["cu"][1:], lens))
+    assert wl["S"] == max(lens) and wl["B"] == 1
+    assert bench.varlen_workload("varlen_gqa32x8_mix32", 0)["lens"] == lens      # seeded
+    assert bench.varlen_workload("varlen_gqa32x8_mix32", 1)["lens"] != lens
+    # FLOPs are the per-sequence causal counts summed
+    assert bench.varlen_flops([512, 1000], 32, 128, 128) == (synth.causal_flops(1, 512, 32, 128, 128)
+                                                              + synth.causal_flops(1, 1000, 32, 128, 128))
+    picked = bench.varlen_parity_sequences([5, 0, 900, 3, 40])
+    assert picked == [2, 3, 4] or picked == sorted({2, 3, 4})
+
+
+def test_reference_arm_on_packed_workload():
+    env = dict(os.environ, OMP_NUM_THREADS=os.environ.get("OMP_NUM_THREADS", "4"))
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "varlen_gqa32x8_mix32", "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                         env=env, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC_VARLEN and line["value"] > 0
