@@ -1,0 +1,59 @@
+"""The pages' workloads at full size, in the launch configuration bench.py
+times (fused Q/K/V prepass, then the FP8 attention; the BF16 attention on the
+same bf16 inputs), checked on sampled query rows the oracle computes one by
+one: the first and last rows, rows at 128-row tile edges and seeded random
+rows, for every head.  The prepass codes and scales are compared in full."""
+import numpy as np
+import pytest
+import torch
+
+from bf16_causal_prefill_fp8_b200 import synth, zyfa
+from oracle import oracle as orc
+
+from helpers import TOL_BF16, TOL_FP8
+
+pytestmark = pytest.mark.gpu
+
+WORKLOADS = [  # name, B, S, Hq, Hkv, Dqk, Dv, kind, hadamard
+    ("gqa32x8_s16k_outlier", 1, 16384, 32, 8, 128, 128, "outlier_k", False),
+    ("mha32_s32k", 1, 32768, 32, 32, 128, 128, "gaussian", False),
+    ("mla16_s16k_192_128", 1, 16384, 16, 16, 192, 128, "mla", False),
+    ("sweep_s64k_hadamard", 1, 65536, 32, 32, 128, 128, "gaussian", True),
+]
+
+
+def sampled_rows(S, n, seed):
+    edges = [0, 1, 127, 128, S // 2 - 1, S // 2, S - 129, S - 128, S - 1]
+    rng = np.random.default_rng(seed)
+    extra = rng.choice(S, size=n - len(edges), replace=False)
+    return np.unique(np.concatenate([edges, extra])).astype(np.int32)
+
+
+@pytest.mark.parametrize("wl", WORKLOADS, ids=lambda w: w[0])
+def test_full_size_sampled_parity(wl):
+    name, B, S, Hq, Hkv, Dqk, Dv, kind, hadamard = wl
+    tb = [torch.from_numpy(x).to(torch.bfloat16) for x in synth.make_qkv(0, B, S, Hq, Hkv, Dqk, Dv, kind)]
+    dq, dk, dv = (t.cuda() for t in tb)
+    (cq, sq), (ck, sk), (cv, sv) = zyfa.quantize_qkv(dq, dk, dv, hadamard_qk=hadamard)
+    o8 = zyfa.attn_fwd(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv)
+    ob = zyfa.attn_fwd(dq, dk, dv)
+    torch.cuda.synchronize()
+    assert zyfa.device_status() == zyfa.OK
+    del dq, dk, dv
+    xs = [t.float().numpy() for t in tb]
+    codes = [orc.quantize(xs[0], hadamard), orc.quantize(xs[1], hadamard), orc.quantize(xs[2], False)]
+    for (gc, gs), (rc, rs) in zip(((cq, sq), (ck, sk), (cv, sv)), codes):
+        assert np.array_equal(gs.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+        assert np.array_equal(gc.cpu().numpy(), rc)
+    rows = sampled_rows(S, 16, 3)
+    deq = [orc.dequantize(c, s) for c, s in codes]
+    ref8 = orc.attention(*deq, rows=rows)
+    del deq
+    got8 = o8.float().cpu().numpy()[:, rows].astype(np.float64)
+    err8 = orc.rel_fro(got8, ref8)
+    refb = orc.attention(*[x.astype(np.float64) for x in xs], rows=rows)
+    gotb = ob.float().cpu().numpy()[:, rows].astype(np.float64)
+    errb = orc.rel_fro(gotb, refb)
+    print(f"{name}: fp8 vs fp64 (dequantized) {err8:.3e}; bf16 {errb:.3e}")
+    assert err8 <= TOL_FP8, err8
+    assert errb <= TOL_BF16, errb
