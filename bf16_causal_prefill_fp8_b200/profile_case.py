@@ -4,7 +4,8 @@
 
 Each iteration launches, in order: zyfa_quantize_qkv (zero, amax, codes and
 finalize kernels over Q, K and V together), the FP8 attention kernel, then the
-BF16 attention kernel on the same bf16 inputs.  Prints nothing but a completion line; timing
+BF16 attention kernel on the same bf16 inputs (for a packed-batch workload,
+the varlen forms of the same three calls).  Prints nothing but a completion line; timing
 numbers come from bench.py, never from a profiled run.
 """
 import argparse
@@ -16,20 +17,35 @@ from . import synth, zyfa
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--workload", default="gqa32x8_s16k_outlier", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="gqa32x8_s16k_outlier",
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.VARLEN_WORKLOADS))
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--hadamard", action="store_true")
     ap.add_argument("--only", choices=["all", "fp8", "bf16"], default="all")
     args = ap.parse_args()
-    wl = synth.WORKLOADS[args.workload]
-    q, k, v = synth.make_qkv(0, wl["B"], wl["S"], wl["Hq"], wl["Hkv"], wl["Dqk"], wl["Dv"], wl["kind"])
-    dq, dk, dv = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (q, k, v))
+    if args.workload in synth.VARLEN_WORKLOADS:
+        # packed batch: the varlen prepass and varlen attention launches
+        wl = synth.VARLEN_WORKLOADS[args.workload]
+        lens = synth.varlen_lengths(0, wl["nseq"], wl["lo"], wl["hi"])
+        cu = [0]
+        for n in lens:
+            cu.append(cu[-1] + n)
+        q, k, v = synth.make_qkv(0, 1, cu[-1], wl["Hq"], wl["Hkv"], wl["Dqk"], wl["Dv"], wl["kind"])
+        dq, dk, dv = (torch.from_numpy(x[0]).to(torch.bfloat16).cuda() for x in (q, k, v))
+        quant = lambda: zyfa.quantize_qkv_varlen(dq, dk, dv, cu, hadamard_qk=args.hadamard)
+        attn = lambda *t, **kw: zyfa.attn_fwd_varlen(*t, cu, **kw)
+    else:
+        wl = synth.WORKLOADS[args.workload]
+        q, k, v = synth.make_qkv(0, wl["B"], wl["S"], wl["Hq"], wl["Hkv"], wl["Dqk"], wl["Dv"], wl["kind"])
+        dq, dk, dv = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (q, k, v))
+        quant = lambda: zyfa.quantize_qkv(dq, dk, dv, hadamard_qk=args.hadamard)
+        attn = zyfa.attn_fwd
     for _ in range(args.iters):
         if args.only in ("all", "fp8"):
-            (cq, sq), (ck, sk), (cv, sv) = zyfa.quantize_qkv(dq, dk, dv, hadamard_qk=args.hadamard)
-            zyfa.attn_fwd(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv)
+            (cq, sq), (ck, sk), (cv, sv) = quant()
+            attn(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv)
         if args.only in ("all", "bf16"):
-            zyfa.attn_fwd(dq, dk, dv)
+            attn(dq, dk, dv)
     torch.cuda.synchronize()
     st = zyfa.device_status()
     print(f"profile_case {args.workload}: {args.iters} iterations done, device status {st}")
