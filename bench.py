@@ -112,6 +112,19 @@ def row_flops(rows, Hq, Dqk, Dv, B):
     return float(B * Hq * sum(2.0 * (int(i) + 1) * (Dqk + Dv) for i in rows))
 
 
+def max_head_rel_fro(got, ref):
+    """Largest per-head relative Frobenius error; arrays [..., H, D] with the
+    head axis second to last."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    H = ref.shape[-2]
+    errs = []
+    for h in range(H):
+        g, r = got[..., h, :], ref[..., h, :]
+        errs.append(float(np.linalg.norm((g - r).ravel()) / np.linalg.norm(r.ravel())))
+    return max(errs)
+
+
 def oracle_inputs(wl, seed, xq, xk, xv, hadamard=False):
     """The oracle's own quantization of the bf16 inputs (widened to fp32)."""
     from oracle import oracle as orc
@@ -425,7 +438,10 @@ def run_ours(args, wl):
         unq = orc.attention(q, k, v, rows=rows)
         parity = {"rows_sampled": int(len(rows)), "fp8_vs_fp64_dequantized": orc.rel_fro(o_gpu, o_ref),
                   "fp8_vs_fp64_unquantized": orc.rel_fro(o_gpu, unq),
-                  "bf16_vs_fp64": orc.rel_fro(ob_gpu, ob_ref), "prepass_codes_bit_exact": bool(gpu_codes_equal),
+                  "bf16_vs_fp64": orc.rel_fro(ob_gpu, ob_ref),
+                  "fp8_vs_fp64_dequantized_worst_head": max_head_rel_fro(o_gpu, o_ref),
+                  "bf16_vs_fp64_worst_head": max_head_rel_fro(ob_gpu, ob_ref),
+                  "prepass_codes_bit_exact": bool(gpu_codes_equal),
                   "tolerances": {"bf16": 5e-3, "fp8": 3e-2}}
         if abl_ms is not None:
             ox = o8x.float().cpu().numpy()[:, rows].astype(np.float64)

@@ -89,3 +89,13 @@ def test_reference_arm_on_packed_workload():
     assert out.returncode == 0, out.stderr[-2000:]
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC_VARLEN and line["value"] > 0
+
+
+def test_max_head_rel_fro():
+    rng = np.random.default_rng(0)
+    ref = rng.normal(size=(1, 5, 3, 8))
+    got = ref.copy()
+    got[:, :, 1, :] *= 1.01                      # head 1 off by 1 %
+    assert abs(bench.max_head_rel_fro(got, ref) - 0.01) < 1e-12
+    assert bench.max_head_rel_fro(ref, ref) == 0.0
+    assert bench.max_head_rel_fro(got, ref) >= orc.rel_fro(got, ref)
