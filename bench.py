@@ -112,6 +112,48 @@ def row_flops(rows, Hq, Dqk, Dv, B):
     return float(B * Hq * sum(2.0 * (int(i) + 1) * (Dqk + Dv) for i in rows))
 
 
+def e2e_pipelined(torch, pin, bufs, run_step, outs, host_outs, steps):
+    """End-to-end steps with copies overlapped: step i's H2D (copy stream)
+    runs beside step i-1's compute (current stream) and step i-2's D2H (D2H
+    stream); every step still copies its inputs in and its output out.  Buffer
+    set i % 2 is rewritten only after step i-2's compute has read it, and
+    output i % 2 only after step i-2's D2H has read it.  Returns ms per step:
+    events on the current stream around the loop, which waits for the other
+    streams' last copies."""
+    main = torch.cuda.current_stream()
+    cp, dh = torch.cuda.Stream(), torch.cuda.Stream()
+    h2d = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    d2h = [torch.cuda.Event() for _ in range(2)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(main)
+    cp.wait_event(e0)
+    dh.wait_event(e0)
+    for i in range(steps):
+        s = i % 2
+        if i >= 2:
+            cp.wait_event(done[s])
+        with torch.cuda.stream(cp):
+            for dst, src in zip(bufs[s], pin):
+                dst.copy_(src, non_blocking=True)
+        h2d[s].record(cp)
+        main.wait_event(h2d[s])
+        if i >= 2:
+            main.wait_event(d2h[s])
+        run_step(s)
+        done[s].record(main)
+        dh.wait_event(done[s])
+        with torch.cuda.stream(dh):
+            host_outs[s].copy_(outs[s], non_blocking=True)
+        d2h[s].record(dh)
+    for s in range(min(steps, 2)):
+        main.wait_event(d2h[s])
+    e1.record(main)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def max_head_rel_fro(got, ref):
     """Largest per-head relative Frobenius error; arrays [..., H, D] with the
     head axis second to last."""
@@ -403,9 +445,36 @@ def run_ours(args, wl):
         host_o.copy_(o8, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    ms_e2e_serial = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
     h2d = sum(t.numel() * t.element_size() for t in pin)
     d2h = host_o.numel() * host_o.element_size()
+
+    # e2e pipelined: the same steps, each step's copies overlapping its
+    # neighbours' compute (two buffer sets); the last output must equal the
+    # resident-input output bit for bit, else the serial figure stands
+    ref_o = o8.cpu()
+    ms_pipe, pipe_note = float("inf"), None
+    try:
+        bufs = [(dq, dk, dv), tuple(torch.empty_like(t) for t in (dq, dk, dv))]
+        outs = [torch.empty_like(o8), torch.empty_like(o8)]
+        host_outs = [host_o, torch.empty(o8.shape, dtype=torch.bfloat16).pin_memory()]
+
+        def step_on(sidx):
+            xq, xk, xv = bufs[sidx]
+            zyfa.quantize_qkv(xq, xk, xv, hadamard_qk=args.hadamard, out=((cq, sq), (ck, sk), (cv, sv)))
+            zyfa.attn_fwd(cq, ck, cv, o=outs[sidx], q_scale=sq, k_scale=sk, v_scale=sv)
+
+        barrier()
+        ms_try = e2e_pipelined(torch, pin, bufs, step_on, outs, host_outs, e2e_steps)
+        if torch.equal(host_outs[(e2e_steps - 1) % 2], ref_o):
+            ms_pipe = ms_try
+        else:
+            pipe_note = "pipelined output differs from the resident-input output"
+    except Exception as exc:   # the serial figure stands; say why
+        pipe_note = f"pipelined e2e failed: {exc!r}"[:200]
+        torch.cuda.synchronize()
+    ms_pipe = max_over_ranks(ms_pipe)
+    ms_e2e = ms_pipe if ms_pipe != float("inf") else ms_e2e_serial
 
     if rank != 0:
         if world > 1:
@@ -492,7 +561,11 @@ def run_ours(args, wl):
                                 "instead of Lean P; errors under parity.exact_p_*"}},
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-                "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize_qkv -> zyfa_attn_fwd -> D2H O"},
+                "serial_ms_per_step": ms_e2e_serial,
+                "pipelined": ms_pipe != float("inf"), "note": pipe_note,
+                "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize_qkv -> zyfa_attn_fwd -> D2H O; "
+                        "pipelined: step i's H2D and step i-1's D2H overlap step i's neighbours' compute "
+                        "(copy and D2H streams, two buffer sets)"},
         "gpu_launches": args.steps * (launches_per_fp8_step + 1),
         "clocks": clk,
         "parity": parity,

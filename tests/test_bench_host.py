@@ -99,3 +99,163 @@ def test_max_head_rel_fro():
     assert abs(bench.max_head_rel_fro(got, ref) - 0.01) < 1e-12
     assert bench.max_head_rel_fro(ref, ref) == 0.0
     assert bench.max_head_rel_fro(got, ref) >= orc.rel_fro(got, ref)
+
+
+class _FakeCuda:
+    """Streams, events and copies as queues of operations, run in a random
+    order that respects stream order and event waits, with every buffer
+    tagged by the step whose data it holds: checks bench.e2e_pipelined's
+    hazards without a GPU."""
+
+    def __init__(self, rng):
+        self.rng = rng
+        self.streams = []
+        self.cur = self.Stream()
+        self.log = []
+
+    # --- the torch.cuda surface e2e_pipelined uses
+    def Stream(self):
+        s = _FakeStream(self)
+        self.streams.append(s)
+        return s
+
+    def Event(self, enable_timing=False):
+        return _FakeEvent()
+
+    def current_stream(self):
+        return self.cur
+
+    def stream(self, s):
+        fake = self
+
+        class _Ctx:
+            def __enter__(self_):
+                self_.prev = fake.cur
+                fake.cur = s
+
+            def __exit__(self_, *a):
+                fake.cur = self_.prev
+        return _Ctx()
+
+    def synchronize(self):
+        while any(s.q for s in self.streams):
+            ready = [s for s in self.streams if s.q and s.ready()]
+            assert ready, "deadlock: every stream waits"
+            self.rng.choice(ready).step()
+
+
+class _FakeEvent:
+    def __init__(self):
+        self.target = None          # (stream, op index) of the latest record
+
+    def record(self, stream):
+        self.target = stream.enqueue(("record",))
+
+    def elapsed_time(self, other):
+        return 1.0
+
+
+class _FakeStream:
+    def __init__(self, cuda):
+        self.cuda, self.q, self.done = cuda, [], 0
+
+    def enqueue(self, op):
+        self.q.append(op)
+        return (self, self.done + len(self.q) - 1)
+
+    def wait_event(self, ev):
+        if ev.target is not None:
+            self.enqueue(("wait", ev.target))
+
+    def ready(self):
+        op = self.q[0]
+        if op[0] != "wait":
+            return True
+        st, idx = op[1]
+        return st.done > idx
+
+    def step(self):
+        op = self.q.pop(0)
+        self.done += 1
+        if op[0] == "run":
+            op[1]()
+
+
+class _FakeTensor:
+    def __init__(self, cuda, name):
+        self.cuda, self.name, self.tag, self.writes = cuda, name, None, 0
+
+    def copy_(self, src, non_blocking=False):
+        step_of_src = src.tag if isinstance(src, _FakeTensor) and src.name.startswith("out") else None
+        dst = self
+
+        def run():
+            if step_of_src is not None:                    # D2H: the output must hold the step it is read for
+                assert src.tag == step_of_src_expected[0], (src.name, src.tag)
+            dst.tag = src.tag
+        step_of_src_expected = [None]
+        self.cuda.cur.enqueue(("run", run))
+        return step_of_src_expected
+
+
+def test_e2e_pipeline_has_no_buffer_hazards():
+    import random
+    for seed in range(200):
+        rng = random.Random(seed)
+        cuda = _FakeCuda(rng)
+        fake_torch = type("T", (), {"cuda": cuda})
+        steps = rng.randint(1, 7)
+        pin = [_FakeTensor(cuda, f"pin{j}") for j in range(3)]
+        bufs = [tuple(_FakeTensor(cuda, f"buf{s}{j}") for j in range(3)) for s in range(2)]
+        outs = [_FakeTensor(cuda, f"out{s}") for s in range(2)]
+        host = [_FakeTensor(cuda, f"host{s}") for s in range(2)]
+        counter = {"h2d": [0, 0], "run": [0, 0], "d2h": [0, 0]}
+        got = []
+
+        for t in pin:
+            t.tag = "input"
+
+        # tag every H2D copy with its step: H2D of buffer set s happens for steps s, s + 2, ...
+        orig_copy = _FakeTensor.copy_
+
+        def copy_(self, src, non_blocking=False):
+            if self.name.startswith("buf"):
+                s = int(self.name[3])
+                step = s + 2 * (counter["h2d"][s] // 3)
+                counter["h2d"][s] += 1
+                dst = self
+
+                def run():
+                    dst.tag = step
+                cuda.cur.enqueue(("run", run))
+            elif self.name.startswith("host"):
+                s = int(self.name[4])
+                step = s + 2 * counter["d2h"][s]
+                counter["d2h"][s] += 1
+                dst = self
+
+                def run():
+                    assert src.tag == step, f"D2H of step {step} read output of step {src.tag}"
+                    dst.tag = step
+                    got.append(step)
+                cuda.cur.enqueue(("run", run))
+            else:
+                orig_copy(self, src, non_blocking)
+
+        def run_step(s):
+            step = s + 2 * counter["run"][s]
+            counter["run"][s] += 1
+
+            def run():
+                for b in bufs[s]:
+                    assert b.tag == step, f"compute of step {step} read {b.name} holding step {b.tag}"
+                outs[s].tag = step
+            cuda.cur.enqueue(("run", run))
+
+        _FakeTensor.copy_ = copy_
+        try:
+            bench.e2e_pipelined(fake_torch, pin, bufs, run_step, outs, host, steps)
+        finally:
+            _FakeTensor.copy_ = orig_copy
+        assert sorted(got) == list(range(steps))
+        assert not any(s.q for s in cuda.streams)
