@@ -172,3 +172,26 @@ def test_quantize_varlen_argument_errors(L):
     assert e3(Dqk=64) == -3
     assert e3(Dv=12) == -3
     assert e3(had=3) == -6
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch):
+    """No fallback: with the shared library absent, the first call raises."""
+    monkeypatch.setattr(zyfa, "LIB_PATH", zyfa.LIB_PATH + ".absent")
+    monkeypatch.setattr(zyfa, "_lib", None)
+    with pytest.raises(ImportError):
+        zyfa.lib()
+    with pytest.raises(ImportError):
+        zyfa.status_string(0)
+
+
+def test_product_package_never_touches_the_oracle():
+    """The oracle is test infrastructure: nothing in the package imports it."""
+    import os
+    import re
+    pkg = os.path.dirname(zyfa.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
+                assert "oracle.c" not in text and "liboracle" not in text, f
