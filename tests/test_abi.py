@@ -195,3 +195,21 @@ def test_product_package_never_touches_the_oracle():
                 text = open(os.path.join(root, f), encoding="utf-8").read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
                 assert "oracle.c" not in text and "liboracle" not in text, f
+
+
+def test_oracle_uses_nothing_from_the_package():
+    """The other direction: the oracle includes only the C library and imports
+    neither the package nor its headers."""
+    import os
+    import re
+    here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    odir = os.path.join(here, "oracle")
+    for f in os.listdir(odir):
+        path = os.path.join(odir, f)
+        if f.endswith(".c"):
+            incs = re.findall(r'^\s*#\s*include\s*[<"]([^>"]+)[>"]', open(path).read(), flags=re.M)
+            assert set(incs) <= {"math.h", "stdint.h", "stdlib.h", "string.h", "omp.h"}, (f, incs)
+        elif f.endswith(".py"):
+            imports = re.findall(r"^\s*(?:import|from)\s+([\w.]+)", open(path).read(), flags=re.M)
+            assert not any(m.startswith("bf16_causal_prefill_fp8_b200") for m in imports), (f, imports)
+            assert "libzyfa" not in open(path).read(), f
