@@ -52,7 +52,9 @@ def test_varlen_covers_every_unit_once(grid, lens, Hq, Hkv, Dqk, dt):
 
 @pytest.mark.parametrize("grid", [1, 7, 148])
 @pytest.mark.parametrize("B,S,Hq,Hkv,Dqk,dt", [(2, 1000, 4, 2, 128, FP8), (3, 777, 6, 3, 192, BF16),
-                                               (1, 16384, 32, 8, 128, FP8)])
+                                               (1, 16384, 32, 8, 128, FP8),
+                                               (1, 32768, 32, 32, 128, FP8),     # 6 L2 groups of 6 slots
+                                               (4, 16384, 16, 16, 192, BF16)])   # 64 slots, 4 per group
 def test_fixed_covers_every_unit_once_and_equals_varlen(grid, B, S, Hq, Hkv, Dqk, dt):
     fixed = all_units(grid, Hq=Hq, Hkv=Hkv, Dqk=Dqk, dtype=dt, B=B, S=S)
     assert sorted(u for cta in fixed for u in cta) == expected_units([S] * B, Hq)
@@ -117,3 +119,12 @@ def test_schedule_argument_errors():
     with pytest.raises(zyfa.ZyfaError):
         zyfa.attn_schedule(Hq=2, Hkv=2, Dqk=128, dtype=FP8, grid=4, cta=0, cu_seqlens=[0, 5, 3])
     assert zyfa.attn_schedule(Hq=2, Hkv=2, Dqk=128, dtype=FP8, grid=4, cta=0, cu_seqlens=[0, 0]) == []
+
+
+def test_multi_group_fixed_schedule_keeps_groups_contiguous():
+    """MHA 32K FP8: 8 MiB of K/V per kv head, so groups of 6 heads (48 MiB);
+    with one CTA the issue order walks the groups in slot order."""
+    order = zyfa.attn_schedule(Hq=32, Hkv=32, Dqk=128, dtype=FP8, grid=1, cta=0, B=1, S=32768)
+    groups = [hq // 6 for _, hq, _ in order]
+    assert groups == sorted(groups)
+    assert len(set(groups)) == 6
