@@ -399,22 +399,33 @@ __global__ void __launch_bounds__(kQuantThreads) quant3_codes_kernel(const __gri
 
 // Variable-length batch: tensors packed [T, H, D], sequence s at rows
 // cu[s] .. cu[s+1]-1 with its own scale per head ([nseq, H] per tensor).
-// Grid = (sum of chunk columns, nseq): CTA (x, s) runs the fixed-length step
-// on sequence s alone (base and scale pointers moved to it, S = its length);
-// chunks past the sequence's end have no rows and return at once.
+// Tensor i's CTAs (grid columns first[i] .. first[i+1]-1) enumerate the
+// chunks of every sequence in order, ceil(len / rows_per_cta) per sequence,
+// so no CTA is idle; each runs the fixed-length step on its sequence alone
+// (base and scale pointers moved to it, S = its length).
 constexpr int kMaxQuantSeqs = 384;
 struct Quant3VarArgs {
   Quant3Args q;                  // t[i].S unused; rows_per_cta per tensor
+  int n;                         // sequences
   int cu[kMaxQuantSeqs + 1];
 };
+static_assert(sizeof(Quant3VarArgs) <= 4096, "kernel parameter space");
 
 template <typename T>
 __device__ __forceinline__ bool quant3v_select(const Quant3VarArgs& a, QuantArgs& t, int& i, int& chunk) {
   i = quant3_pick(a.q, blockIdx.x);
-  chunk = blockIdx.x - a.q.first[i];
-  const int s = blockIdx.y, r0 = a.cu[s], len = a.cu[s + 1] - r0;
   t = a.q.t[i];
-  if (static_cast<long long>(chunk) * t.rows_per_cta >= len) return false;
+  // the sequence this chunk belongs to: a scan over the sequences' chunk
+  // counts (every thread takes the same path)
+  int c = blockIdx.x - a.q.first[i], s = 0;
+  for (; s < a.n; ++s) {
+    const int nch = (a.cu[s + 1] - a.cu[s] + t.rows_per_cta - 1) / t.rows_per_cta;
+    if (c < nch) break;
+    c -= nch;
+  }
+  if (s >= a.n) return false;   // past the last chunk (the host sizes the grid exactly)
+  chunk = c;
+  const int r0 = a.cu[s], len = a.cu[s + 1] - r0;
   const size_t off = static_cast<size_t>(r0) * t.H * t.D;
   t.x = static_cast<const T*>(t.x) + off;
   t.out += off;

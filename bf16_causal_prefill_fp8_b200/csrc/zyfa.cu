@@ -482,8 +482,6 @@ static int quantize_varlen_n(int n, const void* const* xs, void* const* outs, fl
   if (cudaGetDevice(&dev) != cudaSuccess) return ZYFA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ZYFA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int max_len = 0;
-  for (int i = 0; i < nseq; ++i) max_len = std::max(max_len, cu[i + 1] - cu[i]);
   const int T = cu[nseq];
   // CTAs per average sequence as in the fixed-length prepass, split among
   // the tensors in proportion to their bytes; a longer sequence gets
@@ -519,9 +517,13 @@ static int quantize_varlen_n(int n, const void* const* xs, void* const* outs, fl
     t.H = Hs[i]; t.D = Ds[i];
     t.rows_per_cta = static_cast<int>((mean_len + chunks - 1) / chunks);
     q3.had[i] = had[i];
-    q3.first[i + 1] = q3.first[i] + (max_len + t.rows_per_cta - 1) / t.rows_per_cta;
+    long long cols = 0;   // every sequence's chunks, in order
+    for (int sq = 0; sq < nseq; ++sq) cols += (cu[sq + 1] - cu[sq] + t.rows_per_cta - 1) / t.rows_per_cta;
+    if (q3.first[i] + cols > 0x7fffffffll) return ZYFA_ERR_BAD_SHAPE;
+    q3.first[i + 1] = q3.first[i] + static_cast<int>(cols);
     max_h = std::max(max_h, Hs[i]);
   }
+  a.n = nseq;
   for (int i = 0; i <= nseq; ++i) a.cu[i] = cu[i];
   const int n0 = nseq * Hs[0], n1 = n > 1 ? nseq * Hs[1] : 0, n2 = n > 2 ? nseq * Hs[2] : 0;
   const int nn = n0 + n1 + n2;
@@ -529,7 +531,7 @@ static int quantize_varlen_n(int n, const void* const* xs, void* const* outs, fl
   float* s2 = n > 2 ? scs[2] : scs[0];
   quant3_zero_kernel<<<(nn + 255) / 256, 256, 0, st>>>(scs[0], s1, s2, n0, n1, n2);
   if (q3.first[3] > 0) {   // some sequence has rows
-    const dim3 grid(static_cast<unsigned>(q3.first[3]), static_cast<unsigned>(nseq));
+    const dim3 grid(static_cast<unsigned>(q3.first[3]), 1u);
     const size_t shm = static_cast<size_t>(max_h) * 8;   // amax, or scale and its reciprocal, per head
     if (in_dtype == ZYFA_BF16) {
       quant3v_amax_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
