@@ -459,6 +459,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (Cf::TAIL) tma_load_4d(dst + Cf::NCH * Cf::CHUNK, mt, br, 128, h, row, bb, pol);
     };
     auto load_k = [&](const TS& t) -> bool {
+      // checked builds: the unit's indices and its tile's first row
+      range_ok(t.b >= 0 && t.b < a.B && t.hq >= 0 && t.hq < a.Hq && t.hkv >= 0 && t.hkv < a.Hkv && t.j >= 0 &&
+                   t.j <= t.qt, kChkUnit);
+      range_ok(VARLEN ? (t.qt * 128 < t.len && t.r0 >= 0 && t.r0 + t.len <= a.S) : (t.qt * 128 < a.S), kChkRow);
       // tensor-map row and batch coordinates of the unit's sequence
       const int row0 = VARLEN ? t.r0 : 0, tb = VARLEN ? 0 : t.b;
       if (t.j == 0) {                      // first tile of a unit: its Q tile first
@@ -631,8 +635,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l = 0.0f;
         m_own = __int_as_float(0xff800000);
         if (FP8) {
-          const float qs = a.q_scale ? a.q_scale[t.b * a.Hq + t.hq] : 1.0f;
-          const float ks = a.k_scale ? a.k_scale[t.b * a.Hkv + t.hkv] : 1.0f;
+          const bool sok = range_ok(t.b >= 0 && t.b < a.B && t.hq >= 0 && t.hq < a.Hq && t.hkv >= 0 &&
+                                    t.hkv < a.Hkv, kChkScale);
+          const float qs = (a.q_scale && sok) ? a.q_scale[t.b * a.Hq + t.hq] : 1.0f;
+          const float ks = (a.k_scale && sok) ? a.k_scale[t.b * a.Hkv + t.hkv] : 1.0f;
           A = leanp_slope(qs, ks, a.C);
         }
       }
@@ -823,13 +829,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float inv, lse_log2;   // lse_log2: log-sum-exp of the scaled scores, in binades
       const int grow = qt * 128 + row;
       if (FP8) {
-        const float vsc = a.v_scale ? a.v_scale[b * a.Hkv + hkv] : 1.0f;
+        const bool sok = range_ok(b >= 0 && b < a.B && hq >= 0 && hq < a.Hq && hkv >= 0 && hkv < a.Hkv,
+                                  kChkScale);
+        const float vsc = (a.v_scale && sok) ? a.v_scale[b * a.Hkv + hkv] : 1.0f;
         const float lv = __uint_as_float(tmem_ld1(lb + Cf::TL));
         tmem_wait_ld();
         inv = vsc / lv;
         if (a.lse) {   // weights are 2^((s - m) A / 8) against the final reference m
-          const float qs = a.q_scale ? a.q_scale[b * a.Hq + hq] : 1.0f;
-          const float ks = a.k_scale ? a.k_scale[b * a.Hkv + hkv] : 1.0f;
+          const float qs = (a.q_scale && sok) ? a.q_scale[b * a.Hq + hq] : 1.0f;
+          const float ks = (a.k_scale && sok) ? a.k_scale[b * a.Hkv + hkv] : 1.0f;
           const float A8 = __fmul_rn(leanp_slope(qs, ks, a.C), 0.125f);
           lse_log2 = __fmaf_rn(lfin_s[(u_it & 3) * 128 + row], A8, log2f(lv));
         }
@@ -845,13 +853,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // output row: (b, grow) of [B, S, Hq, 128], or packed row r0 + grow of
       // [T, Hq, 128]; lse [B, Hq, S] or [Hq, T]
+      // checked builds: a row that is stored must lie inside the tensor
+      const bool wok = range_ok(grow >= (VARLEN ? len : a.S) ||
+                                    (hq >= 0 && hq < a.Hq &&
+                                     (VARLEN ? (r0 >= 0 && r0 + grow < a.S) : (b >= 0 && b < a.B))),
+                                kChkStore);
       __nv_bfloat16* orow;
       if constexpr (VARLEN) {
-        if (a.lse && grow < len)
+        if (a.lse && grow < len && wok)
           a.lse[static_cast<size_t>(hq) * a.S + r0 + grow] = lse_log2 * 0.69314718055994530942f;
         orow = a.o + ((static_cast<size_t>(r0) + grow) * a.Hq + hq) * 128;
       } else {
-        if (a.lse && grow < a.S)
+        if (a.lse && grow < a.S && wok)
           a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.S + grow] = lse_log2 * 0.69314718055994530942f;
         orow = a.o + ((static_cast<size_t>(b) * a.S + grow) * a.Hq + hq) * 128;
       }
@@ -864,7 +877,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (grow < (VARLEN ? len : a.S)) {
+        if (grow < (VARLEN ? len : a.S) && wok) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);

@@ -18,6 +18,30 @@ enum DeviceError : int {
 
 __device__ int g_device_status;
 
+// Checked builds (compiled with ZYFA_CHECKS): range checks on the work-unit
+// indices, the scale reads and the output writes.  The first failing check
+// records its site in g_device_check (read by zyfa_device_check) and the
+// access it guards is skipped.  In normal builds range_ok() is a constant
+// true, the checks compile to nothing and the word stays 0.
+#ifdef ZYFA_CHECKS
+constexpr bool kRangeChecks = true;
+#else
+constexpr bool kRangeChecks = false;
+#endif
+enum CheckSite : int {
+  kChkUnit = 1,     // a scheduled unit's batch / head / tile index out of range
+  kChkRow = 2,      // a tile's first row outside its sequence
+  kChkScale = 3,    // a scale read outside [B*H]
+  kChkStore = 4,    // an output or LSE row outside the tensor
+};
+
+__device__ int g_device_check;
+
+__device__ __forceinline__ bool range_ok(bool ok, int site) {
+  if (kRangeChecks && !ok) atomicCAS(&g_device_check, 0, site);
+  return !kRangeChecks || ok;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

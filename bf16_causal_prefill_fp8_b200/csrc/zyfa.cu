@@ -628,6 +628,16 @@ extern "C" int zyfa_device_status(void* stream) {
   return v == kDevOk ? ZYFA_OK : ZYFA_ERR_DEVICE_TIMEOUT;
 }
 
+extern "C" int zyfa_device_check(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZYFA_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_check, sizeof(int)) != cudaSuccess) return ZYFA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_check, &zero, sizeof(int)) != cudaSuccess) return ZYFA_ERR_CUDA;
+  return v;
+}
+
+extern "C" int zyfa_checked_build(void) { return kRangeChecks ? 1 : 0; }
+
 extern "C" int zyfa_leanp_codes(const float* s, const float* m, const float* bmax, const float* A,
                                 const unsigned char* masked, int n, unsigned char* code, int* j,
                                 void* stream) {

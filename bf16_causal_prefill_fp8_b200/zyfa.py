@@ -12,7 +12,8 @@ import re
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libzyfa.so")
+# ZYFA_CHECKED=1 selects the build with device-side range checks compiled in
+LIB_PATH = os.path.join(HERE, "libzyfa_checked.so" if os.environ.get("ZYFA_CHECKED") == "1" else "libzyfa.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "zyfa.h")
 
 BF16, FP8_E4M3, FP32 = 0, 1, 2
@@ -60,6 +61,10 @@ def lib() -> ctypes.CDLL:
         L.zyfa_device_status.argtypes = [p]
         L.zyfa_set_wait_timeout_ns.restype = None
         L.zyfa_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+        L.zyfa_device_check.restype = i
+        L.zyfa_device_check.argtypes = [p]
+        L.zyfa_checked_build.restype = i
+        L.zyfa_checked_build.argtypes = []
         L.zyfa_leanp_codes.restype = i
         L.zyfa_leanp_codes.argtypes = [p, p, p, p, p, i, p, p, p]
         L.zyfa_selftest_wait_timeout.restype = i
@@ -338,6 +343,15 @@ def leanp_codes(s, m, bmax, A, masked=None, stream=None):
 
 def device_status(stream=None) -> int:
     return lib().zyfa_device_status(_stream(stream))
+
+
+def device_check(stream=None) -> int:
+    """Checked build: site of the first failed range check since the last call (0 = none)."""
+    return lib().zyfa_device_check(_stream(stream))
+
+
+def checked_build() -> bool:
+    return bool(lib().zyfa_checked_build())
 
 
 def set_wait_timeout_ns(ns: int):

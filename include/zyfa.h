@@ -276,6 +276,21 @@ int zyfa_device_status(void* stream);
 void zyfa_set_wait_timeout_ns(unsigned long long ns);
 
 /*
+ * zyfa_device_check -- for a checked build of the library (compiled with
+ * ZYFA_CHECKS, libzyfa_checked.so): synchronises `stream`, then reads and
+ * clears the range-check word of the current device.  Returns 0 if no check
+ * failed since the last call, else the site of the first failure: 1 a
+ * scheduled unit's batch, head or tile index; 2 a tile's first row outside
+ * its sequence; 3 a scale read outside [B*H]; 4 an output or LSE row outside
+ * the tensor (the guarded access was skipped).  ZYFA_ERR_CUDA on a CUDA
+ * error.  A normal build never fails a check (it compiles none) and returns 0.
+ */
+int zyfa_device_check(void* stream);
+
+/* zyfa_checked_build -- 1 for the checked build, 0 for the normal one. */
+int zyfa_checked_build(void);
+
+/*
  * zyfa_leanp_codes -- runs, element-wise, the very __device__ functions the
  * FP8 attention kernel uses to turn scores into Lean-P codes, so that the
  * codes can be compared byte for byte with a CPU emulation.  For element i:

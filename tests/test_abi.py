@@ -213,3 +213,14 @@ def test_oracle_uses_nothing_from_the_package():
             imports = re.findall(r"^\s*(?:import|from)\s+([\w.]+)", open(path).read(), flags=re.M)
             assert not any(m.startswith("bf16_causal_prefill_fp8_b200") for m in imports), (f, imports)
             assert "libzyfa" not in open(path).read(), f
+
+
+def test_checked_build_exports_the_same_symbols():
+    """libzyfa_checked.so (device-side range checks compiled in) has the same
+    C ABI; each library reports which build it is."""
+    Lc = ctypes.CDLL(build.LIB_CHECKED)
+    for n in zyfa.declared_symbols():
+        assert hasattr(Lc, n), n
+    Lc.zyfa_checked_build.restype = ctypes.c_int
+    assert Lc.zyfa_checked_build() == 1
+    assert zyfa.lib().zyfa_checked_build() == 0
