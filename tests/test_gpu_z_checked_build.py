@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from bf16_causal_prefill_fp8_b200 import synth, zyfa
+from bf16_causal_prefill_fp8_b200 import build, synth, zyfa
 
 from helpers import bf16_round
 
@@ -55,6 +55,7 @@ print(json.dumps({"check": zyfa.device_check(), "status": zyfa.device_status()})
 
 
 def test_checked_build_passes_its_checks_and_matches(tmp_path):
+    build.build()   # both libraries (no-op when up to date)
     normal = run_cases()
     assert zyfa.device_check() == 0 and not zyfa.checked_build()
     path = str(tmp_path / "checked.npz")
