@@ -564,8 +564,8 @@ def run_ours(args, wl):
                 "serial_ms_per_step": ms_e2e_serial,
                 "pipelined": ms_pipe != float("inf"), "note": pipe_note,
                 "path": "pinned host bf16 Q,K,V -> H2D -> zyfa_quantize_qkv -> zyfa_attn_fwd -> D2H O; "
-                        "pipelined: step i's H2D and step i-1's D2H overlap step i's neighbours' compute "
-                        "(copy and D2H streams, two buffer sets)"},
+                        "pipelined: each step's H2D overlaps the previous step's compute and its D2H the "
+                        "next step's (copy and D2H streams, two buffer sets)"},
         "gpu_launches": args.steps * (launches_per_fp8_step + 1),
         "clocks": clk,
         "parity": parity,
