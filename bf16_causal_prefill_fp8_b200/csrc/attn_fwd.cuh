@@ -1,7 +1,6 @@
 // attn_fwd.cuh -- causal prefill attention forward, O = softmax(Q K^T * scale
 // + causal mask) V, for sm_100a: persistent causal-aware scheduler, TMA-staged
-// K/V ring, tcgen05 MMAs into tensor memory, warp-specialised softmax and
-// correction.
+// K/V ring, tcgen05 MMAs into tensor memory, warp-specialised softmax.
 //
 // Method: Zyphra ZYFA (news pages: the-ai.news "Zyphra presenteert ZYFA",
 // sections "Waarom presteert FP8 minder goed op de MI355X?" and "Drie
@@ -15,26 +14,28 @@
 //
 // The pages overlap matrix and vector work by instruction order (two waves
 // per SIMD, ping-pong).  Blackwell tracks MMA completion in hardware, so the
-// overlap here is warp specialisation with mbarrier hand-offs.  CTA = 480
-// threads, one per SM (persistent grid):
+// overlap here is warp specialisation with mbarrier hand-offs.  CTA = 512
+// threads (four warpgroups), one per SM (persistent grid); setmaxnreg moves
+// registers to the softmax warpgroups, which hold a whole 128-key row of S:
 //   warps 0-7   softmax, two warpgroups taking alternate KV tiles
 //               (ping-pong): warp w owns rows 32(w%4) .. 32(w%4)+31 of the
-//               tile (TMEM lane quarter w%4), all 128 keys; reference max
-//               (handed from group to group), P (Lean-P codes or bf16),
-//               rescale factor
-//   warps 8-11  correction: rescales O (and the FP8 row sum) when the running
-//               max grew, then the epilogue O / l -> bf16 -> global
+//               tile (TMEM lane quarter w%4), all 128 keys.  Per tile: one
+//               TMEM read of S (the S buffer is released at once), reference
+//               max (handed from group to group), P (Lean-P codes or bf16),
+//               and, when the reference max moved, the O rescale of its rows
+//   warps 8-11  epilogue: O / l -> bf16 -> global, once per unit
 //   warp 12     TMA producer (one elected thread): Q tile per unit, K/V ring
 //   warp 13     S issuer (one elected thread): S = Q K^T
 //   warp 14     P V issuer (one elected thread): O += P V (+ the FP8 row sum)
+//   warp 15     idle (completes the fourth warpgroup for setmaxnreg)
 // The two MMA streams are issued by different warps so that S of a later
 // tile never queues behind P V of an earlier one (each warp commits only its
 // own MMAs; the hand-offs between them go through the barriers).
 // Work unit = (batch, query head, 128-row query tile); KV tiles 0..qt only
 // (fully masked tiles are never issued), ascending, so results are
-// deterministic.  S has two TMEM buffers: the MMA of S for tile j+1 runs
-// while the softmax works on tile j; P V of tile j runs while the softmax
-// works on tile j+1.
+// deterministic.  S has two TMEM buffers: the MMA of S for tile j+2 runs
+// as soon as the softmax has read S of tile j; P V of tile j runs while the
+// softmax works on tile j+1.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -63,15 +64,33 @@ struct AttnArgs {
   unsigned long long timeout_ns;
 };
 
-constexpr int kAttnThreads = 480;
+constexpr int kAttnThreads = 512;
+// Register split (setmaxnreg; the launch holds 512 x 128 = 65536 registers,
+// the whole register file, and the four shares below add up to it):
+// softmax warpgroups hold a 128-key row of S plus its codes, the epilogue
+// warpgroup one 32-column slice of O, the producer / issuer warpgroup only
+// loop state.
+constexpr uint32_t kRegSoftmax = 192, kRegEpilogue = 80, kRegControl = 48;
+static_assert(128 * (2 * kRegSoftmax + kRegEpilogue + kRegControl) == 65536, "register split");
 // Deferred reference max (both paths): the max that the probabilities are
 // taken against moves only when a tile's max exceeds it by more than this
-// many binades (FlashAttention-4's lazy rescale).  O and the row sum always
-// share the reference, so the softmax is unchanged and the O rescale, which
-// serialises P V behind the previous tile, becomes rare.  FP8: the 64-key
-// block shift j renormalises every block to its own max, so the codes keep
-// their precision and j stays >= 8 - kRescaleLog2 >= 0.
-constexpr float kRescaleLog2 = 8.0f;
+// many binades (FlashAttention-4's lazy rescale, with a far larger bound).
+// O and the row sum always share the reference, so the softmax is unchanged,
+// and the O rescale, which makes P V of a tile wait for P V of the previous
+// one, becomes rare.  The bound is set by number range, not precision: FP8
+// renormalises every 64-key block to its own max with the shift j (its top
+// code stays in (112, 120]), so a block above the reference only takes j down
+// to 8 - kRescaleLog2 and an E8M0 scale 2^(kRescaleLog2 - 8) > 1; BF16 P
+// values reach 2^kRescaleLog2, inside bf16's range.  Weights <= 2^64 keep O
+// (at most 2^64 * 448 * 2^17 for S <= 2^17) and the row sum far inside fp32.
+constexpr float kRescaleLog2 = 64.0f;
+static_assert(kRescaleLog2 <= 100.0f, "E8M0 scale range and fp32 accumulator headroom");
+// Unit hand-overs from the softmax warpgroups to the epilogue (the final
+// reference max, and for BF16 each group's partial row sum) go through a ring
+// of this many slots, each with its own barrier.  A group can get ahead of
+// the epilogue by at most P-buffer count + 2 units (its P buffer waits tie it
+// to P V, and P V of the next unit waits for the epilogue), so 8 > 3 + 2.
+constexpr int kHandSlots = 8;
 
 template <bool FP8, int DQK>
 struct AttnCfg {
@@ -97,19 +116,21 @@ struct AttnCfg {
   static constexpr int OFF_V = OFF_K + STK * KB;
   static constexpr int OFF_ONES = OFF_V + STV * VB;   // FP8: 16 x 128 bytes of e4m3 1.0
   static constexpr int OFF_SF = OFF_ONES + (FP8 ? 2048 : 0);   // FP8: NPB x 512 B scale factors
-  static constexpr int OFF_ALPHA = OFF_SF + (FP8 ? NPB * 512 : 0);  // NPB x 128 fp32 rescale factors
-  static constexpr int OFF_LFIN = OFF_ALPHA + NPB * 512;  // BF16: final partial row sums per group (2 x 128 fp32);
-                                                          // FP8: final reference max per unit (4 x 128 fp32)
-  static constexpr int OFF_XCH = OFF_LFIN + 2048;    // running max per group (2 x 128) + BF16 final max per group (2 x 128)
-  static constexpr int OFF_BAR = OFF_XCH + 2048;
+  // unit hand-over ring: reference max per slot x group x row, and (BF16)
+  // the group's partial row sum in a second array of the same shape
+  static constexpr int HAND = kHandSlots * 2 * 128 * 4;
+  static constexpr int OFF_HAND = OFF_SF + (FP8 ? NPB * 512 : 0);
+  static constexpr int OFF_XCH = OFF_HAND + (FP8 ? 1 : 2) * HAND;   // running max per group (2 x 128)
+  static constexpr int OFF_BAR = OFF_XCH + 1024;
   // Barriers (phase bookkeeping: every waiter is at most one phase behind,
   // so a parity test cannot alias): Q full/empty per Q buffer; OF = O read
   // by the epilogue (per unit); OFIN = last P V of a unit done (per unit);
   // per S buffer: SF = S full, SC = S read, MX = running max published; per
-  // P buffer: PF = P/alpha written, PE = P V done (P buffer free, O
-  // updated), OR = O corrected, ready for P V.
+  // P buffer: PF = P written and O rescaled (ready for P V), PE = P V done (P
+  // buffer free, O updated); per hand-over slot: LF = both softmax groups
+  // wrote their unit hand-over.
   enum { QF0 = 0, QF1, QE0, QE1, OF, OFIN, DRAIN, DRAIN2, SF0, SF1, SC0, SC1, PF0, PF1, PF2, PE0, PE1, PE2,
-         OR0, OR1, OR2, MX0, MX1, KF };
+         MX0, MX1, LF0, KF = LF0 + kHandSlots };
   static constexpr int KE = KF + STK, VF = KF + 2 * STK, VE = VF + STV;
   static constexpr int NBAR = VE + STV;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -371,8 +392,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sb + Cf::OFF_BAR + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + Cf::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Cf::OFF_MISC + 4);
-  float* alpha_s = reinterpret_cast<float*>(sm + Cf::OFF_ALPHA);
-  float* lfin_s = reinterpret_cast<float*>(sm + Cf::OFF_LFIN);
+  float* hand_m = reinterpret_cast<float*>(sm + Cf::OFF_HAND);               // [slot][group][row]
+  float* hand_l = reinterpret_cast<float*>(sm + Cf::OFF_HAND + Cf::HAND);    // BF16 only, same shape
   uint32_t* sf_s = reinterpret_cast<uint32_t*>(sm + Cf::OFF_SF);
   float* xch_s = reinterpret_cast<float*>(sm + Cf::OFF_XCH);
 
@@ -394,8 +415,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < Cf::NPB; ++i) {
       mbar_init(bar(Cf::PF0 + i), 128);
       mbar_init(bar(Cf::PE0 + i), 1);
-      mbar_init(bar(Cf::OR0 + i), 128);
     }
+    for (int i = 0; i < kHandSlots; ++i) mbar_init(bar(Cf::LF0 + i), 256);
     for (int i = 0; i < Cf::STK; ++i) {
       mbar_init(bar(Cf::KF + i), 1);
       mbar_init(bar(Cf::KE + i), 1);
@@ -426,15 +447,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
   const WaitCtl ctl{abort_flag, a.timeout_ns};
-  typename std::conditional<VARLEN, VarlenIter, UnitIter>::type units;
-  if constexpr (VARLEN) units.init(gridDim.x, blockIdx.x, vs, a.Hq, a.Hkv);
-  else units.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
 
   if (warp >= 12) {
+   reg_dealloc<kRegControl>();
    // The producer and MMA warps run converged; one elected lane polls the
    // barriers and issues the TMA copies / tcgen05 instructions and the
    // commits, so every operand (descriptors, TMEM addresses, coordinates) is
-   // warp-uniform.
+   // warp-uniform.  Warp 15 has no role.
    const bool leader = elect_one();
    const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
    auto wait1 = [&](uint32_t br, uint32_t parity) -> bool {
@@ -451,6 +470,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     ks.init(gridDim.x, blockIdx.x, a, vs);
     vst.init(gridDim.x, blockIdx.x, a, vs);
     bool ok = true;
+    // the last unit / tile whose Q, K and V copies were armed (-1: none): on an
+    // abort, the last armed phase of every buffer is waited for, so no copy
+    // lands after the CTA exits
+    int last_q = -1, last_k = -1, last_v = -1;
     auto load_rows = [&](uint32_t dst, const CUtensorMap* m, const CUtensorMap* mt, uint32_t br,
                          int h, int row, int bb, uint64_t pol) {
 #pragma unroll
@@ -473,6 +496,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           load_rows(sb + Cf::OFF_Q + slot * Cf::QB, &a.map_q, &a.map_q_tail, bar(Cf::QF0 + slot),
                     t.hq, row0 + t.qt * 128, tb, pol_q);
         }
+        last_q = static_cast<int>(t.u);
       }
       const uint32_t st = t.g % Cf::STK, n = t.g / Cf::STK;
       if (n > 0 && !wait1(bar(Cf::KE + st), (n - 1) & 1)) return false;
@@ -481,6 +505,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         load_rows(sb + Cf::OFF_K + st * Cf::KB, &a.map_k, &a.map_k_tail, bar(Cf::KF + st), t.hkv,
                   row0 + t.j * 128, tb, pol_kv);
       }
+      last_k = static_cast<int>(t.g);
       __syncwarp();
       return true;
     };
@@ -495,6 +520,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_load_4d(sb + Cf::OFF_V + st * Cf::VB + c * Cf::CHUNK, &a.map_v, bar(Cf::VF + st),
                       c * (128 / Cf::EL), t.hkv, row0 + t.j * 128, tb, pol_kv);
       }
+      last_v = static_cast<int>(t.g);
       __syncwarp();
       return true;
     };
@@ -503,16 +529,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ks.next()) ok = load_k(ks);
       if (ok) ok = load_v(vst);
     }
-    if (!ok) {
-      // let copies already in flight land before the CTA exits
-      const uint64_t t0 = globaltimer_ns();
-      while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+    if (!ok && leader) {
+      // let the copies already in flight land before the CTA exits: each
+      // buffer's last armed phase completes when its bytes have arrived
+      // buffer i's last armed use is the largest index <= last with index % n == i
+      auto drain_ring = [&](int last, int n, int bar0) {
+        for (int i = 0; i < n && i <= last; ++i) {
+          const int x = last - (((last - i) % n) + n) % n;
+          drain_wait(bar(bar0 + i), static_cast<uint32_t>(x / n) & 1u, 100000000ull);
+        }
+      };
+      drain_ring(last_q, Cf::QBUF, Cf::QF0);
+      drain_ring(last_k, Cf::STK, Cf::KF);
+      drain_ring(last_v, Cf::STV, Cf::VF);
     }
+    __syncwarp();
    } else if (warp == 13 || warp == 14) {
     // ------------------------------------------------------------ MMA issuers
-    // warp 9: S for tile g is issued as soon as its K tile is loaded and the
-    // softmax has read S of tile g-2 (two S buffers).  warp 10: P V of tile g
-    // once the softmax has written P and the correction has rescaled O.
+    // warp 13: S for tile g is issued as soon as its K tile is loaded and the
+    // softmax has read S of tile g-2 (two S buffers).  warp 14: P V of tile g
+    // once the softmax has written P (and rescaled O, when it had to).
     TS ts;
     ts.init(gridDim.x, blockIdx.x, a, vs);
     bool ok = true;
@@ -560,8 +596,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool first = t.j == 0;
       // O is free once the previous unit's epilogue has read it
       if (first && t.u > 0 && !wait1(bar(Cf::OF), (t.u - 1) & 1)) return false;
-      if (!wait1(bar(Cf::OR0 + buf), ph)) return false;   // P stored, O corrected
       if (!wait1(bar(Cf::VF + st), (t.g / Cf::STV) & 1)) return false;
+      if (!wait1(bar(Cf::PF0 + buf), ph)) return false;   // P stored, O rescaled
       tc_fence_after();
       const uint64_t dvs = dv + ((st * Cf::VB) >> 4);
       const uint32_t tp = tbase + Cf::tp(buf);
@@ -607,13 +643,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
    }
   } else if (warp < 8) {
+    reg_alloc<kRegSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
     // Two groups alternate over the KV tiles: group x = warp / 4 takes the
-    // tiles with (g & 1) == x, i.e. always S buffer x and P buffer x, so one
-    // group computes while the other waits for its next S.  Thread t of a
-    // group owns row 32 (w % 4) + lane (TMEM lane quarter w % 4) and all 128
-    // keys of its tiles.  The running max crosses between the groups once per
-    // tile (smem + per-buffer barrier MX), the only serial dependency.
+    // tiles with (g & 1) == x, i.e. always S buffer x, so one group computes
+    // while the other waits for its next S.  Thread t of a group owns row
+    // 32 (w % 4) + lane (TMEM lane quarter w % 4) and all 128 keys of its
+    // tiles.  The running max crosses between the groups once per tile (smem
+    // + per-buffer barrier MX), the only serial dependency.
     const int grp = warp >> 2;
     const int row = 32 * (warp & 3) + lane;   // query row inside the tile == TMEM lane
     const uint32_t lb = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -628,7 +665,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     TS t;
     t.init(gridDim.x, blockIdx.x, a, vs);
     float A = a.C;
-    float l = 0.0f, m_own = __int_as_float(0xff800000);   // BF16: this group's row sum and its max
+    // this group's latest reference max in the unit, and (BF16) its partial
+    // row sum relative to that max
+    float l = 0.0f, m_own = __int_as_float(0xff800000);
     while (ok && t.next()) {
       const uint32_t g = t.g;
       if (t.j == 0) {
@@ -642,165 +681,119 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           A = leanp_slope(qs, ks, a.C);
         }
       }
-      if ((g & 1) != static_cast<uint32_t>(grp)) continue;
-      const bool diag = t.j == t.qt;
-      if (!(ok = warp_wait(bar(Cf::SF0 + grp), (g >> 1) & 1, ctl))) break;
-      tc_fence_after();
-      // pass 1: block maxima (loops over the two 64-key blocks are kept rolled:
-      // a compact hot loop keeps the instruction cache warm for the 15 warps
-      // of the CTA).  Block 1 stays in registers for pass 2.
-      float bmx0 = 0.0f, bmx1 = 0.0f;
-      uint32_t r[64];
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        tmem_ld32p(ts + 64 * h, &r[0]);
-        tmem_ld32p(ts + 64 * h + 32, &r[32]);
+      if ((g & 1) == static_cast<uint32_t>(grp)) {
+        const bool diag = t.j == t.qt;
+        if (!(ok = warp_wait(bar(Cf::SF0 + grp), (g >> 1) & 1, ctl))) break;
+        tc_fence_after();
+        // the whole 128-key row of S in one TMEM round trip; the S buffer is
+        // free for the tile after next right away
+        uint32_t r[128];
+        tmem_ld32p(ts, &r[0]);
+        tmem_ld32p(ts + 32, &r[32]);
+        tmem_ld32p(ts + 64, &r[64]);
+        tmem_ld32p(ts + 96, &r[96]);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(Cf::SC0 + grp));
         if (diag) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (64 * h + c > row) r[c] = 0xff800000u;   // -inf: key after the query row
+          for (int c = 0; c < 128; ++c)
+            if (c > row) r[c] = 0xff800000u;   // -inf: key after the query row
         }
-        const float bm = max64(r);
-        if (h == 0) bmx0 = bm; else bmx1 = bm;
-      }
-      // running max of the previous tile, from the other group (every tile
-      // waits for it, so the exchange buffers are never reused early)
-      float m_prev = __int_as_float(0xff800000);
-      if (g >= 1) {
-        const uint32_t pb = (g - 1) & 1;
-        if (!(ok = warp_wait(bar(Cf::MX0 + pb), ((g - 1) >> 1) & 1, ctl))) break;
-        if (t.j > 0) m_prev = xch_s[pb * 128 + row];
-      }
-      // reference max after this tile (FP8: A carries a factor 8)
-      float m, alpha = 1.0f;
-      const float tmax = fmaxf(bmx0, bmx1);
-      if (t.j == 0) {
-        m = tmax;
-      } else if (__fmul_rn(tmax - m_prev, A) > (FP8 ? 8.0f * kRescaleLog2 : kRescaleLog2)) {
-        alpha = ex2_approx(FP8 ? __fmul_rn(__fmul_rn(m_prev - tmax, A), 0.125f)
-                               : __fmul_rn(m_prev - tmax, A));
-        m = tmax;
-      } else {
-        m = m_prev;
-      }
-      xch_s[grp * 128 + row] = m;
-      mbar_arrive(bar(Cf::MX0 + grp));
-      // P V of tile g-NPB has read this P buffer (and its scale factors)
-      const uint32_t pbuf = g % Cf::NPB;
-      const uint32_t tp = lb + Cf::tp(pbuf);
-      if (g >= static_cast<uint32_t>(Cf::NPB) &&
-          !(ok = warp_wait(bar(Cf::PE0 + pbuf), ((g / Cf::NPB) - 1) & 1, ctl))) break;
-      // pass 2: probabilities, block 1 first (still in registers), then block
-      // 0 (read again; after that S is no longer needed and its buffer takes
-      // the tile after next)
-      float rowsum = 0.0f;
-      uint32_t sfw = 0;
-#pragma unroll 1
-      for (int h = 1; h >= 0; --h) {
-        if (h == 0) {
-          tmem_ld32p(ts, &r[0]);
-          tmem_ld32p(ts + 32, &r[32]);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(bar(Cf::SC0 + grp));   // S buffer free for the tile after next
-          if (diag) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c > row) r[c] = 0xff800000u;
-          }
+        const float bmx0 = max64(&r[0]), bmx1 = max64(&r[64]);
+        // running max of the previous tile, from the other group (every tile
+        // waits for it, so the exchange buffers are never reused early)
+        float m_prev = __int_as_float(0xff800000);
+        if (g >= 1) {
+          const uint32_t pb = (g - 1) & 1;
+          if (!(ok = warp_wait(bar(Cf::MX0 + pb), ((g - 1) >> 1) & 1, ctl))) break;
+          if (t.j > 0) m_prev = xch_s[pb * 128 + row];
         }
+        // reference max after this tile (FP8: A carries a factor 8)
+        float m, alpha = 1.0f;
+        const float tmax = fmaxf(bmx0, bmx1);
+        if (t.j == 0) {
+          m = tmax;
+        } else if (__fmul_rn(tmax - m_prev, A) > (FP8 ? 8.0f * kRescaleLog2 : kRescaleLog2)) {
+          alpha = ex2_approx(FP8 ? __fmul_rn(__fmul_rn(m_prev - tmax, A), 0.125f)
+                                 : __fmul_rn(m_prev - tmax, A));
+          m = tmax;
+        } else {
+          m = m_prev;
+        }
+        xch_s[grp * 128 + row] = m;
+        mbar_arrive(bar(Cf::MX0 + grp));
+        // P V of tile g-NPB has read this P buffer (and its scale factors)
+        const uint32_t pbuf = g % Cf::NPB;
+        const uint32_t tp = lb + Cf::tp(pbuf);
+        if (g >= static_cast<uint32_t>(Cf::NPB) &&
+            !(ok = warp_wait(bar(Cf::PE0 + pbuf), ((g / Cf::NPB) - 1) & 1, ctl))) break;
         if (FP8) {
-          const int jb = leanp_block_shift(m, h ? bmx1 : bmx0, A);
-          uint32_t p[16];
-          if (EXACTP) {
-            // p = exp2((s - m) A / 8 + j): one FMA, MUFU ex2, then e4m3
-            const float a8 = __fmul_rn(A, 0.125f);
-            const float b8 = __fmaf_rn(-m, a8, static_cast<float>(jb));
+          uint32_t sfw = 0;
 #pragma unroll
-            for (int w = 0; w < 16; ++w) {
-              const float e0 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w]), a8, b8));
-              const float e1 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w + 1]), a8, b8));
-              const float e2 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w + 2]), a8, b8));
-              const float e3 = ex2_approx(__fmaf_rn(__uint_as_float(r[4 * w + 3]), a8, b8));
-              p[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t* rh = &r[64 * h];
+            const int jb = leanp_block_shift(m, h ? bmx1 : bmx0, A);
+            uint32_t p[16];
+            if (EXACTP) {
+              // p = exp2((s - m) A / 8 + j): one FMA, MUFU ex2, then e4m3
+              const float a8 = __fmul_rn(A, 0.125f);
+              const float b8 = __fmaf_rn(-m, a8, static_cast<float>(jb));
+#pragma unroll
+              for (int w = 0; w < 16; ++w) {
+                const float e0 = ex2_approx(__fmaf_rn(__uint_as_float(rh[4 * w]), a8, b8));
+                const float e1 = ex2_approx(__fmaf_rn(__uint_as_float(rh[4 * w + 1]), a8, b8));
+                const float e2 = ex2_approx(__fmaf_rn(__uint_as_float(rh[4 * w + 2]), a8, b8));
+                const float e3 = ex2_approx(__fmaf_rn(__uint_as_float(rh[4 * w + 3]), a8, b8));
+                p[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
+              }
+            } else {
+              const float Bb = leanp_row_offset(m, A, jb);
+              const float a256 = __fmul_rn(A, 0.00390625f), b256 = __fmul_rn(Bb, 0.00390625f);
+#pragma unroll
+              for (int w = 0; w < 16; ++w) {
+                uint32_t w0, w1, w2, w3;
+                leanp_code_word2(__uint_as_float(rh[4 * w]), __uint_as_float(rh[4 * w + 1]), a256, b256, w0, w1);
+                leanp_code_word2(__uint_as_float(rh[4 * w + 2]), __uint_as_float(rh[4 * w + 3]), a256, b256, w2, w3);
+                p[w] = pack4_low_bytes(w0, w1, w2, w3);
+              }
             }
-          } else {
-            const float Bb = leanp_row_offset(m, A, jb);
-            const float a256 = __fmul_rn(A, 0.00390625f), b256 = __fmul_rn(Bb, 0.00390625f);
-#pragma unroll
-            for (int w = 0; w < 16; ++w)
-              p[w] = pack4_low_bytes(leanp_code_word(__uint_as_float(r[4 * w]), a256, b256),
-                                     leanp_code_word(__uint_as_float(r[4 * w + 1]), a256, b256),
-                                     leanp_code_word(__uint_as_float(r[4 * w + 2]), a256, b256),
-                                     leanp_code_word(__uint_as_float(r[4 * w + 3]), a256, b256));
+            tmem_st16p(tp + 16 * h, p);
+            // E8M0 scale code 127 - j for both 32-key MX blocks of this 64-key block
+            sfw |= static_cast<uint32_t>((127 - jb) * 0x0101) << (16 * h);
           }
-          tmem_st16p(tp + 16 * h, p);
-          // E8M0 scale code 127 - j for both 32-key MX blocks of this 64-key block
-          sfw |= static_cast<uint32_t>((127 - jb) * 0x0101) << (16 * h);
+          sf_s[pbuf * 128 + sf_row] = sfw;
+          fence_proxy_async_smem();   // the copy to TMEM reads it through the async proxy
         } else {
           const float mc = m * A;
-          float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          const uint64_t A2 = f2_pack(A, A), nmc2 = f2_pack(-mc, -mc);
+          uint64_t acc2[2] = {0, 0};
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
+          for (int c8 = 0; c8 < 8; ++c8) {
             uint32_t pb[8];
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
-              const float p0 = ex2_approx(__fmaf_rn(__uint_as_float(r[16 * c4 + 2 * w]), A, -mc));
-              const float p1 = ex2_approx(__fmaf_rn(__uint_as_float(r[16 * c4 + 2 * w + 1]), A, -mc));
-              acc[w & 3] += p0 + p1;
+              float x0, x1;
+              f2_unpack(fma2_rn(f2_pack(__uint_as_float(r[16 * c8 + 2 * w]), __uint_as_float(r[16 * c8 + 2 * w + 1])),
+                                A2, nmc2), x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              acc2[w & 1] = add2_rn(acc2[w & 1], f2_pack(p0, p1));
               pb[w] = pack_bf16x2(p0, p1);
             }
-            tmem_st8p(tp + 32 * h + 8 * c4, pb);
+            tmem_st8p(tp + 8 * c8, pb);
           }
-          rowsum += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          float s0, s1, s2, s3;
+          f2_unpack(acc2[0], s0, s1);
+          f2_unpack(acc2[1], s2, s3);
+          // this group's partial row sum, kept relative to the newest max
+          l = l * ex2_approx(__fmul_rn(m_own - m, A)) + ((s0 + s1) + (s2 + s3));
         }
-      }
-      if (FP8) {
-        sf_s[pbuf * 128 + sf_row] = sfw;
-        fence_proxy_async_smem();   // the copy to TMEM reads it through the async proxy
-        // the unit's final reference max, for the log-sum-exp (slot per unit
-        // mod 4: unit u+4's last tile comes after P V of unit u+1's first
-        // tile, which waits for the epilogue of unit u that reads this slot)
-        if (t.j == t.nkv - 1) lfin_s[(t.u & 3) * 128 + row] = m;
-      } else {
-        // this group's partial row sum, kept relative to the newest max
-        l = l * ex2_approx(__fmul_rn(m_own - m, A)) + rowsum;
         m_own = m;
-        if (t.j >= t.nkv - 2) {   // this group's last tile of the unit: hand over (l, m)
-          lfin_s[grp * 128 + row] = l;
-          xch_s[(2 + grp) * 128 + row] = m_own;
-        }
-      }
-      alpha_s[pbuf * 128 + row] = alpha;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(Cf::PF0 + pbuf));
-    }
-  } else {
-    // ------------------------------------------------------------ correction warpgroup
-    const int row = 32 * (warp & 3) + lane;
-    const uint32_t lb = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    uint32_t kv_it = 0, u_it = 0;
-    int b, hkv, hq, qt;
-    int r0 = 0, len = 0;   // VARLEN: the unit's sequence's first packed row and length
-    bool ok = true;
-    while (ok && (VARLEN ? units.next(b, hkv, hq, qt, r0, len) : units.next(b, hkv, hq, qt))) {
-      const int nkv = qt + 1;
-      // BF16: each softmax group hands over its partial row sum and the max it
-      // is relative to at its last tile of the unit (one of the last two)
-      float lg0 = 0.0f, lg1 = 0.0f, mg0 = 0.0f, mg1 = 0.0f;
-      for (int j = 0; j < nkv; ++j, ++kv_it) {
-        const uint32_t buf = kv_it & 1, pbuf = kv_it % Cf::NPB;
-        if (!(ok = warp_wait(bar(Cf::PF0 + pbuf), (kv_it / Cf::NPB) & 1, ctl))) break;
-        const float alpha = alpha_s[pbuf * 128 + row];
-        if (!FP8 && j >= nkv - 2) {
-          const float lv = lfin_s[buf * 128 + row], mv = xch_s[(2 + buf) * 128 + row];
-          if (buf) { lg1 = lv; mg1 = mv; } else { lg0 = lv; mg0 = mv; }
-        }
+        // the reference max moved: O (and the FP8 row sum) still hold tiles
+        // 0 .. g-1 against the old one; rescale this warp's rows once P V of
+        // tile g-1 has landed (P V of tile g waits for PF below)
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-          // O holds tiles 0..j-1: wait for P V of tile j-1, then scale the rows
-          const uint32_t pg = kv_it - 1;
+          const uint32_t pg = g - 1;
           if (!(ok = warp_wait(bar(Cf::PE0 + pg % Cf::NPB), (pg / Cf::NPB) & 1, ctl))) break;
           tc_fence_after();
 #pragma unroll
@@ -817,15 +810,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_wait_ld();
             tmem_st1(lb + Cf::TL, __float_as_uint(__uint_as_float(lv) * alpha));
           }
-          tmem_wait_st();
         }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(Cf::OR0 + pbuf));
+        mbar_arrive(bar(Cf::PF0 + pbuf));
       }
-      if (!ok) break;
-      // ---- epilogue: O / l (* v_scale) -> bf16, rows past S are not written
+      if (t.j == t.nkv - 1) {
+        // the unit's last tile (this group's or the other's): hand this
+        // group's final (row sum, reference max) over to the epilogue
+        const uint32_t hs = t.u % kHandSlots;
+        hand_m[(hs * 2 + grp) * 128 + row] = m_own;
+        if (!FP8) hand_l[(hs * 2 + grp) * 128 + row] = l;
+        mbar_arrive(bar(Cf::LF0 + hs));
+      }
+    }
+  } else {
+    reg_dealloc<kRegEpilogue>();
+    // ------------------------------------------------------------ epilogue warpgroup
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lb = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    typename std::conditional<VARLEN, VarlenIter, UnitIter>::type units;
+    if constexpr (VARLEN) units.init(gridDim.x, blockIdx.x, vs, a.Hq, a.Hkv);
+    else units.init(gridDim.x, blockIdx.x, a.Tq, a.Hq, a.Hkv, a.B, a.group_slots);
+    uint32_t kv_it = 0, u_it = 0;
+    int b, hkv, hq, qt;
+    int r0 = 0, len = 0;   // VARLEN: the unit's sequence's first packed row and length
+    bool ok = true;
+    while (ok && (VARLEN ? units.next(b, hkv, hq, qt, r0, len) : units.next(b, hkv, hq, qt))) {
+      const int nkv = qt + 1;
+      kv_it += nkv;
+      // ---- O / l (* v_scale) -> bf16, rows past S are not written
       if (!(ok = warp_wait(bar(Cf::OFIN), u_it & 1, ctl))) break;
+      const uint32_t hs = u_it % kHandSlots;
+      if (!(ok = warp_wait(bar(Cf::LF0 + hs), (u_it / kHandSlots) & 1, ctl))) break;
       tc_fence_after();
+      // the group of the unit's last tile holds the final reference max
+      const int gl = static_cast<int>((kv_it - 1) & 1);
+      const float m_last = hand_m[(hs * 2 + gl) * 128 + row];
       float inv, lse_log2;   // lse_log2: log-sum-exp of the scaled scores, in binades
       const int grow = qt * 128 + row;
       if (FP8) {
@@ -839,15 +860,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float qs = (a.q_scale && sok) ? a.q_scale[b * a.Hq + hq] : 1.0f;
           const float ks = (a.k_scale && sok) ? a.k_scale[b * a.Hkv + hkv] : 1.0f;
           const float A8 = __fmul_rn(leanp_slope(qs, ks, a.C), 0.125f);
-          lse_log2 = __fmaf_rn(lfin_s[(u_it & 3) * 128 + row], A8, log2f(lv));
+          lse_log2 = __fmaf_rn(m_last, A8, log2f(lv));
         }
       } else {
-        // the group of the unit's last tile holds the final max
-        const bool last1 = ((kv_it - 1) & 1) != 0;
-        const float l_last = last1 ? lg1 : lg0, m_last = last1 ? mg1 : mg0;
-        const float l_oth = last1 ? lg0 : lg1, m_oth = last1 ? mg0 : mg1;
-        float lt = l_last;
-        if (nkv >= 2) lt += l_oth * ex2_approx(__fmul_rn(m_oth - m_last, a.C));
+        // each group's partial row sum is relative to its own latest max
+        const int go = gl ^ 1;
+        float lt = hand_l[(hs * 2 + gl) * 128 + row];
+        if (nkv >= 2)
+          lt += hand_l[(hs * 2 + go) * 128 + row] * ex2_approx(__fmul_rn(hand_m[(hs * 2 + go) * 128 + row] - m_last, a.C));
         inv = 1.0f / lt;
         if (a.lse) lse_log2 = __fmaf_rn(m_last, a.C, log2f(lt));
       }

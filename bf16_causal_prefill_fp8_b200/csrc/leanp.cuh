@@ -18,11 +18,18 @@
 //   B    = fma(-m, A, 56 + 8 j)                                   per row, block
 //   u    = fma(s, A, B)                                           per element
 //   code = trunc(max(u, 0))           (see leanp_code_word)
-// s is the raw fp32 score (sum of products of e4m3 values), m the running row
-// maximum after this key tile and bmax the maximum of the element's 64-key
-// block.  Precondition: s <= bmax <= m, or s = -inf for a masked key; then
-// u <= 120 and the code never exceeds 126 (127 would be NaN).  The weight the
-// matrix unit applies is value(code) * 2^-j: E8M0 scale code 127 - j.
+// s is the raw fp32 score (sum of products of e4m3 values), m the reference
+// row maximum after this key tile and bmax the maximum of the element's 64-key
+// block.  The reference max is deferred: it moves only when a tile's max
+// exceeds it by more than 8 binades, so a block max may lie above m by up to
+// that much, (bmax - m) A <= 64, and then j = 8 + floor of a negative number
+// is 0..7.  Precondition: s <= bmax and j >= 0, or s = -inf for a masked key.
+// Then the block max lands at u = 120 - 8 frac(((m - bmax) A) / 8), in
+// (112, 120] (one lower where the fp32 steps round across an integer), every
+// other u is below it, and the code never exceeds 126 (127 would be NaN; the
+// device code does not clamp at 126 and relies on this bound).  The weight
+// the matrix unit applies is value(code) * 2^-j: E8M0 scale code 127 - j,
+// at most 127 (2^0) for j >= 0.
 #pragma once
 #include <cstdint>
 
@@ -65,6 +72,23 @@ __device__ __forceinline__ uint32_t leanp_word(float x) {
 // One score -> a word whose low byte is its code (a256 = A/256, b256 = B/256).
 __device__ __forceinline__ uint32_t leanp_code_word(float s, float a256, float b256) {
   return leanp_word(leanp_scaled_u(s, a256, b256));
+}
+
+// leanp_word for two values at once: one packed round-toward-zero FMA
+// (fma.rz.f32x2 applies the same IEEE operation to each half, so each word
+// equals leanp_word's).
+__device__ __forceinline__ void leanp_word2(float x0, float x1, uint32_t& w0, uint32_t& w1) {
+  uint64_t x, w;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  asm("fma.rz.f32x2 %0, %1, %2, %3;" : "=l"(w) : "l"(x), "l"(0x4380000043800000ull), "l"(0x4B4000004B400000ull));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(w0), "=r"(w1) : "l"(w));
+}
+
+// Two scores of one (row, block) -> two code words: the saturating FMA per
+// score, then leanp_word2.
+__device__ __forceinline__ void leanp_code_word2(float s0, float s1, float a256, float b256, uint32_t& w0,
+                                                 uint32_t& w1) {
+  leanp_word2(leanp_scaled_u(s0, a256, b256), leanp_scaled_u(s1, a256, b256), w0, w1);
 }
 
 // Four code words -> one 32-bit word holding the four code bytes in order.

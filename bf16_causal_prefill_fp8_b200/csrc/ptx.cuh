@@ -134,6 +134,47 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
 }
 
 // ---------------------------------------------------------------------------
+// setmaxnreg: raise / lower this warpgroup's per-thread register limit (all
+// four warps of the warpgroup execute it; a raise waits until lowered
+// warpgroups have returned enough registers)
+// ---------------------------------------------------------------------------
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------------------
+// Packed fp32 pairs (f32x2: one instruction, the same IEEE operation on both
+// halves; the first value in the low half)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t fma2_rn(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t add2_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ---------------------------------------------------------------------------
 // TMA: 4-D tiled bulk tensor load global -> shared, completion on an mbarrier
 // (complete_tx).  Coordinates innermost first.  No cluster multicast.
 // ---------------------------------------------------------------------------

@@ -205,16 +205,31 @@ int launch_attn_varlen(const void* q, const void* k, const void* v, void* o, con
 
 // ---------------------------------------------------------------- test kernels
 
+// Element pairs (i, i + 1) go through leanp_word2, the packed step the attention
+// kernel uses (an odd last element is paired with itself).
 __global__ void leanp_codes_kernel(const float* s, const float* m, const float* bmax, const float* A,
                                    const unsigned char* masked, int n, unsigned char* code, int* jout) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-    const float Ai = A[i], mi = m[i];
-    const int j = leanp_block_shift(mi, bmax[i], Ai);
-    const float B = leanp_row_offset(mi, Ai, j);
-    const float si = (masked && masked[i]) ? __int_as_float(0xff800000) : s[i];
-    const uint32_t w = leanp_code_word(si, __fmul_rn(Ai, 0.00390625f), __fmul_rn(B, 0.00390625f));
-    code[i] = static_cast<unsigned char>(w & 0xffu);
-    if (jout) jout[i] = j;
+  const int npairs = (n + 1) / 2;
+  for (int pi = blockIdx.x * blockDim.x + threadIdx.x; pi < npairs; pi += gridDim.x * blockDim.x) {
+    const int i0 = 2 * pi, i1 = (2 * pi + 1 < n) ? 2 * pi + 1 : 2 * pi;
+    float a256[2], b256[2], sv[2];
+    int jj[2];
+    const int idx[2] = {i0, i1};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int i = idx[e];
+      const float Ai = A[i], mi = m[i];
+      jj[e] = leanp_block_shift(mi, bmax[i], Ai);
+      const float B = leanp_row_offset(mi, Ai, jj[e]);
+      sv[e] = (masked && masked[i]) ? __int_as_float(0xff800000) : s[i];
+      a256[e] = __fmul_rn(Ai, 0.00390625f);
+      b256[e] = __fmul_rn(B, 0.00390625f);
+    }
+    uint32_t w0, w1;
+    leanp_word2(leanp_scaled_u(sv[0], a256[0], b256[0]), leanp_scaled_u(sv[1], a256[1], b256[1]), w0, w1);
+    code[i0] = static_cast<unsigned char>(w0 & 0xffu);
+    code[i1] = static_cast<unsigned char>(w1 & 0xffu);
+    if (jout) { jout[i0] = jj[0]; jout[i1] = jj[1]; }
   }
 }
 

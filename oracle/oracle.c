@@ -384,9 +384,9 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 /*           p_mode 2: value(exact-P e4m3 code) * 2^-j_block                 */
 /*   alpha = exp2((m - m') A / 8)            (0 on the first tile)          */
 /*   O     = alpha O + sum_j w_j value(vcode_j);  l = alpha l + sum_j w_j   */
-/* Every block shift j must stay >= 0 (weights <= 448, E8M0 scale <= 1):   */
-/* true for the exact max (j >= 8) and for the deferred one (j >= 8 - r);   */
-/* a violation returns -2.                                                  */
+/* Every block shift j must stay >= 8 with the exact max, and >= 8 - r     */
+/* with the deferred one (a block at most r binades above the reference);  */
+/* a violation (a reference that does not move when it must) returns -2.   */
 /* lse (may be NULL) [B, Hq, nrows]: ln 2 (m A/8 + log2 l) at the last tile. */
 /* The row sum l comes from the rounded weights, like the extra matrix      */
 /* instruction per block on the pages.  Output o_i = O / l * v_s.           */
@@ -452,7 +452,8 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
                     if (bmax[1] > mnew) mnew = bmax[1];
                 }
                 for (n = 0; n < 2; ++n)
-                    if (oracle_leanp_block_shift(mnew, bmax[n], A) < 0) {
+                    if (oracle_leanp_block_shift(mnew, bmax[n], A) <
+                        (rescale_log2 > 0.0f ? 8 - (int)ceilf(rescale_log2) : 8)) {
 #pragma omp atomic write
                         shift_err = 1;
                     }

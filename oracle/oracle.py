@@ -217,7 +217,7 @@ def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=
                                      B, Hq, Hkv, S, Dqk, Dv, int(p_mode), ctypes.c_float(rescale_log2), _ptr(r), n, _ptr(o),
                                      _ptr(lse))
     if rc == -2:
-        raise ArithmeticError("oracle_fp8_model_rows: a block shift fell below 0 (reference max too stale)")
+        raise ArithmeticError("oracle_fp8_model_rows: a block shift fell below its bound (reference max too stale)")
     if rc != 0:
         raise ValueError("oracle_fp8_model_rows: bad arguments")
     return (o, lse) if return_lse else o

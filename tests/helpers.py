@@ -21,7 +21,7 @@ TOL_FP8 = 3e-2
 TOL_FP8_MODEL = 8e-3
 # The kernel's deferred reference max: it moves when a tile's max exceeds it
 # by more than this many binades (the CPU replay takes the same rule).
-RESCALE_LOG2 = 8.0
+RESCALE_LOG2 = 64.0
 
 
 def bf16_round(x: np.ndarray) -> torch.Tensor:

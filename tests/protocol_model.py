@@ -2,7 +2,7 @@
 infrastructure; it shares no code with the kernel).
 
 Each role of the kernel (producer, S issuer, P V issuer, the two softmax
-groups, the correction warpgroup) is a generator that takes the same barrier
+groups, the epilogue warpgroup) is a generator that takes the same barrier
 waits and arrivals, in the same order, as its counterpart in
 csrc/attn_fwd.cuh; the tensor-core and TMA engines are queues that complete
 after random delays.  An mbarrier is a phase counter: a parity wait passes
@@ -12,9 +12,12 @@ when the completed-phase count has the other parity.  The model checks that
   (no aliasing: the waiter is never two phases behind);
 - no wait is stuck on a phase that is already complete;
 - nothing deadlocks;
-- no buffer is overwritten before its reader is done (S, P, rescale factors,
-  the reference-max exchange, the row-sum hand-over slots, the O accumulator
-  across units).
+- no buffer is overwritten before its reader is done (S, P, the
+  reference-max exchange, the unit hand-over slots, the O accumulator across
+  units), and O is rescaled only once P V of the previous tile has landed.
+
+`two_producers` splits the TMA producer into a K (and Q) warp and a V warp,
+each walking the tiles on its own (a variant that was once tried).
 
 `mutation` plants a known mistake, for the tests that show the model catches it.
 """
@@ -28,7 +31,8 @@ class Config:
     stv: int      # V ring stages
     qbuf: int     # Q tile buffers
     npb: int      # P buffers
-    fp8: bool     # FP8 hands the final max over per unit; BF16 per group
+    fp8: bool     # FP8 or BF16 (the same protocol)
+    hand: int = 8  # unit hand-over slots (and their barriers)
 
     @property
     def klead(self):
@@ -58,7 +62,7 @@ class _Bar:
             self.c += 1
 
 
-def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5):
+def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_producers=False):
     """Simulate one CTA that processes `units` (KV-tile counts per unit)."""
     rng = random.Random(seed)
     bars = {}
@@ -70,8 +74,10 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5):
         for n, c in (("QF", 1), ("QE", 1), ("SF", 1), ("SC", 128), ("MX", 128)):
             bar(f"{n}{i}", c)
     for i in range(cfg.npb):
-        for n, c in (("PF", 128), ("PE", 1), ("OR", 128)):
+        for n, c in (("PF", 128), ("PE", 1)):
             bar(f"{n}{i}", c)
+    for i in range(cfg.hand):
+        bar(f"LF{i}", 256)
     bar("OF", 128)
     bar("OFIN", 1)
     for i in range(cfg.stk):
@@ -81,9 +87,7 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5):
     tiles = [(u, j, nkv) for u, nkv in enumerate(units) for j in range(nkv)]
     fifos = {"qk": [], "pv": []}
     tma = []
-    st = {"P": {}, "alpha": {}, "O_unit": None, "pv_done": set(), "qk_done": set(), "Sread": {}, "xch": {}, "lfin": {},
-          "hand": {}}
-    lfin_slots = 3 if mutation == "lfin_mod3" else 4
+    st = {"P": {}, "O_unit": None, "pv_done": set(), "qk_done": set(), "Sread": {}, "xch": {}, "hand": {}}
 
     def wait(name, parity, need):
         b = bars[name]
@@ -99,27 +103,26 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5):
                 raise ProtocolError(f"stuck on {name}: phase {need} complete but parity {parity} fails")
             yield "wait"
 
+    def load_k(g):
+        u, j, nkv = tiles[g]
+        if j == 0:
+            slot, n = u % cfg.qbuf, u // cfg.qbuf
+            if n > 0:
+                yield from wait(f"QE{slot}", (n - 1) & 1, n - 1)
+            tma.append([rng.randint(5, 40), f"QF{slot}"])
+        s_, n = g % cfg.stk, g // cfg.stk
+        if n > 0:
+            yield from wait(f"KE{s_}", (n - 1) & 1, n - 1)
+        tma.append([rng.randint(5, 40), f"KF{s_}"])
+
+    def load_v(g):
+        s_, n = g % cfg.stv, g // cfg.stv
+        if n > 0:
+            yield from wait(f"VE{s_}", (n - 1) & 1, n - 1)
+        tma.append([rng.randint(5, 40), f"VF{s_}"])
+
     def producer():
         ks = vs = 0
-
-        def load_k(g):
-            u, j, nkv = tiles[g]
-            if j == 0:
-                slot, n = u % cfg.qbuf, u // cfg.qbuf
-                if n > 0:
-                    yield from wait(f"QE{slot}", (n - 1) & 1, n - 1)
-                tma.append([rng.randint(5, 40), f"QF{slot}"])
-            s, n = g % cfg.stk, g // cfg.stk
-            if n > 0:
-                yield from wait(f"KE{s}", (n - 1) & 1, n - 1)
-            tma.append([rng.randint(5, 40), f"KF{s}"])
-
-        def load_v(g):
-            s, n = g % cfg.stv, g // cfg.stv
-            if n > 0:
-                yield from wait(f"VE{s}", (n - 1) & 1, n - 1)
-            tma.append([rng.randint(5, 40), f"VF{s}"])
-
         for _ in range(cfg.klead):
             if ks < len(tiles):
                 yield from load_k(ks); ks += 1
@@ -129,28 +132,38 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5):
             yield from load_v(vs); vs += 1
             yield "step"
 
+    def producer_k():
+        for g in range(len(tiles)):
+            yield from load_k(g)
+            yield "step"
+
+    def producer_v():
+        for g in range(len(tiles)):
+            yield from load_v(g)
+            yield "step"
+
     def qk_issuer():
         for g, (u, j, nkv) in enumerate(tiles):
             slot = u % cfg.qbuf
             if j == 0:
                 yield from wait(f"QF{slot}", (u // cfg.qbuf) & 1, u // cfg.qbuf)
-            s, buf = g % cfg.stk, g & 1
-            yield from wait(f"KF{s}", (g // cfg.stk) & 1, g // cfg.stk)
+            s_, buf = g % cfg.stk, g & 1
+            yield from wait(f"KF{s_}", (g // cfg.stk) & 1, g // cfg.stk)
             if g >= 2 and mutation != "no_sc_wait":
                 yield from wait(f"SC{buf}", ((g >> 1) - 1) & 1, (g >> 1) - 1)
             if g >= 2 and st["Sread"].get(buf, -1) < g - 2:
                 raise ProtocolError(f"S buffer {buf} overwritten by tile {g} before tile {g - 2} read it")
             fifos["qk"].append([rng.randint(5, 30), "qk", g])
-            fifos["qk"].append([0, "commit", [f"SF{buf}", f"KE{s}"] + ([f"QE{slot}"] if j == nkv - 1 else [])])
+            fifos["qk"].append([0, "commit", [f"SF{buf}", f"KE{s_}"] + ([f"QE{slot}"] if j == nkv - 1 else [])])
             yield "step"
 
     def pv_issuer():
         for g, (u, j, nkv) in enumerate(tiles):
-            s, buf = g % cfg.stv, g % cfg.npb
+            s_, buf = g % cfg.stv, g % cfg.npb
             if j == 0 and u > 0:
                 yield from wait("OF", (u - 1) & 1, u - 1)
-            yield from wait(f"OR{buf}", (g // cfg.npb) & 1, g // cfg.npb)
-            yield from wait(f"VF{s}", (g // cfg.stv) & 1, g // cfg.stv)
+            yield from wait(f"VF{s_}", (g // cfg.stv) & 1, g // cfg.stv)
+            yield from wait(f"PF{buf}", (g // cfg.npb) & 1, g // cfg.npb)
             if st["P"].get(buf) != g:
                 raise ProtocolError(f"P buffer {buf} holds tile {st['P'].get(buf)} at P V of tile {g}")
             if j == 0:
@@ -158,77 +171,82 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5):
                     raise ProtocolError(f"O still in use by unit {st['O_unit']} at unit {u}")
                 st["O_unit"] = u
             fifos["pv"].append([rng.randint(5, 30), "pv", g])
-            fifos["pv"].append([0, "commit", [f"VE{s}", f"PE{buf}"] + (["OFIN"] if j == nkv - 1 else [])])
+            fifos["pv"].append([0, "commit", [f"VE{s_}", f"PE{buf}"] + (["OFIN"] if j == nkv - 1 else [])])
             yield "step"
 
     def softmax_group(grp):
         for g, (u, j, nkv) in enumerate(tiles):
-            if (g & 1) != grp:
-                continue
-            buf = grp
-            yield from wait(f"SF{buf}", (g >> 1) & 1, g >> 1)
-            if g not in st["qk_done"]:
-                raise ProtocolError(f"S of tile {g} read before its MMA finished")
-            yield "pass1"
-            if g >= 1:
-                pb = (g - 1) & 1
-                yield from wait(f"MX{pb}", ((g - 1) >> 1) & 1, (g - 1) >> 1)
-                if st["xch"].get(pb) != g - 1:
-                    raise ProtocolError(f"reference max of tile {g - 1} overwritten before tile {g} read it")
-            st["xch"][grp] = g
-            bars[f"MX{grp}"].arrive(128)
-            pbuf = g % cfg.npb
-            back = 2 if mutation == "pe_wait_two_back" else cfg.npb
-            if g >= back:
-                yield from wait(f"PE{pbuf}", ((g - back) // cfg.npb) & 1, (g - back) // cfg.npb)
-            if g >= cfg.npb and (g - cfg.npb) not in st["pv_done"]:
-                raise ProtocolError(f"P buffer {pbuf} rewritten by tile {g} before P V of tile {g - cfg.npb}")
-            for _ in range(rng.randint(0, 3)):
-                yield "codes"
-            st["Sread"][buf] = g
-            bars[f"SC{buf}"].arrive(128)
-            for _ in range(rng.randint(0, 3)):
-                yield "codes"
-            if cfg.fp8 and j == nkv - 1:
-                st["lfin"][u % lfin_slots] = u       # the unit's final reference max
-            if not cfg.fp8 and j >= nkv - 2:
-                st["hand"][grp] = g                  # this group's partial row sum and its max
-            st["P"][pbuf] = g
-            slot = (g & 1) if mutation == "alpha_by_group" else pbuf
-            st["alpha"][slot] = g
-            bars[f"PF{pbuf}"].arrive(128)
-
-    def correction():
-        for g, (u, j, nkv) in enumerate(tiles):
-            pbuf = g % cfg.npb
-            yield from wait(f"PF{pbuf}", (g // cfg.npb) & 1, g // cfg.npb)
-            slot = (g & 1) if mutation == "alpha_by_group" else pbuf
-            if st["alpha"].get(slot) != g:
-                raise ProtocolError(f"rescale factor of tile {g} overwritten before the correction read it")
-            if not cfg.fp8 and j >= nkv - 2 and st["hand"].get(g & 1) != g:
-                raise ProtocolError(f"row-sum hand-over of tile {g} overwritten before the correction read it")
-            if j > 0 and rng.random() < p_rescale:
-                pg = g - 1
-                yield from wait(f"PE{pg % cfg.npb}", (pg // cfg.npb) & 1, pg // cfg.npb)
-                if pg not in st["pv_done"]:
-                    raise ProtocolError(f"O rescaled for tile {g} before P V of tile {pg} finished")
-                yield "rescale"
-            bars[f"OR{pbuf}"].arrive(128)
+            if (g & 1) == grp:
+                buf = grp
+                yield from wait(f"SF{buf}", (g >> 1) & 1, g >> 1)
+                if g not in st["qk_done"]:
+                    raise ProtocolError(f"S of tile {g} read before its MMA finished")
+                yield "load"
+                st["Sread"][buf] = g               # the whole row in registers: S released at once
+                bars[f"SC{buf}"].arrive(128)
+                yield "max"
+                if g >= 1:
+                    pb = (g - 1) & 1
+                    yield from wait(f"MX{pb}", ((g - 1) >> 1) & 1, (g - 1) >> 1)
+                    if st["xch"].get(pb) != g - 1:
+                        raise ProtocolError(f"reference max of tile {g - 1} overwritten before tile {g} read it")
+                st["xch"][grp] = g
+                bars[f"MX{grp}"].arrive(128)
+                pbuf = g % cfg.npb
+                back = 2 if mutation == "pe_wait_two_back" else cfg.npb
+                if g >= back:
+                    yield from wait(f"PE{pbuf}", ((g - back) // cfg.npb) & 1, (g - back) // cfg.npb)
+                if g >= cfg.npb and (g - cfg.npb) not in st["pv_done"]:
+                    raise ProtocolError(f"P buffer {pbuf} rewritten by tile {g} before P V of tile {g - cfg.npb}")
+                for _ in range(rng.randint(0, 4)):
+                    yield "codes"
+                st["P"][pbuf] = g
+                if j > 0 and rng.random() < p_rescale:
+                    # the reference max moved: O holds tiles 0 .. g-1 and is rescaled
+                    pg = g - 1
+                    if mutation != "no_rescale_wait":
+                        yield from wait(f"PE{pg % cfg.npb}", (pg // cfg.npb) & 1, pg // cfg.npb)
+                    if pg not in st["pv_done"]:
+                        raise ProtocolError(f"O rescaled for tile {g} before P V of tile {pg} finished")
+                    yield "rescale"
+                bars[f"PF{pbuf}"].arrive(128)
             if j == nkv - 1:
-                yield from wait("OFIN", u & 1, u)
-                if not all(t in st["pv_done"] for t in range(g - j, g + 1)):
-                    raise ProtocolError(f"epilogue of unit {u} before its last P V finished")
-                for _ in range(rng.randint(0, 3)):   # the row-sum load from TMEM comes first
-                    yield "epilogue"
-                if cfg.fp8 and st["lfin"].get(u % lfin_slots) != u:
-                    raise ProtocolError(f"final max of unit {u} overwritten before its epilogue read it")
-                for _ in range(rng.randint(1, 8)):
-                    yield "epilogue"
-                st["O_unit"] = "free"
-                bars["OF"].arrive(128)
+                # the unit's last tile: this group's hand-over to the epilogue
+                hs = u % cfg.hand
+                prev = st["hand"].get((hs, grp))
+                if prev is not None and prev != u and prev not in st.setdefault("hand_read", set()):
+                    raise ProtocolError(f"hand-over slot {hs} of unit {prev} overwritten by unit {u} before "
+                                        f"the epilogue read it")
+                st["hand"][(hs, grp)] = u
+                bars[f"LF{hs}"].arrive(128)
 
-    roles = {"producer": producer(), "qk": qk_issuer(), "pv": pv_issuer(), "softmax0": softmax_group(0),
-             "softmax1": softmax_group(1), "correction": correction()}
+    def epilogue():
+        g_end = 0
+        for u, nkv in enumerate(units):
+            g_end += nkv
+            yield from wait("OFIN", u & 1, u)
+            if not all(t in st["pv_done"] for t in range(g_end - nkv, g_end)):
+                raise ProtocolError(f"epilogue of unit {u} before its last P V finished")
+            hs = u % cfg.hand
+            yield from wait(f"LF{hs}", (u // cfg.hand) & 1, u // cfg.hand)
+            for grp in (0, 1):
+                if st["hand"].get((hs, grp)) != u:
+                    raise ProtocolError(f"hand-over of unit {u} (group {grp}) overwritten before the epilogue read it")
+            for _ in range(rng.randint(0, 3)):
+                yield "epilogue"
+            st.setdefault("hand_read", set()).add(u)
+            for _ in range(rng.randint(1, 8)):
+                yield "epilogue"
+            st["O_unit"] = "free"
+            bars["OF"].arrive(128)
+
+    roles = {"qk": qk_issuer(), "pv": pv_issuer(), "softmax0": softmax_group(0),
+             "softmax1": softmax_group(1), "epilogue": epilogue()}
+    if two_producers:
+        roles["producer_k"] = producer_k()
+        roles["producer_v"] = producer_v()
+    else:
+        roles["producer"] = producer()
     done, idle = set(), 0
     while len(done) < len(roles):
         progressed = False

@@ -70,11 +70,13 @@ def test_fp8_block_scales_engaged(q_gain, kind):
 
 
 def test_deferred_reference_max_on_growing_scores():
-    """Scores that jump by ~20 binades, then ~4 (deferred), fall, then ~8.2
-    above the stale reference (rescaled): FP8 against fp64 attention and the
-    CPU replay with the same deferral rule; BF16 on the same values."""
+    """Scores that jump past the kernel's deferral bound (64 binades: a
+    rescale), then ~33 binades above the reference (deferred: block shifts
+    below 0 and E8M0 scales above 1), fall, then ~78 above it (rescaled): FP8
+    against fp64 attention and the CPU replay with the same deferral rule;
+    BF16 on the same values."""
     from test_oracle_pins import _growing_score_case
-    qc, kc, vc, qs, ks, vs = _growing_score_case(21)
+    qc, kc, vc, qs, ks, vs = _growing_score_case(21, RESCALE_LOG2)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     o = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs))
     torch.cuda.synchronize()

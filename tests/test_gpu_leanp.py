@@ -60,3 +60,56 @@ def test_leanp_block_shift_cap_and_empty_block():
     _compare(s, m, bmax, A)
     bmax_inf = np.full(n, -np.inf, np.float32)
     _compare(np.full(n, -np.inf, np.float32), m, bmax_inf, A)
+
+
+def _deferred_case(rng, n, jt):
+    """Scores of blocks whose shift is jt: (m - bmax) A / 8 in [jt - 8 + 1/16, jt - 7 - 1/16].
+    jt < 8 puts the block max above the reference m (the deferred reference max)."""
+    m = rng.normal(0, 50, n).astype(np.float32)
+    A = np.exp(rng.uniform(np.log(1e-4), np.log(30), n)).astype(np.float32)
+    e = (8.0 * (jt - 8) + rng.uniform(0.5, 7.5, n)).astype(np.float32)   # (m - bmax) A
+    bmax = (m - e / A).astype(np.float32)
+    s = (bmax - np.abs(rng.normal(0, 40, n)).astype(np.float32) / A).astype(np.float32)
+    s[::17] = bmax[::17]                       # the block max itself
+    return s, m, bmax, A
+
+
+def test_leanp_deferred_reference_max_every_shift():
+    # every block shift j the kernel can produce, 0..126: byte-exact codes and
+    # shifts, the deferred regime (block max above m, j = 0..7) included
+    rng = np.random.default_rng(33)
+    parts = [_deferred_case(rng, 2048, jt) for jt in range(0, 126)]
+    s, m, bmax, A = (np.concatenate([p[i] for p in parts]) for i in range(4))
+    # the cap: blocks 118 or more binades under m
+    capm = rng.normal(0, 10, 4096).astype(np.float32)
+    capA = np.full(4096, 2.0, np.float32)
+    capb = (capm - rng.uniform(118.5 * 8 / 2.0, 2000, 4096).astype(np.float32)).astype(np.float32)
+    s = np.concatenate([s, capb]); m = np.concatenate([m, capm])
+    bmax = np.concatenate([bmax, capb]); A = np.concatenate([A, capA])
+    _compare(s, m, bmax, A)
+    _, j = orc.leanp_batch(s, m, bmax, A)
+    assert set(range(0, 127)) <= set(j.tolist())
+
+
+def test_leanp_deferred_limit_exact():
+    # (m - bmax) A = -64 exactly (8 binades above m, the most the kernel
+    # defers): j = 0 and the block max is code 120; just past it j = -1 (the
+    # kernel moves the reference before that happens; the functions still agree)
+    n = 2048
+    A = np.full(n, 1.0, np.float32)
+    m = np.full(n, 10.0, np.float32)
+    bmax = np.full(n, 74.0, np.float32)
+    s = np.linspace(-60.0, 74.0, n).astype(np.float32)
+    _compare(s, m, bmax, A)
+    code, j = orc.leanp_batch(s, m, bmax, A)
+    assert np.all(j == 0) and code[-1] == 120
+    bmax2 = np.full(n, 74.5, np.float32)
+    s2 = np.minimum(s, np.float32(74.5))
+    _compare(s2, m, bmax2, A)
+    # powers of two of A and m: every code 0..120 reached exactly on its integer
+    u = np.arange(0, 121, dtype=np.float32)
+    s3 = (u - np.float32(120.0) + np.float32(74.0)).astype(np.float32)
+    k = s3.size
+    c3, _ = orc.leanp_batch(s3, np.full(k, 10.0, np.float32), np.full(k, 74.0, np.float32), np.ones(k, np.float32))
+    assert np.array_equal(c3, u.astype(np.uint8))
+    _compare(s3, np.full(k, 10.0, np.float32), np.full(k, 74.0, np.float32), np.ones(k, np.float32))

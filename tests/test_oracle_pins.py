@@ -190,9 +190,13 @@ def test_gqa_single_kv_head_equals_replicated_mha():
 # --- Lean P ----------------------------------------------------------------------
 
 def test_leanp_zero_scores_give_8j_plus_56():
+    # s = m = 0: u = 56 + 8j exactly, so the code is 8j + 56 while that is a
+    # finite e4m3 code (j <= 8) and the clamp value 126 beyond
     for A in [1e-4, 0.37, 5.0]:
-        for j in [8, 9, 20, 126]:
-            assert orc.leanp_code(0.0, 0.0, A, j) == min(126, 8 * j + 56) or j > 8
+        for j in range(0, 9):
+            assert orc.leanp_code(0.0, 0.0, A, j) == 8 * j + 56
+        for j in [9, 20, 126]:
+            assert orc.leanp_code(0.0, 0.0, A, j) == 126
         assert orc.leanp_block_shift(0.0, 0.0, A) == 8
         assert orc.leanp_code(0.0, 0.0, A, 8) == 120
     assert orc.leanp_code(5.0, 5.0, 0.25, 8, masked=True) == 0
@@ -224,9 +228,10 @@ def test_leanp_weight_inside_mitchell_band():
     n = 20000
     m = rng.uniform(-30, 30, n).astype(np.float32)
     A = np.exp(rng.uniform(np.log(1e-3), np.log(20), n)).astype(np.float32)
-    gap = rng.uniform(0, 100, n).astype(np.float32)           # m - bmax, in units of A/8
+    # m - bmax in binades (units of 8/A).  Negative gaps are the deferred
+    # reference max: a block up to 8 binades above the reference m (j = 0..7)
+    gap = rng.uniform(-8, 100, n).astype(np.float32)
     bmax = (m - gap * np.float32(8.0) / A).astype(np.float32)
-    bmax = np.minimum(bmax, m)
     frac = rng.uniform(0, 1, n)
     s = (bmax - frac * np.float32(40.0) / A).astype(np.float32)   # up to 5 binades under bmax
     s = np.minimum(s, bmax)
@@ -242,15 +247,46 @@ def test_leanp_weight_inside_mitchell_band():
     # the block max lands in the top binade: u in (112, 120], so its code is
     # in [112, 120] (one lower where the fp32 steps round across an integer)
     cmax, _ = orc.leanp_batch(bmax, m, bmax, A)
-    cap = js < 126
+    cap = (js < 126) & (js >= 0)
     assert np.all((cmax[cap] >= 111) & (cmax[cap] <= 120))
     assert np.mean(cmax[cap] >= 112) > 0.99
+    # the deferred regime (block max above m) is exercised, with every j 0..7
+    above = bmax > m
+    assert above.mean() > 0.05
+    assert set(range(0, 8)) <= set(js[above].tolist())
+    assert np.all(js[above] <= 8)
+    assert np.all((cmax[above & cap] >= 111) & (cmax[above & cap] <= 120))
 
 
 def test_leanp_block_shift_cap():
     assert orc.leanp_block_shift(1e6, -1e6, 1.0) == 126
     assert orc.leanp_block_shift(10.0, 2.0, 1.0) == 9        # gap 8*1 -> floor(1) = 1
     assert orc.leanp_block_shift(10.0, 2.0001, 1.0) == 8
+
+
+def test_leanp_deferred_reference_max_boundaries():
+    # A block whose max lies above the reference m (the deferred reference max
+    # lets it be up to 8 binades, (bmax - m) A <= 64, above): j = 8 + floor of
+    # a negative number, rounded toward minus infinity, not toward zero
+    A = 1.0
+    assert orc.leanp_block_shift(10.0, 10.0, A) == 8          # on the reference
+    assert orc.leanp_block_shift(10.0, 10.5, A) == 7          # -0.0625 -> floor -1
+    assert orc.leanp_block_shift(10.0, 18.0, A) == 7          # -1 exactly
+    assert orc.leanp_block_shift(10.0, 18.5, A) == 6
+    assert orc.leanp_block_shift(10.0, 74.0, A) == 0          # (m - bmax) A = -64: the limit
+    assert orc.leanp_block_shift(10.0, 74.5, A) == -1         # past the limit (the kernel moves m first)
+    for jt in range(0, 8):
+        # (m - bmax) A = 8 (jt - 8) + 3: floor((...)/8) = jt - 8
+        bm = np.float32(10.0 - (8 * (jt - 8) + 3))
+        j = orc.leanp_block_shift(10.0, bm, A)
+        assert j == jt
+        # the block max lands in the top binade: u = 120 - 3 = 117
+        assert orc.leanp_code(bm, 10.0, A, j) == 117
+        # one binade under the block max: 8 codes lower
+        assert orc.leanp_code(bm - 8.0, 10.0, A, j) == 109
+    # at the limit the block max itself is code 120 with j = 0: weight 2^8 = 256
+    assert orc.leanp_code(74.0, 10.0, A, 0) == 120
+    assert orc.e4m3_values()[120] == 256.0
 
 
 # --- model oracle ----------------------------------------------------------------
@@ -271,16 +307,19 @@ def test_model_oracle_exact_p_equals_plain_definition():
     assert orc.rel_fro(o_model, o_ref) < 1e-6
 
 
-def _growing_score_case(seed):
+def _growing_score_case(seed, threshold=8.0):
     """Q = 1.0 everywhere, K rows near a per-tile level, so the score of key j
-    for every query is about 128 * level(tile of j): levels chosen so that the
-    tile max jumps by ~20 binades, then ~4 (below an 8-binade threshold),
-    falls, then ~8.2 above the deferred reference (scores in binades:
-    s * 8 log2(e) / sqrt(128) / 8)."""
+    for every query is about 128 * level(tile of j), about 16.3 level binades
+    (s * 8 log2(e) / sqrt(128) / 8), a little less for the tile max since K
+    entries take the level or the next lower code at random.  For an
+    8-binade deferral bound the tile max jumps by ~19 binades (rescaled), then
+    ~4 (deferred), falls, then ~11 above the deferred reference (rescaled);
+    for a 64-binade bound by ~70 binades (rescaled), then ~30 (deferred),
+    falls, then ~78 above the reference (rescaled)."""
     rng = np.random.default_rng(seed)
     vals = orc.e4m3_values()
     code_of = {float(vals[c]): c for c in range(0x00, 0x7F)}
-    levels = [0.5, 1.75, 2.0, 1.5, 2.25]
+    levels = {8.0: [0.5, 1.75, 2.0, 1.5, 2.5], 64.0: [0.5, 5.0, 7.0, 3.0, 10.0]}[threshold]
     S, D = 128 * len(levels), 128
     qc = np.full((1, S, 1, D), code_of[1.0], dtype=np.uint8)
     kc = np.empty((1, S, 1, D), dtype=np.uint8)
@@ -293,20 +332,32 @@ def _growing_score_case(seed):
     return qc, kc, vc, one, one, one
 
 
-def test_model_oracle_deferred_max_equals_plain_definition():
-    """With exact probabilities the deferred reference max (8 binades) must give
+@pytest.mark.parametrize("r", [8.0, 64.0])
+def test_model_oracle_deferred_max_equals_plain_definition(r):
+    """With exact probabilities the deferred reference max (r binades) must give
     the plain softmax: pins the deferral rule, its alpha and that O and l are
     rescaled together, on scores that grow far beyond the fp32 exp2 range."""
-    qc, kc, vc, qs, ks, vs = _growing_score_case(21)
+    qc, kc, vc, qs, ks, vs = _growing_score_case(21, r)
     deq = tuple(orc.dequantize(x, sc) for x, sc in ((qc, qs), (kc, ks), (vc, vs)))
     ref = orc.attention(*deq)
-    o_lazy = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True, rescale_log2=8.0)
+    o_lazy = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True, rescale_log2=r)
     assert orc.rel_fro(o_lazy, ref) < 1e-6
     # the deferral changes the Lean-P codes (the reference moves), not the bar
     o_exact = orc.fp8_model(qc, kc, vc, qs, ks, vs)
-    o_def = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=8.0)
+    o_def = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=r)
     assert not np.array_equal(o_exact, o_def)
     assert orc.rel_fro(o_def, ref) < 3e-2 and orc.rel_fro(o_exact, ref) < 3e-2
+    # the case exercises what it is meant to: tile maxima (in binades) that jump
+    # past the bound (a rescale), stay within it above the reference (deferred,
+    # block shifts below 8), fall, and pass the bound again
+    A8 = float(orc.leanp_slope(1.0, 1.0, 128)) / 8.0
+    qv = orc.e4m3_values()[qc[0, 0, 0]].astype(np.float64)
+    tmax = [float((orc.e4m3_values()[kc[0, 128 * t:128 * t + 128, 0]].astype(np.float64) @ qv).max()) * A8
+            for t in range(5)]
+    assert tmax[1] - tmax[0] > r                     # moves the reference
+    assert 0 < tmax[2] - tmax[1] <= r                # deferred: block above the reference
+    assert tmax[3] < tmax[1]
+    assert tmax[4] - tmax[1] > r                     # moves it again
 
 
 def test_model_oracle_zero_q_gives_prefix_means():
