@@ -203,6 +203,13 @@ int launch_attn_varlen(const void* q, const void* k, const void* v, void* o, con
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
+// Sequence rows per prepass CTA: at most 2^30 elements of one batch entry
+// (the kernels count a chunk's rows and 16-byte vectors in 32 bits).
+long long prepass_rows(long long rows, int H, int D) {
+  const long long cap = std::max(1ll, (1ll << 30) / (static_cast<long long>(H) * D));
+  return std::max(1ll, std::min(rows, cap));
+}
+
 // ---------------------------------------------------------------- test kernels
 
 // Element pairs (i, i + 1) go through leanp_word2, the packed step the attention
@@ -355,7 +362,7 @@ extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* sc
   a.out = static_cast<uint8_t*>(x_fp8);
   a.scale = scale;
   a.S = S; a.H = H; a.D = D;
-  a.rows_per_cta = static_cast<int>((S + chunks - 1) / chunks);
+  a.rows_per_cta = static_cast<int>(prepass_rows((S + chunks - 1) / chunks, H, D));
   const dim3 grid(static_cast<unsigned>((S + a.rows_per_cta - 1) / a.rows_per_cta), static_cast<unsigned>(B));
   const size_t shm = static_cast<size_t>(H) * 8;   // amax, or scale and its reciprocal, per head
   if (cudaMemsetAsync(scale, 0, static_cast<size_t>(B) * H * sizeof(float), st) != cudaSuccess)
@@ -421,9 +428,11 @@ extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, in
     t.out = static_cast<uint8_t*>(outs[i]);
     t.scale = scs[i];
     t.S = S; t.H = Hs[i]; t.D = Ds[i];
-    t.rows_per_cta = static_cast<int>((S + chunks - 1) / chunks);
+    t.rows_per_cta = static_cast<int>(prepass_rows((S + chunks - 1) / chunks, Hs[i], Ds[i]));
     a.had[i] = (i < 2) ? hadamard_qk : 0;
-    a.first[i + 1] = a.first[i] + (S + t.rows_per_cta - 1) / t.rows_per_cta;
+    const long long cols = a.first[i] + (static_cast<long long>(S) + t.rows_per_cta - 1) / t.rows_per_cta;
+    if (cols > 0x7fffffffll) return ZYFA_ERR_BAD_SHAPE;
+    a.first[i + 1] = static_cast<int>(cols);
     if (Hs[i] > max_h) max_h = Hs[i];
   }
   const dim3 grid(static_cast<unsigned>(a.first[3]), static_cast<unsigned>(B));
@@ -530,7 +539,7 @@ static int quantize_varlen_n(int n, const void* const* xs, void* const* outs, fl
     t.scale = scs[i];
     t.S = 0;
     t.H = Hs[i]; t.D = Ds[i];
-    t.rows_per_cta = static_cast<int>((mean_len + chunks - 1) / chunks);
+    t.rows_per_cta = static_cast<int>(prepass_rows((mean_len + chunks - 1) / chunks, Hs[i], Ds[i]));
     q3.had[i] = had[i];
     long long cols = 0;   // every sequence's chunks, in order
     for (int sq = 0; sq < nseq; ++sq) cols += (cu[sq + 1] - cu[sq] + t.rows_per_cta - 1) / t.rows_per_cta;

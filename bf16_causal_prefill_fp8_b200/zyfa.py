@@ -102,6 +102,101 @@ def _ptr(t):
 def _dev(t, name):
     if not (t.is_cuda and t.is_contiguous()):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()} (the library launches there)")
+
+
+# --- argument checks ----------------------------------------------------------
+# Shapes, dtypes and devices of every tensor a call passes, checked before the
+# library sees a pointer: a wrong extent would let a copy or a store run past
+# an allocation.  They take any tensor-like object (the CPU tests pass meta
+# tensors); _dev() adds the CUDA and current-device checks at call time.
+
+FP8_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _want(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _same_device(ref, named):
+    for t, n in named:
+        if t is not None and not isinstance(t, bool):
+            _want(t.device == ref.device, f"{n} is on {t.device}, q on {ref.device}")
+
+
+def _scale_check(t, n, count):
+    if t is not None:
+        _want(t.dtype == torch.float32, f"{n} must be fp32")
+        _want(t.numel() == count, f"{n} holds {t.numel()} values, expected {count} (one per batch entry and head)")
+
+
+def check_attn_args(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, lse=None):
+    """attn_fwd's tensors: q [B,S,Hq,Dqk], k [B,S,Hkv,Dqk], v [B,S,Hkv,Dv] of one
+    dtype; o bf16 [B,S,Hq,Dv]; lse fp32 [B,Hq,S]; scales fp32 with B*H values;
+    all on q's device.  Returns (B, S, Hq, Hkv, Dqk, Dv, dtype code)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _want(t.dim() == 4, f"{n} must be 4-D [B, S, H, D], got {tuple(t.shape)}")
+    B, S, Hq, Dqk = q.shape
+    Hkv, Dv = k.shape[2], v.shape[3]
+    _want(tuple(k.shape) == (B, S, Hkv, Dqk), f"k is {tuple(k.shape)}, expected (B, S, Hkv, Dqk) = {(B, S, Hkv, Dqk)}")
+    _want(tuple(v.shape[:3]) == (B, S, Hkv), f"v is {tuple(v.shape)}, expected (B, S, Hkv, Dv) with {(B, S, Hkv)}")
+    _want(q.dtype == k.dtype == v.dtype, f"q, k, v dtypes differ: {q.dtype}, {k.dtype}, {v.dtype}")
+    if q.dtype == torch.bfloat16:
+        dt = BF16
+    elif q.dtype in FP8_DTYPES:
+        dt = FP8_E4M3
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    if o is not None:
+        _want(o.dtype == torch.bfloat16 and tuple(o.shape) == (B, S, Hq, Dv),
+              f"o must be bf16 [B, S, Hq, Dv] = {(B, S, Hq, Dv)}, got {o.dtype} {tuple(o.shape)}")
+    if lse is not None and not isinstance(lse, bool):
+        _want(lse.dtype == torch.float32 and tuple(lse.shape) == (B, Hq, S),
+              f"lse must be fp32 [B, Hq, S] = {(B, Hq, S)}, got {lse.dtype} {tuple(lse.shape)}")
+    for t, n, c in ((q_scale, "q_scale", B * Hq), (k_scale, "k_scale", B * Hkv), (v_scale, "v_scale", B * Hkv)):
+        _scale_check(t, n, c)
+    _same_device(q, ((k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (q_scale, "q_scale"), (k_scale, "k_scale"),
+                     (v_scale, "v_scale")))
+    return B, S, Hq, Hkv, Dqk, Dv, dt
+
+
+def check_quantize_args(x, out=None, scale=None, rows_first=False):
+    """quantize's tensors: x bf16 / fp32 [B,S,H,D] (or packed [T,H,D] with
+    rows_first), out uint8 / e4m3 of x's shape, scale fp32 (its count is
+    checked by the caller, which knows B or the sequence count)."""
+    _want(x.dim() == (3 if rows_first else 4), f"x has {x.dim()} dimensions")
+    _want(x.dtype in (torch.bfloat16, torch.float32), f"unsupported input dtype {x.dtype}")
+    if out is not None:
+        _want(tuple(out.shape) == tuple(x.shape) and out.dtype in FP8_DTYPES,
+              f"out must be uint8 / float8_e4m3fn of x's shape {tuple(x.shape)}, got {out.dtype} {tuple(out.shape)}")
+    if scale is not None:
+        _want(scale.dtype == torch.float32, "scale must be fp32")
+    _same_device(x, ((out, "out"), (scale, "scale")))
+
+
+def check_varlen_args(q, k, v, T, nseq, o=None, q_scale=None, k_scale=None, v_scale=None, lse=None):
+    """attn_fwd_varlen's tensors: packed q [T,Hq,Dqk], k [T,Hkv,Dqk], v [T,Hkv,Dv]
+    of one dtype; o bf16 [T,Hq,Dv]; lse fp32 [Hq,T]; scales fp32 with nseq*H
+    values; all on q's device."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _want(t.dim() == 3, f"{n} must be 3-D [T, H, D], got {tuple(t.shape)}")
+        _want(t.shape[0] == T, f"{n} holds {t.shape[0]} rows, cu_seqlens[-1] = {T}")
+    _, Hq, Dqk = q.shape
+    Hkv, Dv = k.shape[1], v.shape[2]
+    _want(k.shape[2] == Dqk and v.shape[1] == Hkv, f"k {tuple(k.shape)} / v {tuple(v.shape)} do not match q {tuple(q.shape)}")
+    _want(q.dtype == k.dtype == v.dtype, f"q, k, v dtypes differ: {q.dtype}, {k.dtype}, {v.dtype}")
+    if o is not None:
+        _want(o.dtype == torch.bfloat16 and tuple(o.shape) == (T, Hq, Dv),
+              f"o must be bf16 [T, Hq, Dv] = {(T, Hq, Dv)}, got {o.dtype} {tuple(o.shape)}")
+    if lse is not None and not isinstance(lse, bool):
+        _want(lse.dtype == torch.float32 and tuple(lse.shape) == (Hq, T), f"lse must be fp32 [Hq, T] = {(Hq, T)}")
+    for t, n, c in ((q_scale, "q_scale", nseq * Hq), (k_scale, "k_scale", nseq * Hkv), (v_scale, "v_scale", nseq * Hkv)):
+        _scale_check(t, n, c)
+    _same_device(q, ((k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (q_scale, "q_scale"), (k_scale, "k_scale"),
+                     (v_scale, "v_scale")))
 
 
 def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=None, exact_p=False, lse=False):
@@ -111,24 +206,15 @@ def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=N
     (zyfa_attn_fwd_fp8_exact_p) instead of Lean P.  Returns o [B,S,Hq,Dv] bf16;
     with lse=True (or an fp32 [B,Hq,S] tensor) returns (o, lse) through
     zyfa_attn_fwd_lse."""
+    B, S, Hq, Hkv, Dqk, Dv, dt = check_attn_args(q, k, v, o, q_scale, k_scale, v_scale, lse)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
-    if q.dtype == torch.bfloat16:
-        dt = BF16
-    elif q.dtype in (torch.uint8, torch.float8_e4m3fn):
-        dt = FP8_E4M3
-    else:
-        raise ValueError(f"unsupported dtype {q.dtype}")
-    B, S, Hq, Dqk = q.shape
-    Hkv, Dv = k.shape[2], v.shape[3]
     if o is None:
         o = torch.empty((B, S, Hq, Dv), dtype=torch.bfloat16, device=q.device)
     _dev(o, "o")
     for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
         if t is not None:
             _dev(t, n)
-            if t.dtype != torch.float32:
-                raise ValueError(f"{n} must be fp32")
     if lse is not False and lse is not None:
         if exact_p:
             raise ValueError("lse is not produced by the exact-P ablation")
@@ -153,18 +239,15 @@ def attn_fwd(q, k, v, o=None, q_scale=None, k_scale=None, v_scale=None, stream=N
 
 def quantize(x, hadamard=False, out=None, scale=None, stream=None):
     """x [B,S,H,D] bf16 or fp32 -> (codes uint8 [B,S,H,D], scale fp32 [B,H])."""
+    check_quantize_args(x, out, scale)
     _dev(x, "x")
-    if x.dtype == torch.bfloat16:
-        dt = BF16
-    elif x.dtype == torch.float32:
-        dt = FP32
-    else:
-        raise ValueError(f"unsupported input dtype {x.dtype}")
+    dt = BF16 if x.dtype == torch.bfloat16 else FP32
     B, S, H, D = x.shape
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scale is None:
         scale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    _scale_check(scale, "scale", B * H)
     _dev(out, "out"); _dev(scale, "scale")
     st = lib().zyfa_quantize(_ptr(x), dt, _ptr(out), _ptr(scale), B, S, H, D, int(bool(hadamard)),
                              _stream(stream))
@@ -177,21 +260,22 @@ def quantize_qkv(q, k, v, hadamard_qk=False, out=None, stream=None):
     identical to three quantize() calls (Hadamard on Q and K only), in four launches.  `out`: optional
     ((q8, qs), (k8, ks), (v8, vs)) to write into."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        check_quantize_args(t)
+    _want(q.dtype == k.dtype == v.dtype, "q, k and v must share a dtype")
+    _want(k.shape[:2] == q.shape[:2] and v.shape[:3] == k.shape[:3] and k.shape[3] == q.shape[3],
+          f"q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)} do not form one problem")
+    _same_device(q, ((k, "k"), (v, "v")))
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
-    if not (q.dtype == k.dtype == v.dtype):
-        raise ValueError("q, k and v must share a dtype")
-    if q.dtype == torch.bfloat16:
-        dt = BF16
-    elif q.dtype == torch.float32:
-        dt = FP32
-    else:
-        raise ValueError(f"unsupported input dtype {q.dtype}")
+    dt = BF16 if q.dtype == torch.bfloat16 else FP32
     B, S, Hq, Dqk = q.shape
     Hkv, Dv = k.shape[2], v.shape[3]
     if out is None:
         out = tuple((torch.empty(t.shape, dtype=torch.uint8, device=t.device),
                      torch.empty((B, t.shape[2]), dtype=torch.float32, device=t.device)) for t in (q, k, v))
-    for (c, sc), n in zip(out, "qkv"):
+    for (c, sc), x, n in zip(out, (q, k, v), "qkv"):
+        check_quantize_args(x, c, sc)
+        _scale_check(sc, n + "_scale", B * x.shape[2])
         _dev(c, n + "_fp8"); _dev(sc, n + "_scale")
     (q8, qs), (k8, ks), (v8, vs) = out
     st = lib().zyfa_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs), _ptr(ks),
@@ -221,36 +305,29 @@ def attn_fwd_varlen(q, k, v, cu_seqlens, o=None, q_scale=None, k_scale=None, v_s
     v [T,Hkv,Dv] with sequence s at rows cu_seqlens[s] .. cu_seqlens[s+1]-1; bf16, or e4m3 codes
     with fp32 scales [nseq,H].  Returns o [T,Hq,Dv] bf16, or (o, lse [Hq,T] fp32) with lse=True
     (or an fp32 [Hq,T] tensor)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _dev(t, n)
     if q.dtype == torch.bfloat16:
         dt = BF16
-    elif q.dtype in (torch.uint8, torch.float8_e4m3fn):
+    elif q.dtype in FP8_DTYPES:
         dt = FP8_E4M3
     else:
         raise ValueError(f"unsupported dtype {q.dtype}")
-    T, Hq, Dqk = q.shape
-    Hkv, Dv = k.shape[1], v.shape[2]
-    for t, n in ((k, "k"), (v, "v")):
-        if t.shape[0] != T:
-            raise ValueError(f"{n} holds {t.shape[0]} rows, q holds {T}")
+    T = q.shape[0]
     cu, nseq = _cu_host(cu_seqlens, T)
+    check_varlen_args(q, k, v, T, nseq, o, q_scale, k_scale, v_scale, lse)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    _, Hq, Dqk = q.shape
+    Hkv, Dv = k.shape[1], v.shape[2]
     if o is None:
         o = torch.empty((T, Hq, Dv), dtype=torch.bfloat16, device=q.device)
-    if o.shape[0] != T:
-        raise ValueError(f"o holds {o.shape[0]} rows, q holds {T}")
     _dev(o, "o")
     for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
         if t is not None:
             _dev(t, n)
-            if t.dtype != torch.float32:
-                raise ValueError(f"{n} must be fp32")
     out = None
     if lse is not False and lse is not None:
         out = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if lse is True else lse
         _dev(out, "lse")
-        if tuple(out.shape) != (Hq, T):
-            raise ValueError("lse must be [Hq, T]")
     st = lib().zyfa_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(out), cu, nseq, Hq, Hkv, Dqk, Dv,
                                     dt, _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _stream(stream))
     _check(st, "zyfa_attn_fwd_varlen")
@@ -267,6 +344,7 @@ def _in_dtype(x):
 
 def quantize_varlen(x, cu_seqlens, hadamard=False, out=None, scale=None, stream=None):
     """x [T,H,D] bf16 or fp32, packed -> (codes uint8 [T,H,D], scale fp32 [nseq,H])."""
+    check_quantize_args(x, out, scale, rows_first=True)
     _dev(x, "x")
     dt = _in_dtype(x)
     T, H, D = x.shape
@@ -275,6 +353,7 @@ def quantize_varlen(x, cu_seqlens, hadamard=False, out=None, scale=None, stream=
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scale is None:
         scale = torch.empty((nseq, H), dtype=torch.float32, device=x.device)
+    _scale_check(scale, "scale", nseq * H)
     _dev(out, "out"); _dev(scale, "scale")
     st = lib().zyfa_quantize_varlen(_ptr(x), dt, _ptr(out), _ptr(scale), cu, nseq, H, D, int(bool(hadamard)),
                                     _stream(stream))
@@ -285,21 +364,25 @@ def quantize_varlen(x, cu_seqlens, hadamard=False, out=None, scale=None, stream=
 def quantize_qkv_varlen(q, k, v, cu_seqlens, hadamard_qk=False, out=None, stream=None):
     """Packed Q, K, V [T,H,D] (same dtype) -> ((q8, q_scale), (k8, k_scale), (v8, v_scale)), scales
     [nseq,H]; identical to three quantize_varlen() calls, in four launches."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _dev(t, n)
-    if not (q.dtype == k.dtype == v.dtype):
-        raise ValueError("q, k and v must share a dtype")
+    for t in (q, k, v):
+        check_quantize_args(t, rows_first=True)
+    _want(q.dtype == k.dtype == v.dtype, "q, k and v must share a dtype")
     dt = _in_dtype(q)
     T, Hq, Dqk = q.shape
     Hkv, Dv = k.shape[1], v.shape[2]
     for t, n in ((k, "k"), (v, "v")):
         if t.shape[0] != T:
             raise ValueError(f"{n} holds {t.shape[0]} rows, q holds {T}")
+    _same_device(q, ((k, "k"), (v, "v")))
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
     cu, nseq = _cu_host(cu_seqlens, T)
     if out is None:
         out = tuple((torch.empty(t.shape, dtype=torch.uint8, device=t.device),
                      torch.empty((nseq, t.shape[1]), dtype=torch.float32, device=t.device)) for t in (q, k, v))
-    for (c, sc), n in zip(out, "qkv"):
+    for (c, sc), x, n in zip(out, (q, k, v), "qkv"):
+        check_quantize_args(x, c, sc, rows_first=True)
+        _scale_check(sc, n + "_scale", nseq * x.shape[1])
         _dev(c, n + "_fp8"); _dev(sc, n + "_scale")
     (q8, qs), (k8, ks), (v8, vs) = out
     st = lib().zyfa_quantize_qkv_varlen(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),

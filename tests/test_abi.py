@@ -224,3 +224,74 @@ def test_checked_build_exports_the_same_symbols():
     Lc.zyfa_checked_build.restype = ctypes.c_int
     assert Lc.zyfa_checked_build() == 1
     assert zyfa.lib().zyfa_checked_build() == 0
+
+
+# --- the binding's argument checks (meta tensors: shapes, dtypes and devices only)
+
+def _meta(shape, dtype=None):
+    import torch
+    return torch.empty(shape, dtype=dtype or torch.bfloat16, device="meta")
+
+
+def test_binding_rejects_mismatched_attention_tensors():
+    import torch
+    q, k, v = _meta((2, 256, 4, 128)), _meta((2, 256, 2, 128)), _meta((2, 256, 2, 128))
+    assert zyfa.check_attn_args(q, k, v) == (2, 256, 4, 2, 128, 128, zyfa.BF16)
+    u8 = lambda *s: _meta(s, torch.uint8)
+    f32 = lambda *s: _meta(s, torch.float32)
+    assert zyfa.check_attn_args(u8(2, 256, 4, 192), u8(2, 256, 2, 192), u8(2, 256, 2, 128),
+                                q_scale=f32(2, 4), k_scale=f32(4), v_scale=f32(2, 2))[6] == zyfa.FP8_E4M3
+    bad = [dict(k=_meta((2, 255, 2, 128))),                 # S differs
+           dict(k=_meta((1, 256, 2, 128))),                 # B differs
+           dict(k=_meta((2, 256, 2, 64))),                  # Dqk differs
+           dict(v=_meta((2, 256, 3, 128))),                 # Hkv differs
+           dict(v=_meta((2, 256, 2, 128), torch.float32)),  # dtype differs
+           dict(q=_meta((2, 256, 4, 128), torch.float16), k=_meta((2, 256, 2, 128), torch.float16),
+                v=_meta((2, 256, 2, 128), torch.float16)),  # unsupported dtype
+           dict(k=_meta((2, 256, 128))),                    # not 4-D
+           dict(o=_meta((2, 256, 4, 64))),                  # o shape
+           dict(o=_meta((2, 256, 4, 128), torch.float32)),  # o dtype
+           dict(lse=f32(2, 4, 255)), dict(lse=_meta((2, 4, 256))),
+           dict(q_scale=f32(3)), dict(k_scale=f32(2, 4)), dict(v_scale=_meta((4,)))]
+    for case in bad:
+        args = dict(q=q, k=k, v=v)
+        args.update(case)
+        with pytest.raises(ValueError):
+            zyfa.check_attn_args(**args)
+    # every tensor on q's device
+    with pytest.raises(ValueError):
+        zyfa.check_attn_args(q, k, torch.empty((2, 256, 2, 128), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        zyfa.check_attn_args(q, k, v, o=torch.empty((2, 256, 4, 128), dtype=torch.bfloat16))
+
+
+def test_binding_rejects_mismatched_prepass_and_packed_tensors():
+    import torch
+    x = _meta((1, 128, 8, 128))
+    zyfa.check_quantize_args(x, _meta((1, 128, 8, 128), torch.uint8), _meta((1, 8), torch.float32))
+    for out, scale in ((_meta((1, 128, 8, 64), torch.uint8), None), (_meta((1, 128, 8, 128)), None),
+                       (None, _meta((8,)))):
+        with pytest.raises(ValueError):
+            zyfa.check_quantize_args(x, out, scale)
+    with pytest.raises(ValueError):
+        zyfa.check_quantize_args(_meta((1, 128, 8, 128), torch.float16))
+    with pytest.raises(ValueError):
+        zyfa._scale_check(_meta((7,), torch.float32), "scale", 8)
+    q, k, v = _meta((300, 4, 128)), _meta((300, 2, 128)), _meta((300, 2, 128))
+    zyfa.check_varlen_args(q, k, v, 300, 3, o=_meta((300, 4, 128)), lse=_meta((4, 300), torch.float32))
+    for case in (dict(T=299), dict(k=_meta((300, 2, 64))), dict(v=_meta((300, 3, 128))),
+                 dict(o=_meta((300, 4, 64))), dict(lse=_meta((300, 4), torch.float32)),
+                 dict(q_scale=_meta((4,), torch.float32))):
+        args = dict(q=q, k=k, v=v, T=300, nseq=3)
+        args.update(case)
+        with pytest.raises(ValueError):
+            zyfa.check_varlen_args(**args)
+
+
+def test_binding_refuses_host_tensors_before_any_launch():
+    import torch
+    q = torch.zeros((1, 128, 2, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        zyfa.attn_fwd(q, q, q)
+    with pytest.raises(ValueError):
+        zyfa.quantize(q)
