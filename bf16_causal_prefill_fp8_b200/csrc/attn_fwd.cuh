@@ -66,12 +66,15 @@ struct AttnArgs {
 
 constexpr int kAttnThreads = 512;
 // Register split (setmaxnreg; the launch holds 512 x 128 = 65536 registers,
-// the whole register file, and the four shares below add up to it):
-// softmax warpgroups hold a 128-key row of S plus its codes, the epilogue
-// warpgroup one 32-column slice of O, the producer / issuer warpgroup only
-// loop state.
+// the whole register file, and the four shares below add up to it; zyfa.cu
+// checks the compiled count before the first launch, since a raise that asks
+// for more than the launch holds would wait forever): softmax warpgroups
+// hold a 128-key row of S plus its codes, the epilogue warpgroup one
+// 32-column slice of O, the producer / issuer warpgroup only loop state.
 constexpr uint32_t kRegSoftmax = 192, kRegEpilogue = 80, kRegControl = 48;
-static_assert(128 * (2 * kRegSoftmax + kRegEpilogue + kRegControl) == 65536, "register split");
+constexpr int kLaunchRegs = 128;
+static_assert(128 * (2 * kRegSoftmax + kRegEpilogue + kRegControl) == kAttnThreads * kLaunchRegs,
+              "register split");
 // Deferred reference max (both paths): the max that the probabilities are
 // taken against moves only when a tile's max exceeds it by more than this
 // many binades (FlashAttention-4's lazy rescale, with a far larger bound).

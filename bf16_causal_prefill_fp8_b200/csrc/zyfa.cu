@@ -157,6 +157,13 @@ bool prepare_device(int dev, int inst) {
   if (di.sms == 0 && cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return false;
   if (!di.attr_set[inst]) {
+    // the warpgroups' setmaxnreg shares must add up to what the launch holds:
+    // a raise asking for more than that would wait forever, so a build whose
+    // register count differs is refused here, before any launch
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<FP8, DQK, EXACTP, VARLEN>) != cudaSuccess ||
+        fa.numRegs != kLaunchRegs)
+      return false;
     if (cudaFuncSetAttribute(attn_fwd_kernel<FP8, DQK, EXACTP, VARLEN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM) != cudaSuccess)
       return false;
