@@ -11,8 +11,8 @@ import torch
 from bf16_causal_prefill_fp8_b200 import zyfa
 from oracle import oracle as orc
 
-from helpers import (RESCALE_LOG2, TOL_BF16, TOL_FP8, TOL_FP8_MODEL, bf16_round, fp8_references, inputs,
-                     run_bf16, run_fp8)
+from helpers import (RESCALE_LOG2, ROW_TOL_BF16, ROW_TOL_FP8, ROW_TOL_FP8_MODEL, TOL_BF16, TOL_FP8, TOL_FP8_MODEL,
+                     bf16_round, check_local, fp8_references, inputs, run_bf16, run_fp8)
 
 pytestmark = pytest.mark.gpu
 
@@ -108,6 +108,8 @@ def test_many_units_per_cta(kind, q_gain):
     e_ref, e_model = orc.rel_fro(o[:, rows], ref), orc.rel_fro(o[:, rows], model)
     print(f"many units fp8 {kind} gain={q_gain}: vs fp64 {e_ref:.3e}  vs model {e_model:.3e}")
     assert e_ref <= TOL_FP8 and e_model <= TOL_FP8_MODEL
+    check_local(o[:, rows], ref, TOL_FP8, ROW_TOL_FP8, f"many units fp8 {kind} vs fp64", rows)
+    check_local(o[:, rows], model, TOL_FP8_MODEL, ROW_TOL_FP8_MODEL, f"many units fp8 {kind} vs model", rows)
     (qc, qs), (kc, ks), (vc, vs) = codes
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     o2 = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs))
@@ -118,6 +120,7 @@ def test_many_units_per_cta(kind, q_gain):
     e_b = orc.rel_fro(ob[:, rows], refb)
     print(f"many units bf16 {kind} gain={q_gain}: vs fp64 {e_b:.3e}")
     assert e_b <= TOL_BF16
+    check_local(ob[:, rows], refb, TOL_BF16, ROW_TOL_BF16, f"many units bf16 {kind} vs fp64", rows)
     ob2, _ = run_bf16(q, k, v)
     assert np.array_equal(ob2, ob)
 
