@@ -367,14 +367,16 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 
 /* ------------------------------------------------------------------------ */
 /* Model oracle: the FP8 pipeline in the pages' order, in fp64 except the   */
-/* Lean-P decisions (fp32, above).  Per query row i, KV tiles of 128 keys   */
-/* are visited in ascending order (tiles 0 .. i/128); each tile is two      */
-/* 64-key blocks.  For tile t:                                              */
+/* Lean-P decisions (fp32, above).  Per query row i, KV tiles of kv_tile    */
+/* keys (128 or 256: the tile a kernel processes at a time, which is where  */
+/* the deferred reference max is decided) are visited in ascending order    */
+/* (tiles 0 .. i/kv_tile); each tile is kv_tile/64 blocks of 64 keys.       */
+/* For tile t:                                                              */
 /*   s_j   = fl32(sum_d value(qcode) * value(kcode))   keys j <= i, j < S    */
 /*   bmax  = max s_j over each block (-inf if the block has no live key)    */
-/*   m'    = max(m, bmax_0, bmax_1)          running max after this tile    */
+/*   m'    = max(m, bmax_0, bmax_1, ..)      running max after this tile    */
 /*           (rescale_log2 > 0: reference max instead -- m' = tile max on    */
-/*           tile 0; later m' = max(bmax_0, bmax_1) only when               */
+/*           tile 0; later m' = max(bmax_0, bmax_1, ..) only when           */
 /*           fl32(fl32(that - m) * A) > 8 rescale_log2, i.e. when the tile  */
 /*           max is more than rescale_log2 binades above m, else m' = m.    */
 /*           The softmax is unchanged: O and l share the reference and the */
@@ -396,11 +398,13 @@ void oracle_leanp_batch(const float *s, const float *m, const float *bmax,
 int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *vc,
                           const float *q_s, const float *k_s, const float *v_s,
                           int B, int Hq, int Hkv, int S, int Dqk, int Dv,
-                          int p_mode, float rescale_log2,
+                          int p_mode, float rescale_log2, int kv_tile,
                           const int *rows, int nrows, double *o, double *lse)
 {
     int b, shift_err = 0;
+    const int nblk = kv_tile / 64;
     if (!qc || !kc || !vc || !q_s || !k_s || !v_s || !o) return -1;
+    if (kv_tile != 128 && kv_tile != 256) return -1;
     if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Hq % Hkv != 0 || Dqk < 1 || Dv < 1) return -1;
     if (!rows) nrows = S;
     for (b = 0; b < B; ++b) {
@@ -413,19 +417,19 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
             float A = oracle_leanp_slope(q_s[(size_t)b * Hq + hq], k_s[(size_t)b * Hkv + kvh], Dqk);
             double *qv = (double *)malloc(sizeof(double) * (size_t)Dqk);
             double *acc = (double *)calloc((size_t)Dv, sizeof(double));
-            float sj[128];
-            int live[128];
+            float sj[256];
+            int live[256];
             double l = 0.0;
             float m = -INFINITY;
             int t, d, n;
             for (d = 0; d < Dqk; ++d)
                 qv[d] = oracle_e4m3_value(qc[(((size_t)b * S + i) * Hq + hq) * (size_t)Dqk + d]);
-            for (t = 0; t <= i / 128; ++t) {
-                float bmax[2] = {-INFINITY, -INFINITY};
-                float mnew;
+            for (t = 0; t <= i / kv_tile; ++t) {
+                float bmax[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                float mnew, tmax;
                 double alpha;
-                for (n = 0; n < 128; ++n) {
-                    int j = 128 * t + n;
+                for (n = 0; n < kv_tile; ++n) {
+                    int j = kv_tile * t + n;
                     live[n] = (j <= i && j < S);
                     sj[n] = -INFINITY;
                     if (live[n]) {
@@ -436,8 +440,10 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
                         if (sj[n] > bmax[n / 64]) bmax[n / 64] = sj[n];
                     }
                 }
+                tmax = bmax[0];
+                for (n = 1; n < nblk; ++n)
+                    if (bmax[n] > tmax) tmax = bmax[n];
                 if (rescale_log2 > 0.0f) {
-                    float tmax = bmax[0] > bmax[1] ? bmax[0] : bmax[1];
                     float grow;
                     if (t == 0) {
                         mnew = tmax;
@@ -447,11 +453,9 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
                         mnew = (grow > 8.0f * rescale_log2) ? tmax : m;
                     }
                 } else {
-                    mnew = m;
-                    if (bmax[0] > mnew) mnew = bmax[0];
-                    if (bmax[1] > mnew) mnew = bmax[1];
+                    mnew = tmax > m ? tmax : m;
                 }
-                for (n = 0; n < 2; ++n)
+                for (n = 0; n < nblk; ++n)
                     if (oracle_leanp_block_shift(mnew, bmax[n], A) <
                         (rescale_log2 > 0.0f ? 8 - (int)ceilf(rescale_log2) : 8)) {
 #pragma omp atomic write
@@ -460,8 +464,8 @@ int oracle_fp8_model_rows(const uint8_t *qc, const uint8_t *kc, const uint8_t *v
                 alpha = (t == 0) ? 0.0 : exp2(((double)m - (double)mnew) * (double)A / 8.0);
                 l *= alpha;
                 for (d = 0; d < Dv; ++d) acc[d] *= alpha;
-                for (n = 0; n < 128; ++n) {
-                    int j = 128 * t + n;
+                for (n = 0; n < kv_tile; ++n) {
+                    int j = kv_tile * t + n;
                     double w;
                     const uint8_t *vj;
                     if (!live[n]) continue;

@@ -44,7 +44,7 @@ def lib():
         L.oracle_leanp_batch.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i, c_p, c_p]
         L.oracle_fp8_model_rows.restype = c_i
         L.oracle_fp8_model_rows.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_i, c_i, c_i, c_i,
-                                            c_i, c_i, c_i, c_f, c_p, c_i, c_p, c_p]
+                                            c_i, c_i, c_i, c_f, c_i, c_p, c_i, c_p, c_p]
         L.oracle_attention_lse_rows.restype = c_i
         L.oracle_attention_lse_rows.argtypes = [c_p, c_p, c_i, c_i, c_i, c_i, c_i, c_d, c_p, c_i, c_p]
         L.oracle_exactp_code.restype = ctypes.c_uint
@@ -195,10 +195,12 @@ def leanp_batch(s, m, bmax, A, masked=None):
 
 
 def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=0.0, p_mode=None,
-              return_lse=False):
+              return_lse=False, kv_tile=128):
     """The FP8 pipeline replayed on the CPU (see oracle.c).  Codes uint8 BSHD,
     scales fp32 [B,H].  rescale_log2 = 0: exact running max; > 0: the reference
     max moves only when a tile max exceeds it by more than that many binades.
+    kv_tile: keys per KV tile (128 or 256), the unit at which that decision
+    is taken.
     p_mode: 0 Lean-P codes (default), 1 exact fp64 weights (exact_p=True),
     2 exact exp2 rounded to e4m3 (the exact-P ablation).
     Returns o fp64 [B, S or len(rows), Hq, Dv] (and lse [B, Hq, rows] with
@@ -214,7 +216,8 @@ def fp8_model(qc, kc, vc, q_s, k_s, v_s, exact_p=False, rows=None, rescale_log2=
     o = np.empty((B, n, Hq, Dv), dtype=np.float64)
     lse = np.empty((B, Hq, n), dtype=np.float64) if return_lse else None
     rc = lib().oracle_fp8_model_rows(_ptr(qc), _ptr(kc), _ptr(vc), _ptr(q_s), _ptr(k_s), _ptr(v_s),
-                                     B, Hq, Hkv, S, Dqk, Dv, int(p_mode), ctypes.c_float(rescale_log2), _ptr(r), n, _ptr(o),
+                                     B, Hq, Hkv, S, Dqk, Dv, int(p_mode), ctypes.c_float(rescale_log2), int(kv_tile),
+                                     _ptr(r), n, _ptr(o),
                                      _ptr(lse))
     if rc == -2:
         raise ArithmeticError("oracle_fp8_model_rows: a block shift fell below its bound (reference max too stale)")
@@ -271,7 +274,7 @@ def quantize_varlen(x, cu, hadamard: bool = False):
     return codes, scale
 
 
-def fp8_model_varlen(qc, kc, vc, q_s, k_s, v_s, cu, rescale_log2=0.0, p_mode=0, return_lse=False):
+def fp8_model_varlen(qc, kc, vc, q_s, k_s, v_s, cu, rescale_log2=0.0, p_mode=0, return_lse=False, kv_tile=128):
     """fp8_model over a packed batch: codes [T,H,D], scales [nseq,H].  Returns o [T,Hq,Dv] (and
     lse [Hq,T] with return_lse)."""
     T, Hq = qc.shape[0], qc.shape[1]
@@ -281,7 +284,8 @@ def fp8_model_varlen(qc, kc, vc, q_s, k_s, v_s, cu, rescale_log2=0.0, p_mode=0, 
         if r1 == r0:
             continue
         res = fp8_model(qc[None, r0:r1], kc[None, r0:r1], vc[None, r0:r1], q_s[s:s + 1], k_s[s:s + 1],
-                        v_s[s:s + 1], rescale_log2=rescale_log2, p_mode=p_mode, return_lse=return_lse)
+                        v_s[s:s + 1], rescale_log2=rescale_log2, p_mode=p_mode, return_lse=return_lse,
+                        kv_tile=kv_tile)
         if return_lse:
             o[r0:r1] = res[0][0]
             lse[:, r0:r1] = res[1][0]

@@ -299,15 +299,40 @@ def _quantized_case(seed, B, S, Hq, Hkv, D, Dv=None):
                                       orc.dequantize(vc, vs)), (q, k, v)
 
 
-def test_model_oracle_exact_p_equals_plain_definition():
+@pytest.mark.parametrize("kv_tile", [128, 256])
+def test_model_oracle_exact_p_equals_plain_definition(kv_tile):
     codes, deq, _ = _quantized_case(12, 1, 300, 4, 2, 128)
     qc, kc, vc, qs, ks, vs = codes
-    o_model = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True)
+    o_model = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True, kv_tile=kv_tile)
     o_ref = orc.attention(*deq)
     assert orc.rel_fro(o_model, o_ref) < 1e-6
+    o_lazy = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True, kv_tile=kv_tile, rescale_log2=64.0)
+    assert orc.rel_fro(o_lazy, o_ref) < 1e-6
 
 
-def _growing_score_case(seed, threshold=8.0):
+def test_model_oracle_tile_size_moves_the_reference_decision():
+    """The deferred reference is decided once per KV tile, so 128- and 256-key
+    tiles give different Lean-P codes (the first tile's max differs for rows
+    past key 127), both within the FP8 bar.  (So does the exact running max:
+    the codes depend on the max the tile is coded against, and that max
+    covers the whole tile.)"""
+    codes, deq, _ = _quantized_case(15, 1, 700, 2, 2, 128)
+    qc, kc, vc, qs, ks, vs = codes
+    ref = orc.attention(*deq)
+    o128 = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=64.0, kv_tile=128)
+    o256 = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=64.0, kv_tile=256)
+    assert not np.array_equal(o128[:, 128:], o256[:, 128:])
+    assert np.array_equal(o128[:, :128], o256[:, :128])   # rows 0..127 see one tile either way
+    assert orc.rel_fro(o128, ref) < 3e-2 and orc.rel_fro(o256, ref) < 3e-2
+
+
+def test_model_oracle_rejects_other_tile_sizes():
+    codes, _, _ = _quantized_case(16, 1, 64, 1, 1, 128)
+    with pytest.raises(ValueError):
+        orc.fp8_model(*codes, kv_tile=192)
+
+
+def _growing_score_case(seed, threshold=8.0, tile=128):
     """Q = 1.0 everywhere, K rows near a per-tile level, so the score of key j
     for every query is about 128 * level(tile of j), about 16.3 level binades
     (s * 8 log2(e) / sqrt(128) / 8), a little less for the tile max since K
@@ -315,36 +340,37 @@ def _growing_score_case(seed, threshold=8.0):
     8-binade deferral bound the tile max jumps by ~19 binades (rescaled), then
     ~4 (deferred), falls, then ~11 above the deferred reference (rescaled);
     for a 64-binade bound by ~70 binades (rescaled), then ~30 (deferred),
-    falls, then ~78 above the reference (rescaled)."""
+    falls, then ~78 above the reference (rescaled).  `tile` keys share a level
+    (the KV tile of the replay under test)."""
     rng = np.random.default_rng(seed)
     vals = orc.e4m3_values()
     code_of = {float(vals[c]): c for c in range(0x00, 0x7F)}
     levels = {8.0: [0.5, 1.75, 2.0, 1.5, 2.5], 64.0: [0.5, 5.0, 7.0, 3.0, 10.0]}[threshold]
-    S, D = 128 * len(levels), 128
+    S, D = tile * len(levels), 128
     qc = np.full((1, S, 1, D), code_of[1.0], dtype=np.uint8)
     kc = np.empty((1, S, 1, D), dtype=np.uint8)
     for t, lv in enumerate(levels):
         c = code_of[lv]
-        kc[0, 128 * t:128 * (t + 1), 0, :] = c - rng.integers(0, 2, size=(128, D))  # lv or next lower
+        kc[0, tile * t:tile * (t + 1), 0, :] = c - rng.integers(0, 2, size=(tile, D))  # lv or next lower
     vc = rng.integers(0x20, 0x50, size=(1, S, 1, D), dtype=np.uint8)
     vc |= (rng.integers(0, 2, size=vc.shape) << 7).astype(np.uint8)              # random signs
     one = np.ones((1, 1), dtype=np.float32)
     return qc, kc, vc, one, one, one
 
 
-@pytest.mark.parametrize("r", [8.0, 64.0])
-def test_model_oracle_deferred_max_equals_plain_definition(r):
+@pytest.mark.parametrize("r,tile", [(8.0, 128), (64.0, 128), (64.0, 256)])
+def test_model_oracle_deferred_max_equals_plain_definition(r, tile):
     """With exact probabilities the deferred reference max (r binades) must give
     the plain softmax: pins the deferral rule, its alpha and that O and l are
     rescaled together, on scores that grow far beyond the fp32 exp2 range."""
-    qc, kc, vc, qs, ks, vs = _growing_score_case(21, r)
+    qc, kc, vc, qs, ks, vs = _growing_score_case(21, r, tile)
     deq = tuple(orc.dequantize(x, sc) for x, sc in ((qc, qs), (kc, ks), (vc, vs)))
     ref = orc.attention(*deq)
-    o_lazy = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True, rescale_log2=r)
+    o_lazy = orc.fp8_model(qc, kc, vc, qs, ks, vs, exact_p=True, rescale_log2=r, kv_tile=tile)
     assert orc.rel_fro(o_lazy, ref) < 1e-6
     # the deferral changes the Lean-P codes (the reference moves), not the bar
-    o_exact = orc.fp8_model(qc, kc, vc, qs, ks, vs)
-    o_def = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=r)
+    o_exact = orc.fp8_model(qc, kc, vc, qs, ks, vs, kv_tile=tile)
+    o_def = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=r, kv_tile=tile)
     assert not np.array_equal(o_exact, o_def)
     assert orc.rel_fro(o_def, ref) < 3e-2 and orc.rel_fro(o_exact, ref) < 3e-2
     # the case exercises what it is meant to: tile maxima (in binades) that jump
@@ -352,7 +378,7 @@ def test_model_oracle_deferred_max_equals_plain_definition(r):
     # block shifts below 8), fall, and pass the bound again
     A8 = float(orc.leanp_slope(1.0, 1.0, 128)) / 8.0
     qv = orc.e4m3_values()[qc[0, 0, 0]].astype(np.float64)
-    tmax = [float((orc.e4m3_values()[kc[0, 128 * t:128 * t + 128, 0]].astype(np.float64) @ qv).max()) * A8
+    tmax = [float((orc.e4m3_values()[kc[0, tile * t:tile * t + tile, 0]].astype(np.float64) @ qv).max()) * A8
             for t in range(5)]
     assert tmax[1] - tmax[0] > r                     # moves the reference
     assert 0 < tmax[2] - tmax[1] <= r                # deferred: block above the reference
@@ -360,20 +386,22 @@ def test_model_oracle_deferred_max_equals_plain_definition(r):
     assert tmax[4] - tmax[1] > r                     # moves it again
 
 
-def test_model_oracle_zero_q_gives_prefix_means():
+@pytest.mark.parametrize("kv_tile", [128, 256])
+def test_model_oracle_zero_q_gives_prefix_means(kv_tile):
     codes, deq, _ = _quantized_case(13, 1, 200, 2, 2, 128)
     qc, kc, vc, qs, ks, vs = codes
     qz = np.zeros_like(qc)
-    o = orc.fp8_model(qz, kc, vc, qs, ks, vs)
+    o = orc.fp8_model(qz, kc, vc, qs, ks, vs, kv_tile=kv_tile)
     pref = np.cumsum(deq[2], axis=1) / np.arange(1, 201)[None, :, None, None]
     assert np.allclose(o, pref, atol=1e-12)
     assert np.array_equal(o[:, 0], deq[2][:, 0])
 
 
-def test_model_oracle_leanp_error_against_fp64_is_within_fp8_bar():
+@pytest.mark.parametrize("kv_tile", [128, 256])
+def test_model_oracle_leanp_error_against_fp64_is_within_fp8_bar(kv_tile):
     codes, deq, _ = _quantized_case(14, 1, 512, 2, 2, 128)
     qc, kc, vc, qs, ks, vs = codes
-    o = orc.fp8_model(qc, kc, vc, qs, ks, vs)
+    o = orc.fp8_model(qc, kc, vc, qs, ks, vs, kv_tile=kv_tile, rescale_log2=64.0)
     ref = orc.attention(*deq)
     err = orc.rel_fro(o, ref)
     assert 1e-3 < err < 3e-2
