@@ -850,7 +850,7 @@ def run_ours(args, wl):
         "warmup": args.warmup, "ms_per_step": ms8, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
         "config": config_for(args, wl, world),
-        "roofline": roofline(ach8, peaks, "fp8", f"attn_fwd_kernel<FP8,{Dqk}>", sm_mhz, load_traffic(args.workload)),
+        "roofline": roofline(ach8, peaks, "fp8", fp8_kernel_name(Dqk), sm_mhz, load_traffic(args.workload)),
         "bf16": {"value": value_b, "unit": "TFLOP/s", "ms_per_step": msb,
                  "roofline": roofline(achb, peaks, "bf16", f"attn_fwd_kernel<BF16,{Dqk}>", sm_mhz)},
         "fp8_breakdown_ms": {"prepass": ms8_pre, "attention": ms8_attn},
@@ -862,7 +862,7 @@ def run_ours(args, wl):
         "peaks_measured": gemm,
         "sustained": sus,
         "ablation": None if msx is None else {
-            "exact_p": {"kernel": f"attn_fwd_kernel<FP8,{Dqk},exact P>", "attention_ms": msx,
+            "exact_p": {"kernel": fp8_kernel_name(Dqk, "exact P"), "attention_ms": msx,
                         "attention_tflops": flops / (msx * 1e-3) / 1e12,
                         "frac": flops / (msx * 1e-3) / 1e12 / peaks.fp8,
                         "lean_p_attention_tflops": ach8,
@@ -902,7 +902,7 @@ def run_extra(torch, zyfa, args, wname, rank, world, dev, flush, stream, peaks, 
                "fp8_attention_tflops": vc.flops / (out["attn8"] * 1e-3) / 1e12,
                "bf16_attention_tflops": vc.flops / (out["bf16"] * 1e-3) / 1e12, "ms": out,
                "roofline": {"fp8": roofline(vc.flops / (out["attn8"] * 1e-3) / 1e12, peaks, "fp8",
-                                            f"attn_fwd_kernel<FP8,{wl['Dqk']},varlen>"),
+                                            fp8_kernel_name(wl['Dqk'], "varlen")),
                             "bf16": roofline(vc.flops / (out["bf16"] * 1e-3) / 1e12, peaks, "bf16",
                                              f"attn_fwd_kernel<BF16,{wl['Dqk']},varlen>")}}
         if world == 1:
@@ -924,7 +924,7 @@ def run_extra(torch, zyfa, args, wname, rank, world, dev, flush, stream, peaks, 
            "bf16_attention_tflops": fl / (out["bf16"] * 1e-3) / 1e12,
            "exact_p_attention_tflops": fl / (out["exact_p"] * 1e-3) / 1e12, "ms": out,
            "prepass_gbs": prepass_bytes(wl["B"], wl["S"], wl["Hq"], wl["Hkv"], Dqk, wl["Dv"]) / (out["prepass"] * 1e-3) / 1e9,
-           "roofline": {"fp8": roofline(fl / (out["attn8"] * 1e-3) / 1e12, peaks, "fp8", f"attn_fwd_kernel<FP8,{Dqk}>"),
+           "roofline": {"fp8": roofline(fl / (out["attn8"] * 1e-3) / 1e12, peaks, "fp8", fp8_kernel_name(Dqk)),
                         "bf16": roofline(fl / (out["bf16"] * 1e-3) / 1e12, peaks, "bf16",
                                          f"attn_fwd_kernel<BF16,{Dqk}>")}}
     if world == 1:
@@ -1142,7 +1142,7 @@ def run_varlen(args, wl):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms["step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3",
         "data": "synthetic", "config": dict(config_for(args, wl, world), lens=vc.lens),
-        "roofline": roofline(ach8, peaks, "fp8", f"attn_fwd_kernel<FP8,{wl['Dqk']},varlen>", sm_mhz),
+        "roofline": roofline(ach8, peaks, "fp8", fp8_kernel_name(wl['Dqk'], "varlen"), sm_mhz),
         "bf16": {"value": world * flops / (ms["bf16"] * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms["bf16"],
                  "roofline": roofline(achb, peaks, "bf16", f"attn_fwd_kernel<BF16,{wl['Dqk']},varlen>", sm_mhz)},
         "fp8_breakdown_ms": {"prepass": ms["prepass"], "attention": ms["attn8"]},
@@ -1163,7 +1163,16 @@ def run_varlen(args, wl):
     return 0
 
 
-KERNEL_SOURCES = ("attn_fwd.cuh", "leanp.cuh", "ptx.cuh")
+KERNEL_SOURCES = ("attn_fwd.cuh", "attn_fwd_wide.cuh", "leanp.cuh", "ptx.cuh")
+
+
+def fp8_kernel_name(Dqk, extra=""):
+    """The FP8 attention kernel instance the library runs for Dqk: 256-key KV
+    tiles for Dqk 128 (attn_fwd_wide_kernel), 128-key tiles otherwise."""
+    tail = f",{extra}" if extra else ""
+    if Dqk == 128:
+        return f"attn_fwd_wide_kernel<FP8,128{tail}>"
+    return f"attn_fwd_kernel<FP8,{Dqk}{tail}>"
 
 
 def kernel_source_hash():

@@ -288,9 +288,10 @@ __device__ __forceinline__ bool elect_one() {
 
 // The CTA's sequence of (unit, KV tile) pairs in issue order; g counts tiles
 // and u counts units across the whole sequence (ring stages and barrier phases
-// derive from them).  VARLEN: r0 and len are the unit's sequence's first
-// packed row and length.
-template <bool VARLEN>
+// derive from them).  KT keys per KV tile (128, or 256 for the wide FP8
+// kernel): a unit of query tile qt visits tiles 0 .. qt*128/KT.  VARLEN: r0
+// and len are the unit's sequence's first packed row and length.
+template <bool VARLEN, int KT = 128>
 struct TileStream {
   typename std::conditional<VARLEN, VarlenIter, UnitIter>::type units;
   int b, hkv, hq, qt, j, nkv;
@@ -309,7 +310,7 @@ struct TileStream {
     } else {
       if (!units.next(b, hkv, hq, qt)) return false;
     }
-    nkv = qt + 1; j = 0; ++g; ++u;
+    nkv = qt * 128 / KT + 1; j = 0; ++g; ++u;
     return true;
   }
 };

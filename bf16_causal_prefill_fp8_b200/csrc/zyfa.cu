@@ -15,6 +15,7 @@
 
 #include "../../include/zyfa.h"
 #include "attn_fwd.cuh"
+#include "attn_fwd_wide.cuh"
 #include "leanp.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
@@ -62,7 +63,7 @@ EncodeTiledFn encode_fn() {
 
 struct DeviceInfo {
   int sms = 0;
-  bool attr_set[10] = {};
+  bool attr_set[14] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -148,10 +149,9 @@ bool fill_attn_args(AttnArgs& a, const void* q, const void* k, const void* v, vo
   return true;
 }
 
-// SM count of the device, and the kernel instance's shared-memory opt-in (once)
-template <bool FP8, int DQK, bool EXACTP, bool VARLEN>
-bool prepare_device(int dev, int inst) {
-  using Cf = AttnCfg<FP8, DQK>;
+// SM count of the device, and a kernel instance's shared-memory opt-in (once)
+template <typename Kernel>
+bool prepare_kernel(int dev, int inst, Kernel kernel, int smem) {
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceInfo& di = g_dev[dev];
   if (di.sms == 0 && cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -161,15 +161,17 @@ bool prepare_device(int dev, int inst) {
     // a raise asking for more than that would wait forever, so a build whose
     // register count differs is refused here, before any launch
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<FP8, DQK, EXACTP, VARLEN>) != cudaSuccess ||
-        fa.numRegs != kLaunchRegs)
-      return false;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<FP8, DQK, EXACTP, VARLEN>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM) != cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs != kLaunchRegs) return false;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return false;
     di.attr_set[inst] = true;
   }
   return true;
+}
+
+template <bool FP8, int DQK, bool EXACTP, bool VARLEN>
+bool prepare_device(int dev, int inst) {
+  return prepare_kernel(dev, inst, attn_fwd_kernel<FP8, DQK, EXACTP, VARLEN>, AttnCfg<FP8, DQK>::SMEM);
 }
 
 template <bool FP8, int DQK, bool EXACTP = false>
@@ -207,6 +209,41 @@ int launch_attn_varlen(const void* q, const void* k, const void* v, void* o, con
   if (!prepare_device<FP8, DQK, false, true>(dev, inst)) return ZYFA_ERR_CUDA;
   const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
   attn_fwd_kernel<FP8, DQK, false, true><<<grid, kAttnThreads, Cf::SMEM, stream>>>(a, t);
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+// FP8 with Dqk = 128 runs the 256-key-tile kernel (attn_fwd_wide.cuh).
+template <bool EXACTP>
+int launch_attn_wide(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int S,
+                     const float* qs, const float* ks, const float* vs, cudaStream_t stream, int dev, int inst,
+                     float* lse = nullptr) {
+  AttnArgs a;
+  if (!fill_attn_args<true, 128>(a, q, k, v, o, B, Hq, Hkv, S, qs, ks, vs, lse)) return ZYFA_ERR_CUDA;
+  a.B = B; a.S = S;
+  a.Tq = (S + 127) / 128;
+  a.group_slots = group_slots_for(B, Hkv, S, 128, 1);
+  if (!prepare_kernel(dev, inst, attn_fwd_wide_kernel<EXACTP, false>, WideCfg::SMEM)) return ZYFA_ERR_CUDA;
+  const long long units = static_cast<long long>(B) * Hq * a.Tq;
+  const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
+  attn_fwd_wide_kernel<EXACTP, false><<<grid, kAttnThreads, WideCfg::SMEM, stream>>>(a, SeqTable<false>{});
+  return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
+}
+
+int launch_attn_wide_varlen(const void* q, const void* k, const void* v, void* o, const int* cu, int nseq, int Hq,
+                            int Hkv, const float* qs, const float* ks, const float* vs, cudaStream_t stream,
+                            int dev, int inst, float* lse) {
+  const long long units = varlen_units(cu, nseq, Hq);
+  if (units == 0) return ZYFA_OK;
+  const int T = cu[nseq];
+  AttnArgs a;
+  if (!fill_attn_args<true, 128>(a, q, k, v, o, 1, Hq, Hkv, T, qs, ks, vs, lse)) return ZYFA_ERR_CUDA;
+  a.B = nseq; a.S = T;
+  a.Tq = 0; a.group_slots = 0;
+  SeqTable<true> t;
+  fill_varlen_table(t, cu, nseq, 128, 1);
+  if (!prepare_kernel(dev, inst, attn_fwd_wide_kernel<false, true>, WideCfg::SMEM)) return ZYFA_ERR_CUDA;
+  const int grid = static_cast<int>(units < g_dev[dev].sms ? units : g_dev[dev].sms);
+  attn_fwd_wide_kernel<false, true><<<grid, kAttnThreads, WideCfg::SMEM, stream>>>(a, t);
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
@@ -311,7 +348,7 @@ extern "C" int zyfa_attn_fwd(const void* q, const void* k, const void* v, void* 
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == ZYFA_FP8_E4M3) {
-    if (Dqk == 128) return launch_attn<true, 128>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 0);
+    if (Dqk == 128) return launch_attn_wide<false>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 10);
     return launch_attn<true, 192>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 1);
   }
   if (Dqk == 128) return launch_attn<false, 128>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 2);
@@ -329,7 +366,7 @@ extern "C" int zyfa_attn_fwd_lse(const void* q, const void* k, const void* v, vo
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == ZYFA_FP8_E4M3) {
-    if (Dqk == 128) return launch_attn<true, 128>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 0, lse);
+    if (Dqk == 128) return launch_attn_wide<false>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 10, lse);
     return launch_attn<true, 192>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 1, lse);
   }
   if (Dqk == 128) return launch_attn<false, 128>(q, k, v, o, B, Hq, Hkv, S, nullptr, nullptr, nullptr, st, dev, 2, lse);
@@ -344,7 +381,7 @@ extern "C" int zyfa_attn_fwd_fp8_exact_p(const void* q, const void* k, const voi
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZYFA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (Dqk == 128) return launch_attn<true, 128, true>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 4);
+  if (Dqk == 128) return launch_attn_wide<true>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 11);
   return launch_attn<true, 192, true>(q, k, v, o, B, Hq, Hkv, S, q_scale, k_scale, v_scale, st, dev, 5);
 }
 
@@ -494,8 +531,8 @@ extern "C" int zyfa_attn_fwd_varlen(const void* q, const void* k, const void* v,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == ZYFA_FP8_E4M3) {
     if (Dqk == 128)
-      return launch_attn_varlen<true, 128>(q, k, v, o, cu_seqlens, nseq, Hq, Hkv, q_scale, k_scale, v_scale, st,
-                                           dev, 6, lse);
+      return launch_attn_wide_varlen(q, k, v, o, cu_seqlens, nseq, Hq, Hkv, q_scale, k_scale, v_scale, st, dev, 12,
+                                     lse);
     return launch_attn_varlen<true, 192>(q, k, v, o, cu_seqlens, nseq, Hq, Hkv, q_scale, k_scale, v_scale, st,
                                          dev, 7, lse);
   }
@@ -616,6 +653,12 @@ extern "C" int zyfa_quantize_qkv_varlen(const void* q, const void* k, const void
   float* scs[3] = {q_scale, k_scale, v_scale};
   const int Hs[3] = {Hq, Hkv, Hkv}, Ds[3] = {Dqk, Dqk, Dv}, had[3] = {hadamard_qk, hadamard_qk, 0};
   return quantize_varlen_n(3, xs, outs, scs, Hs, Ds, had, in_dtype, cu_seqlens, nseq, stream);
+}
+
+extern "C" int zyfa_attn_kv_tile(int dtype, int Dqk) {
+  if (dtype != ZYFA_BF16 && dtype != ZYFA_FP8_E4M3) return ZYFA_ERR_BAD_DTYPE;
+  if (Dqk != 128 && Dqk != 192) return ZYFA_ERR_UNSUPPORTED_HEADDIM;
+  return (dtype == ZYFA_FP8_E4M3 && Dqk == 128) ? WideCfg::KT : 128;
 }
 
 extern "C" int zyfa_attn_schedule(int B, int S, const int* cu_seqlens, int Hq, int Hkv, int Dqk, int dtype,

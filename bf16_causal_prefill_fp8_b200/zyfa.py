@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.zyfa_quantize_qkv_varlen.argtypes = [p, p, p, i, p, p, p, p, p, p, p, i, i, i, i, i, i, p]
         L.zyfa_attn_schedule.restype = i
         L.zyfa_attn_schedule.argtypes = [i, i, p, i, i, i, i, i, i, p, i]
+        L.zyfa_attn_kv_tile.restype = i
+        L.zyfa_attn_kv_tile.argtypes = [i, i]
         L.zyfa_status_string.restype = ctypes.c_char_p
         L.zyfa_status_string.argtypes = [i]
         L.zyfa_device_status.restype = i
@@ -409,6 +411,15 @@ def attn_schedule(Hq, Hkv, Dqk, dtype, grid, cta, B=None, S=None, cu_seqlens=Non
     if m != n:
         raise ZyfaError(m if m < 0 else -2, "zyfa_attn_schedule")
     return [(buf[3 * i], buf[3 * i + 1], buf[3 * i + 2]) for i in range(n)]
+
+
+def kv_tile(dtype, Dqk) -> int:
+    """Host-only: keys per KV tile of the attention kernel run for (dtype, Dqk); the deferred
+    reference max is decided once per such tile."""
+    n = lib().zyfa_attn_kv_tile(int(dtype), int(Dqk))
+    if n < 0:
+        raise ZyfaError(n, "zyfa_attn_kv_tile")
+    return n
 
 
 def leanp_codes(s, m, bmax, A, masked=None, stream=None):

@@ -242,11 +242,24 @@ int zyfa_quantize_qkv_varlen(const void* q, const void* k, const void* v, int in
                              int hadamard_qk, void* stream);
 
 /*
+ * zyfa_attn_kv_tile -- host only: the keys per KV tile of the attention
+ * kernel that zyfa_attn_fwd (and its _lse, _fp8_exact_p and _varlen forms)
+ * runs for this dtype and Dqk: 256 for FP8 with Dqk 128 (S = Q K^T over a
+ * 256-key tile is one N = 256 tensor-core accumulator), 128 otherwise.  The
+ * deferred reference max of the online softmax (the running max that the
+ * probabilities are taken against, which moves only when a tile's max
+ * exceeds it by more than 64 binades) is decided once per such tile, so a
+ * replay of the FP8 pipeline needs it.  Returns ZYFA_ERR_BAD_DTYPE or
+ * ZYFA_ERR_UNSUPPORTED_HEADDIM for arguments zyfa_attn_fwd would reject.
+ */
+int zyfa_attn_kv_tile(int dtype, int Dqk);
+
+/*
  * zyfa_attn_schedule -- host only (no device call): the work units that CTA
  * `cta` of a `grid`-CTA attention launch processes, in order, as the kernel
  * enumerates them.  A unit is (b, hq, qt): query tile qt (rows 128 qt ..
  * 128 qt + 127) of query head hq of batch entry / sequence b, which takes
- * key tiles 0..qt.  Fixed length: cu_seqlens = NULL, B entries of S rows.
+ * key tiles 0 .. (128 qt) / kv_tile (kv_tile from zyfa_attn_kv_tile).  Fixed length: cu_seqlens = NULL, B entries of S rows.
  * Packed: cu_seqlens as above with nseq = B (S ignored).  The launch itself
  * uses grid = min(units, SM count).  Writes min(count, cap) units as int
  * triples to `units` (host memory) and returns the count, or a negative

@@ -72,8 +72,16 @@ def fp8_references(codes, rows=None):
     (qc, qs), (kc, ks), (vc, vs) = codes
     deq = (orc.dequantize(qc, qs), orc.dequantize(kc, ks), orc.dequantize(vc, vs))
     ref = orc.attention(*deq, rows=rows)
-    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rows=rows, rescale_log2=RESCALE_LOG2)
+    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rows=rows, rescale_log2=RESCALE_LOG2,
+                          kv_tile=fp8_kv_tile(qc.shape[3]))
     return ref, model
+
+
+def fp8_kv_tile(Dqk):
+    """Keys per KV tile of the FP8 kernel for this Dqk, as the library reports it: the
+    CPU replay takes the deferred reference-max decision at the same tiles."""
+    from bf16_causal_prefill_fp8_b200 import zyfa
+    return zyfa.kv_tile(zyfa.FP8_E4M3, Dqk)
 
 
 # Localised bounds.  A whole-tensor relative error dilutes one bad head or one

@@ -19,6 +19,11 @@ when the completed-phase count has the other parity.  The model checks that
 `two_producers` splits the TMA producer into a K (and Q) warp and a V warp,
 each walking the tiles on its own (a variant that was once tried).
 
+`run_wide` models the FP8 kernel with 256-key tiles (csrc/attn_fwd_wide.cuh):
+one S buffer and one P buffer, both softmax groups on every tile (each on
+its own 128-key half), the tile max exchanged through a two-slot buffer under
+one barrier both groups arrive on, and the hand-over written by group 0.
+
 `mutation` plants a known mistake, for the tests that show the model catches it.
 """
 import random
@@ -251,6 +256,221 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_produce
     while len(done) < len(roles):
         progressed = False
         for fk in rng.sample(["qk", "pv"], 2):     # the tensor core completes each issuer's work in order
+            f = fifos[fk]
+            if not f:
+                continue
+            e = f[0]
+            if e[1] == "commit":
+                for n in e[2]:
+                    bars[n].arrive()
+                f.pop(0)
+            else:
+                e[0] -= 1
+                if e[0] <= 0:
+                    (st["qk_done"] if e[1] == "qk" else st["pv_done"]).add(e[2])
+                    f.pop(0)
+            progressed = True
+        for t in list(tma):
+            t[0] -= 1
+            if t[0] <= 0:
+                bars[t[1]].arrive()
+                tma.remove(t)
+            progressed = True
+        names = [n for n in roles if n not in done]
+        rng.shuffle(names)
+        for n in names:
+            try:
+                if next(roles[n]) != "wait":
+                    progressed = True
+            except StopIteration:
+                done.add(n)
+                progressed = True
+        idle = 0 if progressed else idle + 1
+        if idle >= 1000:
+            raise ProtocolError("deadlock: " + ", ".join(f"{k} {b.c}/{b.pend}" for k, b in bars.items() if b.pend))
+
+
+@dataclass(frozen=True)
+class WideConfig:
+    stk: int = 3   # K ring stages (256-key tiles)
+    stv: int = 2   # V ring stages
+    qbuf: int = 2  # Q tile buffers
+    hand: int = 8  # unit hand-over slots
+
+    @property
+    def klead(self):
+        return self.stk - self.stv + 1
+
+
+WIDE = WideConfig()
+
+
+def run_wide(units, cfg: WideConfig, seed: int, mutation=None, p_rescale=0.5):
+    """Simulate one CTA of the 256-key-tile kernel over `units` (tile counts)."""
+    rng = random.Random(seed)
+    bars = {}
+
+    def bar(n, cnt):
+        bars[n] = _Bar(n, cnt)
+
+    for i in range(cfg.qbuf):
+        bar(f"QF{i}", 1); bar(f"QE{i}", 1)
+    for n, c in (("SF", 1), ("SC", 256), ("MXA", 256), ("PF", 256), ("PE", 1), ("OF", 128), ("OFIN", 1)):
+        bar(n, c)
+    for i in range(cfg.hand):
+        bar(f"LF{i}", 128)
+    for i in range(cfg.stk):
+        bar(f"KF{i}", 1); bar(f"KE{i}", 1)
+    for i in range(cfg.stv):
+        bar(f"VF{i}", 1); bar(f"VE{i}", 1)
+    tiles = [(u, j, nkv) for u, nkv in enumerate(units) for j in range(nkv)]
+    # the rescale decision of a tile: both groups compute the same one
+    rescale = [j > 0 and rng.random() < p_rescale for (u, j, nkv) in tiles]
+    fifos = {"qk": [], "pv": []}
+    tma = []
+    st = {"P": {}, "O_unit": None, "pv_done": set(), "qk_done": set(), "Sread": {0: -1, 1: -1},
+          "xch": {}, "xch_read": {}, "hand": {}, "hand_read": set()}
+
+    def wait(name, parity, need):
+        b = bars[name]
+        while True:
+            passed = (b.c & 1) != parity
+            truly = b.c > need
+            if passed:
+                if not truly:
+                    raise ProtocolError(f"aliasing on {name}: parity {parity} passed at phase count {b.c}, "
+                                        f"needs more than {need}")
+                return
+            if truly:
+                raise ProtocolError(f"stuck on {name}: phase {need} complete but parity {parity} fails")
+            yield "wait"
+
+    def producer():
+        def load_k(g):
+            u, j, nkv = tiles[g]
+            if j == 0:
+                slot, n = u % cfg.qbuf, u // cfg.qbuf
+                if n > 0:
+                    yield from wait(f"QE{slot}", (n - 1) & 1, n - 1)
+                tma.append([rng.randint(5, 40), f"QF{slot}"])
+            s_, n = g % cfg.stk, g // cfg.stk
+            if n > 0:
+                yield from wait(f"KE{s_}", (n - 1) & 1, n - 1)
+            tma.append([rng.randint(5, 40), f"KF{s_}"])
+
+        def load_v(g):
+            s_, n = g % cfg.stv, g // cfg.stv
+            if n > 0:
+                yield from wait(f"VE{s_}", (n - 1) & 1, n - 1)
+            tma.append([rng.randint(5, 40), f"VF{s_}"])
+
+        ks = vs = 0
+        for _ in range(cfg.klead):
+            if ks < len(tiles):
+                yield from load_k(ks); ks += 1
+        while vs < len(tiles):
+            if ks < len(tiles):
+                yield from load_k(ks); ks += 1
+            yield from load_v(vs); vs += 1
+            yield "step"
+
+    def qk_issuer():
+        for g, (u, j, nkv) in enumerate(tiles):
+            slot = u % cfg.qbuf
+            if j == 0:
+                yield from wait(f"QF{slot}", (u // cfg.qbuf) & 1, u // cfg.qbuf)
+            s_ = g % cfg.stk
+            yield from wait(f"KF{s_}", (g // cfg.stk) & 1, g // cfg.stk)
+            if g >= 1 and mutation != "no_sc_wait":
+                yield from wait("SC", (g - 1) & 1, g - 1)
+            if g >= 1 and min(st["Sread"].values()) < g - 1:
+                raise ProtocolError(f"S overwritten by tile {g} before both groups read tile {g - 1}")
+            fifos["qk"].append([rng.randint(5, 30), "qk", g])
+            fifos["qk"].append([0, "commit", ["SF", f"KE{s_}"] + ([f"QE{slot}"] if j == nkv - 1 else [])])
+            yield "step"
+
+    def pv_issuer():
+        for g, (u, j, nkv) in enumerate(tiles):
+            s_ = g % cfg.stv
+            if j == 0 and u > 0:
+                yield from wait("OF", (u - 1) & 1, u - 1)
+            yield from wait(f"VF{s_}", (g // cfg.stv) & 1, g // cfg.stv)
+            yield from wait("PF", g & 1, g)
+            if st["P"].get(0) != g or st["P"].get(1) != g:
+                raise ProtocolError(f"P holds tiles {st['P']} at P V of tile {g}")
+            if j == 0:
+                if st["O_unit"] not in (None, "free"):
+                    raise ProtocolError(f"O still in use by unit {st['O_unit']} at unit {u}")
+                st["O_unit"] = u
+            fifos["pv"].append([rng.randint(5, 30), "pv", g])
+            fifos["pv"].append([0, "commit", [f"VE{s_}", "PE"] + (["OFIN"] if j == nkv - 1 else [])])
+            yield "step"
+
+    def softmax_group(x):
+        for g, (u, j, nkv) in enumerate(tiles):
+            yield from wait("SF", g & 1, g)
+            if g not in st["qk_done"]:
+                raise ProtocolError(f"S of tile {g} read before its MMA finished")
+            yield "load"
+            st["Sread"][x] = g
+            bars["SC"].arrive(128)
+            yield "max"
+            slot = g & 1
+            prev = st["xch"].get((slot, x))
+            if prev is not None and st["xch_read"].get((slot, x)) != prev:
+                raise ProtocolError(f"tile max of tile {prev} (group {x}) overwritten before the other group read it")
+            st["xch"][(slot, x)] = g
+            bars["MXA"].arrive(128)
+            if mutation != "no_mx_wait":
+                yield from wait("MXA", g & 1, g)
+            if st["xch"].get((slot, 1 - x)) != g:
+                raise ProtocolError(f"group {x} read the other group's tile max of tile "
+                                    f"{st['xch'].get((slot, 1 - x))} at tile {g}")
+            st["xch_read"][(slot, 1 - x)] = g
+            for _ in range(rng.randint(0, 4)):
+                yield "codes"
+            if g >= 1 and mutation != "no_pe_wait":
+                yield from wait("PE", (g - 1) & 1, g - 1)
+            if g >= 1 and (g - 1) not in st["pv_done"]:
+                raise ProtocolError(f"P or O touched for tile {g} before P V of tile {g - 1} finished")
+            if rescale[g]:
+                yield "rescale"
+            st["P"][x] = g
+            bars["PF"].arrive(128)
+            if j == nkv - 1 and x == 0:
+                hs = u % cfg.hand
+                prev = st["hand"].get(hs)
+                if prev is not None and prev not in st["hand_read"]:
+                    raise ProtocolError(f"hand-over slot {hs} of unit {prev} overwritten by unit {u} before "
+                                        f"the epilogue read it")
+                st["hand"][hs] = u
+                bars[f"LF{hs}"].arrive(128)
+
+    def epilogue():
+        g_end = 0
+        for u, nkv in enumerate(units):
+            g_end += nkv
+            yield from wait("OFIN", u & 1, u)
+            if not all(t in st["pv_done"] for t in range(g_end - nkv, g_end)):
+                raise ProtocolError(f"epilogue of unit {u} before its last P V finished")
+            hs = u % cfg.hand
+            yield from wait(f"LF{hs}", (u // cfg.hand) & 1, u // cfg.hand)
+            if st["hand"].get(hs) != u:
+                raise ProtocolError(f"hand-over of unit {u} overwritten before the epilogue read it")
+            for _ in range(rng.randint(0, 3)):
+                yield "epilogue"
+            st["hand_read"].add(u)
+            for _ in range(rng.randint(1, 8)):
+                yield "epilogue"
+            st["O_unit"] = "free"
+            bars["OF"].arrive(128)
+
+    roles = {"producer": producer(), "qk": qk_issuer(), "pv": pv_issuer(), "softmax0": softmax_group(0),
+             "softmax1": softmax_group(1), "epilogue": epilogue()}
+    done, idle = set(), 0
+    while len(done) < len(roles):
+        progressed = False
+        for fk in rng.sample(["qk", "pv"], 2):
             f = fifos[fk]
             if not f:
                 continue

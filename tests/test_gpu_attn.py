@@ -12,7 +12,7 @@ from bf16_causal_prefill_fp8_b200 import zyfa
 from oracle import oracle as orc
 
 from helpers import (RESCALE_LOG2, ROW_TOL_BF16, ROW_TOL_FP8, ROW_TOL_FP8_MODEL, TOL_BF16, TOL_FP8, TOL_FP8_MODEL,
-                     bf16_round, check_local, fp8_references, inputs, run_bf16, run_fp8)
+                     bf16_round, check_local, fp8_kv_tile, fp8_references, inputs, run_bf16, run_fp8)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,11 +72,12 @@ def test_fp8_block_scales_engaged(q_gain, kind):
 def test_deferred_reference_max_on_growing_scores():
     """Scores that jump past the kernel's deferral bound (64 binades: a
     rescale), then ~33 binades above the reference (deferred: block shifts
-    below 0 and E8M0 scales above 1), fall, then ~78 above it (rescaled): FP8
+    below 0 and E8M0 scales above 1), fall, then ~78 above it (rescaled), one
+    level per KV tile of the FP8 kernel: FP8
     against fp64 attention and the CPU replay with the same deferral rule;
     BF16 on the same values."""
     from test_oracle_pins import _growing_score_case
-    qc, kc, vc, qs, ks, vs = _growing_score_case(21, RESCALE_LOG2)
+    qc, kc, vc, qs, ks, vs = _growing_score_case(21, RESCALE_LOG2, fp8_kv_tile(128))
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     o = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs))
     torch.cuda.synchronize()
@@ -141,7 +142,7 @@ def test_fp8_exact_p_ablation(shape):
     torch.cuda.synchronize()
     o = o.float().cpu().numpy().astype(np.float64)
     ref, _ = fp8_references(codes)
-    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, p_mode=2, rescale_log2=RESCALE_LOG2)
+    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, p_mode=2, rescale_log2=RESCALE_LOG2, kv_tile=fp8_kv_tile(Dqk))
     e_ref, e_model, e_lean = orc.rel_fro(o, ref), orc.rel_fro(o, model), orc.rel_fro(o_lean, ref)
     print(f"exact-P {shape}: vs fp64 {e_ref:.3e}  vs exact-P model {e_model:.3e}  (Lean P vs fp64 {e_lean:.3e})")
     assert e_ref <= TOL_FP8 and e_model <= TOL_FP8_MODEL
@@ -174,7 +175,8 @@ def test_lse_output(shape):
     o8b, lse8 = zyfa.attn_fwd(dev(qc), dev(kc), dev(vc), q_scale=dev(qs), k_scale=dev(ks), v_scale=dev(vs), lse=True)
     torch.cuda.synchronize()
     assert np.array_equal(o8b.float().cpu().numpy().astype(np.float64), o8)
-    _, lse_model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=RESCALE_LOG2, return_lse=True)
+    _, lse_model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rescale_log2=RESCALE_LOG2, return_lse=True,
+                                 kv_tile=fp8_kv_tile(Dqk))
     deq = [orc.dequantize(x, sc) for x, sc in codes]
     lse_ref = orc.attention_lse(deq[0], deq[1])
     g = lse8.cpu().numpy()

@@ -15,7 +15,7 @@ from bf16_causal_prefill_fp8_b200 import synth, zyfa
 from oracle import oracle as orc
 
 from helpers import (RESCALE_LOG2, ROW_TOL_BF16, ROW_TOL_FP8, ROW_TOL_FP8_MODEL, TOL_BF16, TOL_FP8,
-                     TOL_FP8_MODEL, check_local, tile_rows)
+                     TOL_FP8_MODEL, check_local, fp8_kv_tile, tile_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +48,8 @@ def test_full_size_sampled_parity(wl):
     ref8 = orc.attention(*deq, rows=rows)
     del deq
     (qc, qs), (kc, ks), (vc, vs) = codes
-    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rows=rows, rescale_log2=RESCALE_LOG2)
+    model = orc.fp8_model(qc, kc, vc, qs, ks, vs, rows=rows, rescale_log2=RESCALE_LOG2,
+                          kv_tile=fp8_kv_tile(qc.shape[3]))
     got8 = o8.float().cpu().numpy()[:, rows].astype(np.float64)
     err8, err8m = orc.rel_fro(got8, ref8), orc.rel_fro(got8, model)
     refb = orc.attention(*[x.astype(np.float64) for x in xs], rows=rows)

@@ -14,7 +14,7 @@ import torch
 from bf16_causal_prefill_fp8_b200 import synth, zyfa
 from oracle import oracle as orc
 
-from helpers import RESCALE_LOG2, TOL_BF16, TOL_FP8, TOL_FP8_MODEL, bf16_round
+from helpers import RESCALE_LOG2, TOL_BF16, TOL_FP8, TOL_FP8_MODEL, bf16_round, fp8_kv_tile
 
 pytestmark = pytest.mark.gpu
 
@@ -87,7 +87,8 @@ def test_fp8_varlen_parity_and_equal_to_single_sequence(lens, shape, hadamard):
     seq = np.repeat(np.arange(len(lens)), lens)
     deq = [table[c] * s_[seq][:, :, None].astype(np.float64) for c, s_ in ((rqc, rqs), (rkc, rks), (rvc, rvs))]
     ref = orc.attention_varlen(*deq, cu)
-    model = orc.fp8_model_varlen(rqc, rkc, rvc, rqs, rks, rvs, cu, rescale_log2=RESCALE_LOG2)
+    model = orc.fp8_model_varlen(rqc, rkc, rvc, rqs, rks, rvs, cu, rescale_log2=RESCALE_LOG2,
+                                 kv_tile=fp8_kv_tile(rqc.shape[2]))
     got = o.float().cpu().numpy().astype(np.float64)
     for s, r0, r1 in spans(lens):
         err, err_m = orc.rel_fro(got[r0:r1], ref[r0:r1]), orc.rel_fro(got[r0:r1], model[r0:r1])

@@ -5,7 +5,7 @@ import random
 
 import pytest
 
-from protocol_model import BF16_D128, BF16_D192, FP8, ProtocolError, random_units, run
+from protocol_model import BF16_D128, BF16_D192, FP8, WIDE, ProtocolError, random_units, run, run_wide
 
 CONFIGS = {"fp8": FP8, "bf16_d128": BF16_D128, "bf16_d192": BF16_D192}
 
@@ -47,3 +47,27 @@ def test_two_producer_variant_protocol_holds(name):
     for seed in range(80):
         rng = random.Random(seed)
         run(random_units(rng), cfg, seed, p_rescale=(0.0, 0.3, 0.9)[seed % 3], two_producers=True)
+
+
+def test_wide_tile_protocol_holds_on_random_schedules():
+    # the FP8 kernel with 256-key tiles: one S and one P buffer shared by both
+    # softmax groups, the tile max exchanged under one barrier
+    for seed in range(120):
+        rng = random.Random(seed)
+        run_wide(random_units(rng), WIDE, seed, p_rescale=(0.0, 0.3, 0.9)[seed % 3])
+
+
+@pytest.mark.parametrize("mutation", ["no_sc_wait", "no_mx_wait", "no_pe_wait"])
+def test_wide_model_catches_planted_mistakes(mutation):
+    with pytest.raises(ProtocolError):
+        for seed in range(200):
+            rng = random.Random(seed)
+            run_wide(random_units(rng), WIDE, seed, mutation=mutation)
+
+
+def test_wide_model_catches_a_short_hand_over_ring():
+    import dataclasses
+    with pytest.raises(ProtocolError):
+        for seed in range(400):
+            rng = random.Random(seed)
+            run_wide(random_units(rng), dataclasses.replace(WIDE, hand=1), seed)
