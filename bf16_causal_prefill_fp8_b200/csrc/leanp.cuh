@@ -21,15 +21,15 @@
 // s is the raw fp32 score (sum of products of e4m3 values), m the reference
 // row maximum after this key tile and bmax the maximum of the element's 64-key
 // block.  The reference max is deferred: it moves only when a tile's max
-// exceeds it by more than 8 binades, so a block max may lie above m by up to
-// that much, (bmax - m) A <= 64, and then j = 8 + floor of a negative number
-// is 0..7.  Precondition: s <= bmax and j >= 0, or s = -inf for a masked key.
-// Then the block max lands at u = 120 - 8 frac(((m - bmax) A) / 8), in
-// (112, 120] (one lower where the fp32 steps round across an integer), every
-// other u is below it, and the code never exceeds 126 (127 would be NaN; the
-// device code does not clamp at 126 and relies on this bound).  The weight
-// the matrix unit applies is value(code) * 2^-j: E8M0 scale code 127 - j,
-// at most 127 (2^0) for j >= 0.
+// exceeds it by more than 64 binades, so a block max may lie above m by up to
+// that much, (bmax - m) A <= 512, and then j = 8 + floor of a negative number
+// is -56..7.  Precondition: s <= bmax (or s = -inf for a masked key) and
+// j >= -56.  Then the block max lands at u = 120 - 8 frac(((m - bmax) A) / 8),
+// in (112, 120] (one lower where the fp32 steps round across an integer),
+// every other u is below it, and the code never exceeds 126 (127 would be
+// NaN; the device code does not clamp at 126 and relies on this bound).  The
+// weight the matrix unit applies is value(code) * 2^-j: E8M0 scale code
+// 127 - j, in 1 .. 183 (2^-126 .. 2^56) for j in -56 .. 126.
 #pragma once
 #include <cstdint>
 

@@ -312,12 +312,14 @@ int zyfa_checked_build(void);
  *   B       = fma(-m[i], A[i], 56 + 8 j[i])
  *   code[i] = masked[i] ? 0 : trunc(max(fma(s[i], A[i], B), 0))   (e4m3 code)
  * (the-ai.news "Zyphra presenteert ZYFA", "Drie technieken ..."; spke.com
- * "Lean P").  Precondition, as inside the kernel: s <= bmax and j >= 0, or
- * s = -inf.  The kernel's reference max m is deferred (it moves only when a
- * key tile's max exceeds it by more than 8 binades), so bmax may exceed m by
- * up to 64 / A and j then lies in 0..7; the block max lands in the top binade
- * (u in (112, 120]) for every j.  Outside the precondition (u >= 127) the
- * device functions do not clamp at 126 and the code is unspecified.
+ * "Lean P").  Precondition, as inside the kernel: s <= bmax, or s = -inf,
+ * and j >= -56.  The kernel's reference max m is deferred (it moves only when
+ * a key tile's max exceeds it by more than 64 binades, (tmax - m) A > 512),
+ * so bmax may exceed m by up to 512 / A and j then lies in -56..8; a
+ * negative j means an E8M0 scale 127 - j above 127 (a weight factor 2^-j
+ * above 1).  The block max lands in the top binade (u in (112, 120]) for
+ * every j.  Outside the precondition (u >= 127) the device functions do not
+ * clamp at 126 and the code is unspecified.
  *   s, m, bmax, A: fp32 [n]; masked: uint8 [n] or NULL; code: uint8 [n];
  *   j: int32 [n] or NULL.  n >= 0.  Errors: NULL_PTR, BAD_SHAPE, CUDA.
  */

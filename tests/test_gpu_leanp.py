@@ -75,10 +75,11 @@ def _deferred_case(rng, n, jt):
 
 
 def test_leanp_deferred_reference_max_every_shift():
-    # every block shift j the kernel can produce, 0..126: byte-exact codes and
-    # shifts, the deferred regime (block max above m, j = 0..7) included
+    # every block shift j the kernel can produce, -56..126: byte-exact codes
+    # and shifts, the deferred regime (block max up to 64 binades above m,
+    # j = -56..7) included
     rng = np.random.default_rng(33)
-    parts = [_deferred_case(rng, 2048, jt) for jt in range(0, 126)]
+    parts = [_deferred_case(rng, 2048, jt) for jt in range(-56, 126)]
     s, m, bmax, A = (np.concatenate([p[i] for p in parts]) for i in range(4))
     # the cap: blocks 118 or more binades under m
     capm = rng.normal(0, 10, 4096).astype(np.float32)
@@ -88,28 +89,33 @@ def test_leanp_deferred_reference_max_every_shift():
     bmax = np.concatenate([bmax, capb]); A = np.concatenate([A, capA])
     _compare(s, m, bmax, A)
     _, j = orc.leanp_batch(s, m, bmax, A)
-    assert set(range(0, 127)) <= set(j.tolist())
+    assert set(range(-56, 127)) <= set(j.tolist())
 
 
-def test_leanp_deferred_limit_exact():
-    # (m - bmax) A = -64 exactly (8 binades above m, the most the kernel
-    # defers): j = 0 and the block max is code 120; just past it j = -1 (the
-    # kernel moves the reference before that happens; the functions still agree)
+@pytest.mark.parametrize("binades", [8, 64])
+def test_leanp_deferred_limit_exact(binades):
+    # (m - bmax) A = -8 binades exactly (64 binades above m is the most the
+    # kernel defers): j = 8 - binades and the block max is code 120; just
+    # past it j is one lower (for 64 binades the kernel moves the reference
+    # before that happens; the functions still agree)
     n = 2048
     A = np.full(n, 1.0, np.float32)
     m = np.full(n, 10.0, np.float32)
-    bmax = np.full(n, 74.0, np.float32)
-    s = np.linspace(-60.0, 74.0, n).astype(np.float32)
+    top = np.float32(10.0 + 8.0 * binades)
+    bmax = np.full(n, top, np.float32)
+    s = np.linspace(top - 134.0, top, n).astype(np.float32)
     _compare(s, m, bmax, A)
     code, j = orc.leanp_batch(s, m, bmax, A)
-    assert np.all(j == 0) and code[-1] == 120
-    bmax2 = np.full(n, 74.5, np.float32)
-    s2 = np.minimum(s, np.float32(74.5))
+    assert np.all(j == 8 - binades) and code[-1] == 120
+    bmax2 = np.full(n, top + np.float32(0.5), np.float32)
+    s2 = np.minimum(s, bmax2)
     _compare(s2, m, bmax2, A)
+    _, j2 = orc.leanp_batch(s2, m, bmax2, A)
+    assert np.all(j2 == 7 - binades)
     # powers of two of A and m: every code 0..120 reached exactly on its integer
     u = np.arange(0, 121, dtype=np.float32)
-    s3 = (u - np.float32(120.0) + np.float32(74.0)).astype(np.float32)
+    s3 = (u - np.float32(120.0) + top).astype(np.float32)
     k = s3.size
-    c3, _ = orc.leanp_batch(s3, np.full(k, 10.0, np.float32), np.full(k, 74.0, np.float32), np.ones(k, np.float32))
+    c3, _ = orc.leanp_batch(s3, np.full(k, 10.0, np.float32), np.full(k, top, np.float32), np.ones(k, np.float32))
     assert np.array_equal(c3, u.astype(np.uint8))
-    _compare(s3, np.full(k, 10.0, np.float32), np.full(k, 74.0, np.float32), np.ones(k, np.float32))
+    _compare(s3, np.full(k, 10.0, np.float32), np.full(k, top, np.float32), np.ones(k, np.float32))

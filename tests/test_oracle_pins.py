@@ -191,12 +191,15 @@ def test_gqa_single_kv_head_equals_replicated_mha():
 
 def test_leanp_zero_scores_give_8j_plus_56():
     # s = m = 0: u = 56 + 8j exactly, so the code is 8j + 56 while that is a
-    # finite e4m3 code (j <= 8) and the clamp value 126 beyond
+    # finite e4m3 code (-7 <= j <= 8), the clamp value 126 above and 0 below
+    # (u < 0: the shifts of a block far above the deferred reference)
     for A in [1e-4, 0.37, 5.0]:
-        for j in range(0, 9):
+        for j in range(-7, 9):
             assert orc.leanp_code(0.0, 0.0, A, j) == 8 * j + 56
         for j in [9, 20, 126]:
             assert orc.leanp_code(0.0, 0.0, A, j) == 126
+        for j in [-8, -20, -56]:
+            assert orc.leanp_code(0.0, 0.0, A, j) == 0
         assert orc.leanp_block_shift(0.0, 0.0, A) == 8
         assert orc.leanp_code(0.0, 0.0, A, 8) == 120
     assert orc.leanp_code(5.0, 5.0, 0.25, 8, masked=True) == 0
@@ -229,8 +232,8 @@ def test_leanp_weight_inside_mitchell_band():
     m = rng.uniform(-30, 30, n).astype(np.float32)
     A = np.exp(rng.uniform(np.log(1e-3), np.log(20), n)).astype(np.float32)
     # m - bmax in binades (units of 8/A).  Negative gaps are the deferred
-    # reference max: a block up to 8 binades above the reference m (j = 0..7)
-    gap = rng.uniform(-8, 100, n).astype(np.float32)
+    # reference max: a block up to 64 binades above the reference m (j = -56..7)
+    gap = rng.uniform(-64, 100, n).astype(np.float32)
     bmax = (m - gap * np.float32(8.0) / A).astype(np.float32)
     frac = rng.uniform(0, 1, n)
     s = (bmax - frac * np.float32(40.0) / A).astype(np.float32)   # up to 5 binades under bmax
@@ -247,15 +250,35 @@ def test_leanp_weight_inside_mitchell_band():
     # the block max lands in the top binade: u in (112, 120], so its code is
     # in [112, 120] (one lower where the fp32 steps round across an integer)
     cmax, _ = orc.leanp_batch(bmax, m, bmax, A)
-    cap = (js < 126) & (js >= 0)
+    cap = (js < 126) & (js >= -56)
     assert np.all((cmax[cap] >= 111) & (cmax[cap] <= 120))
     assert np.mean(cmax[cap] >= 112) > 0.99
-    # the deferred regime (block max above m) is exercised, with every j 0..7
+    # the deferred regime (block max above m) is exercised, with every j -56..7
     above = bmax > m
-    assert above.mean() > 0.05
-    assert set(range(0, 8)) <= set(js[above].tolist())
+    assert above.mean() > 0.2
+    assert set(range(-56, 8)) <= set(js[above].tolist())
     assert np.all(js[above] <= 8)
     assert np.all((cmax[above & cap] >= 111) & (cmax[above & cap] <= 120))
+
+
+def test_leanp_weight_doubles_when_the_reference_drops_one_binade():
+    """Moving the reference down by exactly one binade (8/A) lowers the block
+    shift j by one and leaves u, hence the code, unchanged, so the decoded
+    weight value(code) * 2^-j doubles exactly: pins the sign of j in the
+    weight and the row offset 56 + 8j, above and below the reference, with
+    exact arithmetic (A = 1, integer scores)."""
+    s = np.arange(-300, 41, dtype=np.float32)
+    bmax = np.full_like(s, 40.0)
+    A = np.ones_like(s)
+    vals = orc.e4m3_values()
+    for m0 in (96.0, 40.0, 8.0, -200.0, -472.0):   # block 7 binades below .. 64 binades above m
+        c0, j0 = orc.leanp_batch(s, np.full_like(s, m0), bmax, A)
+        c1, j1 = orc.leanp_batch(s, np.full_like(s, m0 - 8.0), bmax, A)
+        assert np.all(j1 == j0 - 1) and np.array_equal(c0, c1)
+        w0 = vals[c0] * np.exp2(-j0.astype(np.float64))
+        w1 = vals[c1] * np.exp2(-j1.astype(np.float64))
+        assert np.array_equal(w1, 2.0 * w0)
+        assert c0[-1] == 120   # the block max on its integer lands on code 120
 
 
 def test_leanp_block_shift_cap():
