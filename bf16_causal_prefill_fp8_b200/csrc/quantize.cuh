@@ -28,7 +28,8 @@
 namespace zyfa {
 
 constexpr int kQuantThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 4;        // rotated paths: rows in flight per warp
+constexpr int kUnrollPlain = 4;   // plain paths: 16-byte loads in flight per thread
 constexpr float kFwhtNorm = 0.08838834764831844055f;   // 2^-3.5 rounded to fp32
 
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
@@ -54,6 +55,16 @@ __device__ __forceinline__ float div_by_scale(float x, float s, float rc) {
   const float q0 = __fmul_rn(x, rc);
   const float r = __fmaf_rn(-q0, s, x);
   return __fmaf_rn(r, rc, q0);
+}
+
+// Division by a runtime divisor d without a divide: m = ceil(2^64 / d)
+// (m = 0 for d = 1), and for n < 2^32 the high word of n * m is floor(n / d)
+// exactly (n m / 2^64 exceeds n / d by n (m - 2^64/d) / 2^64 < n / 2^64 < 1/d,
+// which cannot carry the quotient past the next integer).  The kernels use it
+// for the head index of a 16-byte vector, once per vector.
+__host__ __device__ inline uint64_t div_magic(uint32_t d) { return d <= 1u ? 0ull : ~0ull / d + 1ull; }
+__device__ __forceinline__ uint32_t div_by_magic(uint32_t n, uint64_t m) {
+  return m ? static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(n), m)) : n;
 }
 
 __device__ __forceinline__ float scale_reciprocal(float s) {
@@ -151,7 +162,19 @@ struct QuantArgs {
   float* scale;            // [B*H]: amax accumulator, then the scales
   int S, H, D;
   int rows_per_cta;        // sequence rows of one batch per CTA
+  uint64_t mg_vph;         // div_magic(16-byte vectors per head row: D / 8 bf16, D / 4 fp32)
+  uint64_t mg_h;           // div_magic(H)
 };
+
+// The head of 16-byte vector vi of a chunk (chunks start on whole rows).
+__device__ __forceinline__ uint32_t vec_head(const QuantArgs& a, uint32_t vi) {
+  const uint32_t q = div_by_magic(vi, a.mg_vph);
+  return q - static_cast<uint32_t>(a.H) * div_by_magic(q, a.mg_h);
+}
+// The head of row-vector v (one head's D elements) of a chunk.
+__device__ __forceinline__ uint32_t row_head(const QuantArgs& a, uint32_t v) {
+  return v - static_cast<uint32_t>(a.H) * div_by_magic(v, a.mg_h);
+}
 
 // Step 2 for sequence-row chunk `chunk` of batch b (one CTA); s_amax: [H].
 template <typename T, bool HAD>
@@ -182,7 +205,7 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
         for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[u][i]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) atomicMax(&s_amax[(v0 + u) % a.H], __float_as_uint(mx));
+        if (lane == 0) atomicMax(&s_amax[row_head(a, v0 + u)], __float_as_uint(mx));
       }
     }
   } else if (HAD) {
@@ -209,23 +232,23 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         const int v = v0 + 2 * u + half;
-        if (li == 0 && v < nvec) atomicMax(&s_amax[v % a.H], __float_as_uint(mx));
+        if (li == 0 && v < nvec) atomicMax(&s_amax[row_head(a, v)], __float_as_uint(mx));
       }
     }
   } else {
     constexpr int N = Vec<T>::N;
-    const uint32_t vpr = HD / N, vph = a.D / N;        // 16-byte vectors per row / per head
+    const uint32_t vpr = HD / N;                       // 16-byte vectors per row
     const uint32_t nvec = static_cast<uint32_t>(r1 - r0) * vpr;
     const uint4* src = reinterpret_cast<const uint4*>(base);
-    for (uint32_t v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * kUnroll) {
-      uint4 raw[kUnroll];
+    for (uint32_t v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * kUnrollPlain) {
+      uint4 raw[kUnrollPlain];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kUnrollPlain; ++u) {
         const uint32_t vi = v0 + u * blockDim.x;
         if (vi < nvec) raw[u] = __ldg(src + vi);
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kUnrollPlain; ++u) {
         const uint32_t vi = v0 + u * blockDim.x;
         if (vi >= nvec) break;
         float x[N];
@@ -233,7 +256,7 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
         float mx = 0.0f;
 #pragma unroll
         for (int i = 0; i < N; ++i) mx = fmaxf(mx, fabsf(x[i]));
-        atomicMax(&s_amax[(vi % vpr) / vph], __float_as_uint(mx));
+        atomicMax(&s_amax[vec_head(a, vi)], __float_as_uint(mx));
       }
     }
   }
@@ -274,7 +297,7 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
         if (v0 + u >= nrow) break;
         fwht192_warp(x[u], lane);
         if (lane >= 24) continue;
-        const int hh = (v0 + u) % a.H;
+        const int hh = row_head(a, v0 + u);
         const float sc = s_sc[hh], rc = s_rc[hh];
         uint32_t w[2];
 #pragma unroll
@@ -305,7 +328,7 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
         fwht128_half(x[u], li);
         const int v = v0 + 2 * u + half;
         if (v >= nvec) continue;
-        const int hh = v % a.H;
+        const int hh = row_head(a, v);
         const float sc = s_sc[hh], rc = s_rc[hh];
         uint32_t w[2];
 #pragma unroll
@@ -318,23 +341,23 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
     }
   } else {
     constexpr int N = Vec<T>::N;
-    const uint32_t vpr = HD / N, vph = a.D / N;
+    const uint32_t vpr = HD / N;
     const uint32_t nvec = static_cast<uint32_t>(r1 - r0) * vpr;
     const uint4* src = reinterpret_cast<const uint4*>(base);
-    for (uint32_t v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * kUnroll) {
-      uint4 raw[kUnroll];
+    for (uint32_t v0 = threadIdx.x; v0 < nvec; v0 += blockDim.x * kUnrollPlain) {
+      uint4 raw[kUnrollPlain];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kUnrollPlain; ++u) {
         const uint32_t vi = v0 + u * blockDim.x;
         if (vi < nvec) raw[u] = __ldg(src + vi);
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kUnrollPlain; ++u) {
         const uint32_t vi = v0 + u * blockDim.x;
         if (vi >= nvec) break;
         float x[N];
         Vec<T>::unpack(raw[u], x);
-        const uint32_t hh = (vi % vpr) / vph;
+        const uint32_t hh = vec_head(a, vi);
         const float sc = s_sc[hh], rc = s_rc[hh];
         uint32_t w[N / 4];
 #pragma unroll

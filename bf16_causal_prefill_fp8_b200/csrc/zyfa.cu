@@ -247,6 +247,12 @@ int launch_attn_wide_varlen(const void* q, const void* k, const void* v, void* o
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
+// The divisors the prepass kernels need per 16-byte vector, as multipliers.
+void set_div_magic(QuantArgs& t, int in_dtype) {
+  t.mg_vph = div_magic(static_cast<uint32_t>(t.D / (in_dtype == ZYFA_BF16 ? 8 : 4)));
+  t.mg_h = div_magic(static_cast<uint32_t>(t.H));
+}
+
 // Sequence rows per prepass CTA: at most 2^30 elements of one batch entry
 // (the kernels count a chunk's rows and 16-byte vectors in 32 bits).
 long long prepass_rows(long long rows, int H, int D) {
@@ -407,6 +413,7 @@ extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* sc
   a.scale = scale;
   a.S = S; a.H = H; a.D = D;
   a.rows_per_cta = static_cast<int>(prepass_rows((S + chunks - 1) / chunks, H, D));
+  set_div_magic(a, in_dtype);
   const dim3 grid(static_cast<unsigned>((S + a.rows_per_cta - 1) / a.rows_per_cta), static_cast<unsigned>(B));
   const size_t shm = static_cast<size_t>(H) * 8;   // amax, or scale and its reciprocal, per head
   if (cudaMemsetAsync(scale, 0, static_cast<size_t>(B) * H * sizeof(float), st) != cudaSuccess)
@@ -473,6 +480,7 @@ extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, in
     t.scale = scs[i];
     t.S = S; t.H = Hs[i]; t.D = Ds[i];
     t.rows_per_cta = static_cast<int>(prepass_rows((S + chunks - 1) / chunks, Hs[i], Ds[i]));
+    set_div_magic(t, in_dtype);
     a.had[i] = (i < 2) ? hadamard_qk : 0;
     const long long cols = a.first[i] + (static_cast<long long>(S) + t.rows_per_cta - 1) / t.rows_per_cta;
     if (cols > 0x7fffffffll) return ZYFA_ERR_BAD_SHAPE;
@@ -584,6 +592,7 @@ static int quantize_varlen_n(int n, const void* const* xs, void* const* outs, fl
     t.S = 0;
     t.H = Hs[i]; t.D = Ds[i];
     t.rows_per_cta = static_cast<int>(prepass_rows((mean_len + chunks - 1) / chunks, Hs[i], Ds[i]));
+    set_div_magic(t, in_dtype);
     q3.had[i] = had[i];
     long long cols = 0;   // every sequence's chunks, in order
     for (int sq = 0; sq < nseq; ++sq) cols += (cu[sq + 1] - cu[sq] + t.rows_per_cta - 1) / t.rows_per_cta;

@@ -5,7 +5,8 @@
 Each iteration launches, in order: zyfa_quantize_qkv (zero, amax, codes and
 finalize kernels over Q, K and V together), the FP8 attention kernel, then the
 BF16 attention kernel on the same bf16 inputs (for a packed-batch workload,
-the varlen forms of the same three calls).  Prints nothing but a completion line; timing
+the varlen forms of the same three calls).  --exact-p swaps the FP8 attention
+for the exact-P ablation (fixed-length workloads).  Prints nothing but a completion line; timing
 numbers come from bench.py, never from a profiled run.
 """
 import argparse
@@ -22,6 +23,8 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--hadamard", action="store_true")
     ap.add_argument("--only", choices=["all", "fp8", "bf16"], default="all")
+    ap.add_argument("--exact-p", action="store_true",
+                    help="the FP8 attention launch is the exact-P ablation (e4m3(ex2(.)) instead of Lean P)")
     args = ap.parse_args()
     if args.workload in synth.VARLEN_WORKLOADS:
         # packed batch: the varlen prepass and varlen attention launches
@@ -43,7 +46,10 @@ def main():
     for _ in range(args.iters):
         if args.only in ("all", "fp8"):
             (cq, sq), (ck, sk), (cv, sv) = quant()
-            attn(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv)
+            if args.exact_p:
+                attn(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv, exact_p=True)
+            else:
+                attn(cq, ck, cv, q_scale=sq, k_scale=sk, v_scale=sv)
         if args.only in ("all", "bf16"):
             attn(dq, dk, dv)
     torch.cuda.synchronize()
