@@ -50,8 +50,11 @@ __device__ __forceinline__ float head_scale(float amax) {
 // RN(q0 + residual * rc) is the correctly rounded quotient.  rc == 0 marks a
 // scale too small or too large for the reciprocal to stay normal: plain
 // division.  The quotients here are at most 448 in magnitude.
+// FAST: every head of the CTA has a normal reciprocal, so the correction path
+// runs alone (the CTA decides once; no division code in the loop).
+template <bool FAST>
 __device__ __forceinline__ float div_by_scale(float x, float s, float rc) {
-  if (rc == 0.0f) return __fdiv_rn(x, s);
+  if (!FAST) return __fdiv_rn(x, s);
   const float q0 = __fmul_rn(x, rc);
   const float r = __fmaf_rn(-q0, s, x);
   return __fmaf_rn(r, rc, q0);
@@ -266,16 +269,9 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
 }
 
 // Step 3 for one chunk; reads the finished amax of each (b, h); s_sc: [H].
-template <typename T, bool HAD>
-__device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, int b, float* s_sc) {
-  const int r0 = chunk * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
-  float* s_rc = s_sc + a.H;   // RN(1 / scale) per head
-  for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
-    const float sc = head_scale(a.scale[static_cast<size_t>(b) * a.H + h]);
-    s_sc[h] = sc;
-    s_rc[h] = scale_reciprocal(sc);
-  }
-  __syncthreads();
+template <typename T, bool HAD, bool FAST>
+__device__ __forceinline__ void quant_codes_loop(const QuantArgs& a, int r0, int r1, int b, const float* s_sc,
+                                                 const float* s_rc) {
   const uint32_t HD = static_cast<uint32_t>(a.H) * a.D;
   const size_t off = (static_cast<size_t>(b) * a.S + r0) * HD;
   const T* base = static_cast<const T*>(a.x) + off;
@@ -302,9 +298,9 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
         uint32_t w[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i)
-          w[i] = cvt_e4m3x2(div_by_scale(x[u][4 * i], sc, rc), div_by_scale(x[u][4 * i + 1], sc, rc)) |
-                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(x[u][4 * i + 2], sc, rc),
-                                                   div_by_scale(x[u][4 * i + 3], sc, rc))) << 16);
+          w[i] = cvt_e4m3x2(div_by_scale<FAST>(x[u][4 * i], sc, rc), div_by_scale<FAST>(x[u][4 * i + 1], sc, rc)) |
+                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale<FAST>(x[u][4 * i + 2], sc, rc),
+                                                   div_by_scale<FAST>(x[u][4 * i + 3], sc, rc))) << 16);
         *reinterpret_cast<uint2*>(obase + static_cast<size_t>(v0 + u) * 192 + 8 * lane) = make_uint2(w[0], w[1]);
       }
     }
@@ -333,9 +329,9 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
         uint32_t w[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i)
-          w[i] = cvt_e4m3x2(div_by_scale(x[u][4 * i], sc, rc), div_by_scale(x[u][4 * i + 1], sc, rc)) |
-                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(x[u][4 * i + 2], sc, rc),
-                                                   div_by_scale(x[u][4 * i + 3], sc, rc))) << 16);
+          w[i] = cvt_e4m3x2(div_by_scale<FAST>(x[u][4 * i], sc, rc), div_by_scale<FAST>(x[u][4 * i + 1], sc, rc)) |
+                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale<FAST>(x[u][4 * i + 2], sc, rc),
+                                                   div_by_scale<FAST>(x[u][4 * i + 3], sc, rc))) << 16);
         *reinterpret_cast<uint2*>(obase + static_cast<size_t>(v) * 128 + 8 * li) = make_uint2(w[0], w[1]);
       }
     }
@@ -362,14 +358,30 @@ __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, i
         uint32_t w[N / 4];
 #pragma unroll
         for (int i = 0; i < N / 4; ++i)
-          w[i] = cvt_e4m3x2(div_by_scale(x[4 * i], sc, rc), div_by_scale(x[4 * i + 1], sc, rc)) |
-                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(x[4 * i + 2], sc, rc),
-                                                   div_by_scale(x[4 * i + 3], sc, rc))) << 16);
+          w[i] = cvt_e4m3x2(div_by_scale<FAST>(x[4 * i], sc, rc), div_by_scale<FAST>(x[4 * i + 1], sc, rc)) |
+                 (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale<FAST>(x[4 * i + 2], sc, rc),
+                                                   div_by_scale<FAST>(x[4 * i + 3], sc, rc))) << 16);
         if constexpr (N == 8) *reinterpret_cast<uint2*>(obase + static_cast<size_t>(vi) * 8) = make_uint2(w[0], w[1]);
         else *reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(vi) * 4) = w[0];
       }
     }
   }
+}
+
+template <typename T, bool HAD>
+__device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, int b, float* s_sc) {
+  const int r0 = chunk * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
+  float* s_rc = s_sc + a.H;   // RN(1 / scale) per head
+  int fast = 1;
+  for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+    const float sc = head_scale(a.scale[static_cast<size_t>(b) * a.H + h]);
+    const float rc = scale_reciprocal(sc);
+    s_sc[h] = sc;
+    s_rc[h] = rc;
+    if (rc == 0.0f) fast = 0;
+  }
+  if (__syncthreads_and(fast)) quant_codes_loop<T, HAD, true>(a, r0, r1, b, s_sc, s_rc);
+  else quant_codes_loop<T, HAD, false>(a, r0, r1, b, s_sc, s_rc);
 }
 
 // One tensor: grid = (ceil(S / rows_per_cta), B), block = kQuantThreads,

@@ -2,8 +2,9 @@
 must match byte for byte, with and without the Hadamard rotation."""
 import numpy as np
 import pytest
+import torch
 
-from bf16_causal_prefill_fp8_b200 import synth
+from bf16_causal_prefill_fp8_b200 import synth, zyfa
 from oracle import oracle as orc
 
 from helpers import bf16_round, quantize_gpu
@@ -87,3 +88,25 @@ def test_quantize_quotients_at_e4m3_midpoints():
     assert np.array_equal(scale.cpu().numpy().view(np.uint32), rs.view(np.uint32))
     got = codes.cpu().numpy()
     assert np.array_equal(got, rc), f"{np.count_nonzero(got != rc)} codes differ"
+
+
+@pytest.mark.parametrize("tiny", [1e-37, 3e-39])
+def test_quantize_tiny_head_uses_plain_division(tiny):
+    """A head whose scale amax/448 has no normal reciprocal (below 2^-120, down
+    into fp32 subnormals) makes its CTAs take the IEEE-division path for every
+    head they hold; codes and scales stay byte-exact, for that head and its
+    normal neighbours, in the one-tensor and the fused Q/K/V prepass."""
+    x = synth.gaussian(23, 2, (2, 260, 3, 128)).astype(np.float32)
+    x[:, :, 1] *= np.float32(tiny)
+    codes, scale = quantize_gpu(x)
+    rc, rs = orc.quantize(x)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert float(rs.reshape(2, 3)[0, 1]) < 2.0 ** -120
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    got = zyfa.quantize_qkv(t(x), t(x[:, :, :1]), t(x[:, :, 1:2]))
+    torch.cuda.synchronize()
+    for (c, sc), xi in zip(got, (x, x[:, :, :1], x[:, :, 1:2])):
+        rci, rsi = orc.quantize(np.ascontiguousarray(xi))
+        assert np.array_equal(sc.cpu().numpy().view(np.uint32), rsi.view(np.uint32))
+        assert np.array_equal(c.cpu().numpy(), rci)
