@@ -93,11 +93,10 @@ template <> struct Vec<float> {
   }
 };
 
-// Rotated path, half a warp per row: lane l of a half holds elements
-// 8l .. 8l+7 (16-byte bf16 / 32-byte fp32 loads).  Butterflies of stride
-// 1, 2, 4 in registers and 8 .. 64 across the 16 lanes of the half, in that
-// order (the order the rotation is defined with), each stage the fp32 sum and
-// difference of its pair; four shuffles per element.
+// Eight consecutive elements of a row as fp32 (one 16-byte bf16 load or two
+// fp32 loads).  The rotation is defined by butterflies of stride 1, 2, 4, ...
+// in that order, each stage the fp32 sum and difference of its pair; every
+// layout below keeps that order.
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float (&v)[8]);
 template <>
@@ -111,24 +110,40 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
   Vec<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4*>(p)), v);
 }
 
-__device__ __forceinline__ void fwht128_half(float (&x)[8], int li) {
+// Rotated rows of D = 128, four lanes per row: lane q of a quad holds
+// elements 32q .. 32q+31 (four 16-byte bf16 / eight fp32 loads).  Butterflies
+// of stride 1 .. 16 in registers, then 32 and 64 across the quad (lane xor 1,
+// xor 2): two shuffles per element.
+constexpr int kQuadRows = 1;   // rows in flight per quad lane
+template <typename T>
+__device__ __forceinline__ void load32(const T* p, float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float t[8];
+    load8<T>(p + 8 * c, t);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[8 * c + i] = t[i];
+  }
+}
+
+__device__ __forceinline__ void fwht128_quad(float (&x)[32], int lq) {
   float a, b;
 #pragma unroll
-  for (int st = 1; st < 8; st <<= 1)
+  for (int st = 1; st < 32; st <<= 1)
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 32; ++i)
       if ((i & st) == 0) { a = x[i]; b = x[i + st]; x[i] = a + b; x[i + st] = a - b; }
 #pragma unroll
-  for (int sh = 1; sh < 16; sh <<= 1) {   // strides 8, 16, 32, 64
-    const bool upper = (li & sh) != 0;
+  for (int sh = 1; sh < 4; sh <<= 1) {   // strides 32, 64
+    const bool upper = (lq & sh) != 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 32; ++i) {
       const float o = __shfl_xor_sync(0xffffffffu, x[i], sh);
       x[i] = upper ? (o - x[i]) : (x[i] + o);
     }
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] = x[i] * kFwhtNorm;
+  for (int i = 0; i < 32; ++i) x[i] = x[i] * kFwhtNorm;
 }
 
 // Rotated rows of D = 192 (MLA: H128 on dims 0..127, H64 on 128..191), one
@@ -213,29 +228,29 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
     }
   } else if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    const int half = lane >> 4, li = lane & 15;
-    const int nvec = (r1 - r0) * a.H;          // 128-element rows
-    for (int v0 = warp * 2 * kUnroll; v0 < nvec; v0 += nw * 2 * kUnroll) {
-      float x[kUnroll][8];
+    const int quad = lane >> 2, lq = lane & 3;
+    const int nvec = (r1 - r0) * a.H;          // 128-element rows, 8 per warp and step
+    for (int v0 = warp * 8 * kQuadRows; v0 < nvec; v0 += nw * 8 * kQuadRows) {
+      float x[kQuadRows][32];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = v0 + 2 * u + half;
-        if (v < nvec) load8<T>(base + static_cast<size_t>(v) * 128 + 8 * li, x[u]);
+      for (int u = 0; u < kQuadRows; ++u) {
+        const int v = v0 + 8 * u + quad;
+        if (v < nvec) load32<T>(base + static_cast<size_t>(v) * 128 + 32 * lq, x[u]);
         else
 #pragma unroll
-          for (int i = 0; i < 8; ++i) x[u][i] = 0.0f;
+          for (int i = 0; i < 32; ++i) x[u][i] = 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (v0 + 2 * u >= nvec) break;                  // both halves past the end
-        fwht128_half(x[u], li);
+      for (int u = 0; u < kQuadRows; ++u) {
+        if (v0 + 8 * u >= nvec) break;                  // every row of the step past the end
+        fwht128_quad(x[u], lq);
         float mx = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[u][i]));
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const int v = v0 + 2 * u + half;
-        if (li == 0 && v < nvec) atomicMax(&s_amax[row_head(a, v)], __float_as_uint(mx));
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(x[u][i]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const int v = v0 + 8 * u + quad;
+        if (lq == 0 && v < nvec) atomicMax(&s_amax[row_head(a, v)], __float_as_uint(mx));
       }
     }
   } else {
@@ -306,33 +321,35 @@ __device__ __forceinline__ void quant_codes_loop(const QuantArgs& a, int r0, int
     }
   } else if (HAD) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    const int half = lane >> 4, li = lane & 15;
+    const int quad = lane >> 2, lq = lane & 3;
     const int nvec = (r1 - r0) * a.H;
-    for (int v0 = warp * 2 * kUnroll; v0 < nvec; v0 += nw * 2 * kUnroll) {
-      float x[kUnroll][8];
+    for (int v0 = warp * 8 * kQuadRows; v0 < nvec; v0 += nw * 8 * kQuadRows) {
+      float x[kQuadRows][32];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = v0 + 2 * u + half;
-        if (v < nvec) load8<T>(base + static_cast<size_t>(v) * 128 + 8 * li, x[u]);
+      for (int u = 0; u < kQuadRows; ++u) {
+        const int v = v0 + 8 * u + quad;
+        if (v < nvec) load32<T>(base + static_cast<size_t>(v) * 128 + 32 * lq, x[u]);
         else
 #pragma unroll
-          for (int i = 0; i < 8; ++i) x[u][i] = 0.0f;
+          for (int i = 0; i < 32; ++i) x[u][i] = 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (v0 + 2 * u >= nvec) break;
-        fwht128_half(x[u], li);
-        const int v = v0 + 2 * u + half;
+      for (int u = 0; u < kQuadRows; ++u) {
+        if (v0 + 8 * u >= nvec) break;
+        fwht128_quad(x[u], lq);
+        const int v = v0 + 8 * u + quad;
         if (v >= nvec) continue;
         const int hh = row_head(a, v);
         const float sc = s_sc[hh], rc = s_rc[hh];
-        uint32_t w[2];
+        uint32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
+        for (int i = 0; i < 8; ++i)
           w[i] = cvt_e4m3x2(div_by_scale<FAST>(x[u][4 * i], sc, rc), div_by_scale<FAST>(x[u][4 * i + 1], sc, rc)) |
                  (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale<FAST>(x[u][4 * i + 2], sc, rc),
                                                    div_by_scale<FAST>(x[u][4 * i + 3], sc, rc))) << 16);
-        *reinterpret_cast<uint2*>(obase + static_cast<size_t>(v) * 128 + 8 * li) = make_uint2(w[0], w[1]);
+        uint4* dst = reinterpret_cast<uint4*>(obase + static_cast<size_t>(v) * 128 + 32 * lq);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
     }
   } else {
