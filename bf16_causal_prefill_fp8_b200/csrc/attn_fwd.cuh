@@ -692,10 +692,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // the whole 128-key row of S in one TMEM round trip; the S buffer is
         // free for the tile after next right away
         uint32_t r[128];
-        tmem_ld32p(ts, &r[0]);
-        tmem_ld32p(ts + 32, &r[32]);
-        tmem_ld32p(ts + 64, &r[64]);
-        tmem_ld32p(ts + 96, &r[96]);
+        tmem_ld64p(ts, &r[0]);
+        tmem_ld64p(ts + 64, &r[64]);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(Cf::SC0 + grp));

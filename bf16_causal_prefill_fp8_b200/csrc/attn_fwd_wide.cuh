@@ -336,10 +336,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!(ok = warp_wait(bar(W::SF), g & 1, ctl))) break;
       tc_fence_after();
       uint32_t r[128];
-      tmem_ld32p(tsg, &r[0]);
-      tmem_ld32p(tsg + 32, &r[32]);
-      tmem_ld32p(tsg + 64, &r[64]);
-      tmem_ld32p(tsg + 96, &r[96]);
+      tmem_ld64p(tsg, &r[0]);
+      tmem_ld64p(tsg + 64, &r[64]);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(W::SC));
