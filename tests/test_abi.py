@@ -17,12 +17,24 @@ def test_every_declared_symbol_is_exported(L):
     names = zyfa.declared_symbols()
     assert set(names) >= {"zyfa_attn_fwd", "zyfa_attn_fwd_lse", "zyfa_attn_fwd_fp8_exact_p", "zyfa_quantize",
                           "zyfa_quantize_qkv", "zyfa_attn_fwd_varlen", "zyfa_quantize_varlen",
-                          "zyfa_quantize_qkv_varlen", "zyfa_attn_schedule",
+                          "zyfa_quantize_qkv_varlen", "zyfa_attn_schedule", "zyfa_attn_kv_tile",
                           "zyfa_status_string",
                           "zyfa_device_status",
                           "zyfa_leanp_codes", "zyfa_selftest_wait_timeout", "zyfa_set_wait_timeout_ns"}
     for n in names:
         assert hasattr(L, n), n
+
+
+def test_kv_tile_per_dtype_and_head_dim(L):
+    # FP8 with Dqk 128 runs 256-key KV tiles; the MLA shape and BF16 128-key ones
+    assert zyfa.kv_tile(zyfa.FP8_E4M3, 128) == 256
+    assert zyfa.kv_tile(zyfa.FP8_E4M3, 192) == 128
+    assert zyfa.kv_tile(zyfa.BF16, 128) == 128
+    assert zyfa.kv_tile(zyfa.BF16, 192) == 128
+    assert L.zyfa_attn_kv_tile(7, 128) < 0
+    assert L.zyfa_attn_kv_tile(zyfa.FP8_E4M3, 64) < 0
+    with pytest.raises(zyfa.ZyfaError):
+        zyfa.kv_tile(zyfa.FP8_E4M3, 256)
 
 
 def test_status_strings(L):

@@ -56,6 +56,24 @@ def test_fp8_parity(shape):
     assert err_model <= TOL_FP8_MODEL, err_model
 
 
+@pytest.mark.parametrize("S", [255, 256, 257, 383, 384, 385, 511, 513, 640, 767])
+def test_fp8_kv_tile_edges(S):
+    """Sequence lengths around the 256-key KV tile: the last tile of a unit
+    holds the diagonal in its first half (even query tile, second half all
+    masked) or in its second half (odd query tile), and the ragged tail reads
+    zero-filled rows.  FP8 against fp64 and the replay with the kernel's own
+    KV tile; BF16 on the same values."""
+    q, k, v = inputs(51, 1, S, 4, 2, 128, 128, kind="outlier_k")
+    o, codes = run_fp8(q, k, v)
+    ref, model = fp8_references(codes)
+    e_ref, e_model = orc.rel_fro(o, ref), orc.rel_fro(o, model)
+    print(f"fp8 S={S}: vs fp64 {e_ref:.3e}  vs model {e_model:.3e}")
+    assert e_ref <= TOL_FP8 and e_model <= TOL_FP8_MODEL
+    check_local(o, model, TOL_FP8_MODEL, ROW_TOL_FP8_MODEL, f"fp8 S={S} vs model")
+    ob, deqb = run_bf16(q, k, v)
+    assert orc.rel_fro(ob, orc.attention(*deqb)) <= TOL_BF16
+
+
 @pytest.mark.parametrize("q_gain,kind", [(6.0, "gaussian"), (1.0, "outlier_k"), (12.0, "gaussian")])
 def test_fp8_block_scales_engaged(q_gain, kind):
     # peaked scores: many 64-key blocks sit far below the row max, so the
