@@ -830,7 +830,8 @@ def run_ours(args, wl):
         del pin, host_o
         torch.cuda.empty_cache()
         for wname in extra:
-            subs[wname] = run_extra(torch, zyfa, args, wname, rank, world, dev, flush, stream, peaks, barrier, mx)
+            subs[wname] = run_extra(torch, zyfa, args, wname, rank, world, dev, flush, stream, peaks, barrier, mx,
+                                    bus)
             if subs[wname].get("parity_failed"):
                 print(f"bench: parity failed on {wname}: {json.dumps(subs[wname].get('parity'))}", file=sys.stderr)
                 return 1
@@ -888,9 +889,11 @@ def run_ours(args, wl):
     return 0
 
 
-def run_extra(torch, zyfa, args, wname, rank, world, dev, flush, stream, peaks, barrier, mx):
+def run_extra(torch, zyfa, args, wname, rank, world, dev, flush, stream, peaks, barrier, mx, bus=None):
     """One of the further workloads: timed like the headline (fewer steps),
-    with its roofline and sampled parity."""
+    with its roofline and sampled parity; a fixed-length one also gets short
+    sustained legs of both FP8 kernels (Lean P and exact P) for the energy and
+    clock comparison across input kinds."""
     steps = max(3, min(args.steps, 10))
     if wname in synth.VARLEN_WORKLOADS:
         wl = varlen_workload(wname, args.seed)
@@ -927,6 +930,17 @@ def run_extra(torch, zyfa, args, wname, rank, world, dev, flush, stream, peaks, 
            "roofline": {"fp8": roofline(fl / (out["attn8"] * 1e-3) / 1e12, peaks, "fp8", fp8_kernel_name(Dqk)),
                         "bf16": roofline(fl / (out["bf16"] * 1e-3) / 1e12, peaks, "bf16",
                                          f"attn_fwd_kernel<BF16,{Dqk}>")}}
+    if args.sustained > 0:
+        sus = {}
+        for name, fn in (("fp8_lean_p", case.attn8), ("fp8_exact_p", case.attn8x)):
+            barrier()
+            r = sustained_leg(torch, fn, fl, min(args.sustained, 1.0), bus) if bus else None
+            if r:
+                r["peak"] = peaks.of("fp8", sustained=True)
+                r["frac"] = r["tflops"] / r["peak"]
+            sus[name] = r
+        barrier()
+        res["sustained"] = sus
     if world == 1:
         par, bad, _ = case.parity(args.seed, 24, True, False)
         res["parity"] = par
