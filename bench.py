@@ -424,7 +424,9 @@ def measure_gemm_peaks(torch, dev, bus, seconds):
     """cuBLAS dense GEMM throughput on this GPU, 8192^3: bf16 (torch.matmul) and
     e4m3 (torch._scaled_mm, bf16 out).  Burst: the best of 5 bursts of 10
     back-to-back launches; sustained: back to back for `seconds` with clock and
-    power sampled.  These are the denominators of the roofline fractions."""
+    power sampled.  Both bursts run before either sustained loop, so that no
+    burst is timed on a GPU still held at its power cap by the loop before it.
+    These are the denominators of the roofline fractions."""
     N = 8192
     g = torch.Generator(device=dev)
     g.manual_seed(0)
@@ -435,9 +437,9 @@ def measure_gemm_peaks(torch, dev, bus, seconds):
     one = torch.ones((), device=dev)
     fl = 2.0 * N ** 3
     out = {}
-    for name, fn in (("bf16", lambda: torch.matmul(a, b)),
-                     ("fp8_e4m3", lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one,
-                                                            out_dtype=torch.bfloat16))):
+    gemms = (("bf16", lambda: torch.matmul(a, b)),
+             ("fp8_e4m3", lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)))
+    for name, fn in gemms:
         for _ in range(5):
             fn()
         torch.cuda.synchronize()
@@ -450,7 +452,10 @@ def measure_gemm_peaks(torch, dev, bus, seconds):
             e1.record()
             torch.cuda.synchronize()
             best = min(best, e0.elapsed_time(e1) / 10)
-        entry = {"burst_tflops": fl / (best * 1e-3) / 1e12}
+        out[name] = {"burst_tflops": fl / (best * 1e-3) / 1e12, "burst_ms": best}
+    for name, fn in gemms:
+        entry = out[name]
+        best = entry.pop("burst_ms")
         if seconds > 0:
             n = max(10, int(seconds / (best * 1e-3)))
             smp = make_sampler(bus)

@@ -111,7 +111,10 @@ struct AttnCfg {
   static constexpr int STK = FP8 ? 4 : (DQK == 128 ? 3 : 2);
   static constexpr int STV = FP8 ? 4 : 2;
   static constexpr int QBUF = FP8 ? 2 : 1;           // Q tile buffers (units in flight)
-  static constexpr int KLEAD = STK - STV + 1;         // K tiles the producer keeps ahead of V
+  // K tiles the producer keeps ahead of V.  BF16: the whole K ring, so that
+  // loading K(g + STK) waits only for S(g) to finish and never queues behind
+  // V(g + 1), whose stage frees a whole softmax pass later (P V(g - 1)).
+  static constexpr int KLEAD = FP8 ? STK - STV + 1 : STK;
   static constexpr int NPB = FP8 ? 3 : 2;            // P buffers (tile g uses g % NPB)
   static constexpr int NK_QK = ROWB / 32;            // QK MMA K-steps of 32 bytes
   static constexpr int OFF_Q = 0;
@@ -757,7 +760,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 uint32_t w0, w1, w2, w3;
                 leanp_code_word2(__uint_as_float(rh[4 * w]), __uint_as_float(rh[4 * w + 1]), a256, b256, w0, w1);
                 leanp_code_word2(__uint_as_float(rh[4 * w + 2]), __uint_as_float(rh[4 * w + 3]), a256, b256, w2, w3);
-                p[w] = pack4_low_bytes(w0, w1, w2, w3);
+                p[w] = pack4_codes(w0, w1, w2, w3);
               }
             }
             tmem_st16p(tp + 16 * h, p);

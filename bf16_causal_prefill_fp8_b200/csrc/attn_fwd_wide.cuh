@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t w0, w1, w2, w3;
             leanp_code_word2(__uint_as_float(rh[4 * w]), __uint_as_float(rh[4 * w + 1]), a256, b256, w0, w1);
             leanp_code_word2(__uint_as_float(rh[4 * w + 2]), __uint_as_float(rh[4 * w + 3]), a256, b256, w2, w3);
-            p[16 * h + w] = pack4_low_bytes(w0, w1, w2, w3);
+            p[16 * h + w] = pack4_codes(w0, w1, w2, w3);
           }
         }
         // E8M0 scale code 127 - j for both 32-key MX blocks of this 64-key block

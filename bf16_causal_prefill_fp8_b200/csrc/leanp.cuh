@@ -53,10 +53,13 @@ __device__ __forceinline__ float leanp_row_offset(float m, float A, int j) {
 //   x = sat(fma(s, A/256, B/256))       (= fp32(u)/256 clamped to [0, 1]; the
 //                                         division by 256 is exact and commutes
 //                                         with the rounding for normal values)
-//   w = fma_rz(x, 256, 1.5 * 2^23)       (= 1.5 * 2^23 + trunc(fp32(u)) exactly)
-// so the low byte of w's bits is trunc(max(u, 0)) for 0 <= u < 256: two
-// FMA-pipe instructions per score, no integer conversion.  a256 = A/256 and
-// b256 = B/256 are computed once per (row, block).
+//   w = fma_rz(x, 2^-141, 0)             (= trunc(256 x) * 2^-149 exactly)
+// x * 2^-141 = (256 x) * 2^-149 lies below 2^-126, so the round-toward-zero FMA
+// lands on the subnormal grid, whose spacing is 2^-149: w is the subnormal
+// with fraction field trunc(256 x), and its bit pattern read as an integer is
+// trunc(max(u, 0)) for 0 <= u < 256.  Two FMA-pipe instructions per score, no
+// integer conversion; a256 = A/256 and b256 = B/256 are computed once per
+// (row, block).
 __device__ __forceinline__ float leanp_scaled_u(float s, float a256, float b256) {
   float x;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(x) : "f"(s), "f"(a256), "f"(b256));
@@ -65,38 +68,40 @@ __device__ __forceinline__ float leanp_scaled_u(float s, float a256, float b256)
 
 __device__ __forceinline__ uint32_t leanp_word(float x) {
   float w;
-  asm("fma.rz.f32 %0, %1, 0f43800000, 0f4B400000;" : "=f"(w) : "f"(x));   // x * 256 + 1.5 * 2^23
+  asm("fma.rz.f32 %0, %1, 0f00000100, 0f00000000;" : "=f"(w) : "f"(x));   // x * 2^-141 + 0
   return __float_as_uint(w);
 }
 
-// One score -> a word whose low byte is its code (a256 = A/256, b256 = B/256).
+// One score -> its code as an integer (a256 = A/256, b256 = B/256).
 __device__ __forceinline__ uint32_t leanp_code_word(float s, float a256, float b256) {
   return leanp_word(leanp_scaled_u(s, a256, b256));
 }
 
 // leanp_word for two values at once: one packed round-toward-zero FMA
-// (fma.rz.f32x2 applies the same IEEE operation to each half, so each word
-// equals leanp_word's).
+// (fma.rz.f32x2 applies the same IEEE operation to each half, subnormal
+// results included, so each word equals leanp_word's).
 __device__ __forceinline__ void leanp_word2(float x0, float x1, uint32_t& w0, uint32_t& w1) {
   uint64_t x, w;
   asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
-  asm("fma.rz.f32x2 %0, %1, %2, %3;" : "=l"(w) : "l"(x), "l"(0x4380000043800000ull), "l"(0x4B4000004B400000ull));
+  asm("fma.rz.f32x2 %0, %1, %2, %3;" : "=l"(w) : "l"(x), "l"(0x0000010000000100ull), "l"(0ull));
   asm("mov.b64 {%0, %1}, %2;" : "=r"(w0), "=r"(w1) : "l"(w));
 }
 
-// Two scores of one (row, block) -> two code words: the saturating FMA per
-// score, then leanp_word2.
+// Two scores of one (row, block) -> two codes: the saturating FMA per score,
+// then leanp_word2.
 __device__ __forceinline__ void leanp_code_word2(float s0, float s1, float a256, float b256, uint32_t& w0,
                                                  uint32_t& w1) {
   leanp_word2(leanp_scaled_u(s0, a256, b256), leanp_scaled_u(s1, a256, b256), w0, w1);
 }
 
-// Four code words -> one 32-bit word holding the four code bytes in order.
-__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t w0, uint32_t w1, uint32_t w2,
-                                                    uint32_t w3) {
-  const uint32_t lo = __byte_perm(w0, w1, 0x0040);
-  const uint32_t hi = __byte_perm(w2, w3, 0x0040);
-  return __byte_perm(lo, hi, 0x5410);
+// Four codes (integers below 256) -> one 32-bit word holding them as bytes in
+// order.  cvt.pack.sat.u8.s32.b32 d, a, b, c sets d = sat_u8(b) | sat_u8(a) << 8
+// | c << 16, so two of them pack four codes (three byte permutes did it before).
+__device__ __forceinline__ uint32_t pack4_codes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  uint32_t hi, d;
+  asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(hi) : "r"(w3), "r"(w2), "r"(0u));
+  asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(w1), "r"(w0), "r"(hi));
+  return d;
 }
 
 }  // namespace zyfa

@@ -262,19 +262,20 @@ long long prepass_rows(long long rows, int H, int D) {
 
 // ---------------------------------------------------------------- test kernels
 
-// Element pairs (i, i + 1) go through leanp_word2, the packed step the attention
-// kernel uses (an odd last element is paired with itself).
+// Groups of four elements (i .. i + 3) take the attention kernels' own steps:
+// leanp_word2 on two pairs, then pack4_codes; each code is read back from its
+// byte of the packed word (a ragged last group repeats its last element).
 __global__ void leanp_codes_kernel(const float* s, const float* m, const float* bmax, const float* A,
                                    const unsigned char* masked, int n, unsigned char* code, int* jout) {
-  const int npairs = (n + 1) / 2;
-  for (int pi = blockIdx.x * blockDim.x + threadIdx.x; pi < npairs; pi += gridDim.x * blockDim.x) {
-    const int i0 = 2 * pi, i1 = (2 * pi + 1 < n) ? 2 * pi + 1 : 2 * pi;
-    float a256[2], b256[2], sv[2];
-    int jj[2];
-    const int idx[2] = {i0, i1};
+  const long long nquads = (static_cast<long long>(n) + 3) / 4;
+  for (long long qi = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; qi < nquads;
+       qi += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float a256[4], b256[4], sv[4];
+    int jj[4], idx[4];
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int i = idx[e];
+    for (int e = 0; e < 4; ++e) {
+      const int i = static_cast<int>(4 * qi + e < n ? 4 * qi + e : n - 1);
+      idx[e] = i;
       const float Ai = A[i], mi = m[i];
       jj[e] = leanp_block_shift(mi, bmax[i], Ai);
       const float B = leanp_row_offset(mi, Ai, jj[e]);
@@ -282,11 +283,16 @@ __global__ void leanp_codes_kernel(const float* s, const float* m, const float* 
       a256[e] = __fmul_rn(Ai, 0.00390625f);
       b256[e] = __fmul_rn(B, 0.00390625f);
     }
-    uint32_t w0, w1;
-    leanp_word2(leanp_scaled_u(sv[0], a256[0], b256[0]), leanp_scaled_u(sv[1], a256[1], b256[1]), w0, w1);
-    code[i0] = static_cast<unsigned char>(w0 & 0xffu);
-    code[i1] = static_cast<unsigned char>(w1 & 0xffu);
-    if (jout) { jout[i0] = jj[0]; jout[i1] = jj[1]; }
+    uint32_t w[4];
+    leanp_word2(leanp_scaled_u(sv[0], a256[0], b256[0]), leanp_scaled_u(sv[1], a256[1], b256[1]), w[0], w[1]);
+    leanp_word2(leanp_scaled_u(sv[2], a256[2], b256[2]), leanp_scaled_u(sv[3], a256[3], b256[3]), w[2], w[3]);
+    const uint32_t packed = pack4_codes(w[0], w[1], w[2], w[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (4 * qi + e >= n) break;
+      code[idx[e]] = static_cast<unsigned char>((packed >> (8 * e)) & 0xffu);
+      if (jout) jout[idx[e]] = jj[e];
+    }
   }
 }
 
@@ -727,7 +733,8 @@ extern "C" int zyfa_leanp_codes(const float* s, const float* m, const float* bma
   if (n < 0) return ZYFA_ERR_BAD_SHAPE;
   if (n == 0) return ZYFA_OK;
   if (!s || !m || !bmax || !A || !code) return ZYFA_ERR_NULL_PTR;
-  const int blocks = (n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024;
+  const long long quads = (static_cast<long long>(n) + 3) / 4;
+  const int blocks = static_cast<int>(std::min(1024ll, (quads + 255) / 256));
   leanp_codes_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(s, m, bmax, A, masked, n, code, j);
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }

@@ -304,9 +304,11 @@ int zyfa_device_check(void* stream);
 int zyfa_checked_build(void);
 
 /*
- * zyfa_leanp_codes -- runs, element-wise, the very __device__ functions the
- * FP8 attention kernel uses to turn scores into Lean-P codes, so that the
- * codes can be compared byte for byte with a CPU emulation.  For element i:
+ * zyfa_leanp_codes -- runs the very __device__ functions the FP8 attention
+ * kernels use to turn scores into Lean-P codes, so that the codes can be
+ * compared byte for byte with a CPU emulation: the per-element steps below,
+ * then the same packing of four codes into one 32-bit word (elements
+ * 4k .. 4k+3 share a word).  For element i:
  *   j[i]    = 8 if bmax[i] == -inf, else
  *             min(126, 8 + floor(fp32(fp32(m[i] - bmax[i]) * A[i]) * 0.125))
  *   B       = fma(-m[i], A[i], 56 + 8 j[i])

@@ -38,16 +38,17 @@ class Config:
     npb: int      # P buffers
     fp8: bool     # FP8 or BF16 (the same protocol)
     hand: int = 8  # unit hand-over slots (and their barriers)
+    lead: int = 0  # K tiles the producer keeps ahead of V (0: stk - stv + 1)
 
     @property
     def klead(self):
-        return self.stk - self.stv + 1
+        return self.lead or self.stk - self.stv + 1
 
 
 # the kernel's three instantiations
 FP8 = Config(stk=4, stv=4, qbuf=2, npb=3, fp8=True)
-BF16_D128 = Config(stk=3, stv=2, qbuf=1, npb=2, fp8=False)
-BF16_D192 = Config(stk=2, stv=2, qbuf=1, npb=2, fp8=False)
+BF16_D128 = Config(stk=3, stv=2, qbuf=1, npb=2, fp8=False, lead=3)
+BF16_D192 = Config(stk=2, stv=2, qbuf=1, npb=2, fp8=False, lead=2)
 
 
 class ProtocolError(AssertionError):
