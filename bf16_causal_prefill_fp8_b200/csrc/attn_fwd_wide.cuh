@@ -323,6 +323,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     t.init(gridDim.x, blockIdx.x, a, vs);
     float A = a.C;
     float m_own = __int_as_float(0xff800000);   // the reference max after the previous tile
+    // Two waits per tile are tested early with the non-blocking test_wait and
+    // voted on only where the barrier is needed, so the test's latency
+    // overlaps other work and a barrier found complete costs no blocking
+    // wait: S of the next tile (tested before this tile's P store) and the P
+    // buffer (tested before the codes).  A test that finds the phase pending
+    // falls back to the bounded wait.  Neither can alias: the phase after the
+    // tested one needs work this group has not done yet.
+    bool sf_t = false;
     while (ok && t.next()) {
       const uint32_t g = t.g;
       if (t.j == 0) {
@@ -333,7 +341,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float ks = (a.k_scale && sok) ? a.k_scale[t.b * a.Hkv + t.hkv] : 1.0f;
         A = leanp_slope(qs, ks, a.C);
       }
-      if (!(ok = warp_wait(bar(W::SF), g & 1, ctl))) break;
+      if (!__all_sync(0xffffffffu, sf_t) && !(ok = warp_wait(bar(W::SF), g & 1, ctl))) break;
       tc_fence_after();
       uint32_t r[128];
       tmem_ld64p(tsg, &r[0]);
@@ -370,6 +378,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       } else {
         m = m_own;
       }
+      const bool pe_t = g < 1 || mbar_test_wait(bar(W::PE), (g - 1) & 1);
       // the codes of this group's 128 keys, before waiting for the P buffer
       uint32_t p[32];
       uint32_t sfw = 0;
@@ -404,7 +413,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         sfw |= static_cast<uint32_t>((127 - jb) * 0x0101) << (16 * h);
       }
       // P V of tile g-1 has read the P buffer and its scale factors, and O holds it
-      if (g >= 1 && !(ok = warp_wait(bar(W::PE), (g - 1) & 1, ctl))) break;
+      if (!__all_sync(0xffffffffu, pe_t) && !(ok = warp_wait(bar(W::PE), (g - 1) & 1, ctl))) break;
       tc_fence_after();
       if (__any_sync(0xffffffffu, alpha != 1.0f)) {
         // the reference moved: O and l still hold tiles 0 .. g-1 against the
@@ -424,6 +433,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st1(lb + W::TL, __float_as_uint(__uint_as_float(lv) * alpha));
         }
       }
+      sf_t = mbar_test_wait(bar(W::SF), (g + 1) & 1);
       tmem_st16p(tpg, &p[0]);
       tmem_st16p(tpg + 16, &p[16]);
       // the row's E8M0 word of this half: column (row / 32) of its own lane

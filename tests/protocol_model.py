@@ -346,6 +346,16 @@ def run_wide(units, cfg: WideConfig, seed: int, mutation=None, p_rescale=0.5):
                 raise ProtocolError(f"stuck on {name}: phase {need} complete but parity {parity} fails")
             yield "wait"
 
+    def test(name, parity, need):
+        """Non-blocking test of a phase (test_wait): True when it passes."""
+        b = bars[name]
+        if (b.c & 1) != parity:
+            if b.c <= need:
+                raise ProtocolError(f"aliasing on {name}: early test of parity {parity} passed at phase count "
+                                    f"{b.c}, needs more than {need}")
+            return True
+        return False
+
     def producer():
         def load_k(g):
             u, j, nkv = tiles[g]
@@ -408,8 +418,10 @@ def run_wide(units, cfg: WideConfig, seed: int, mutation=None, p_rescale=0.5):
             yield "step"
 
     def softmax_group(x):
+        sf_t = False        # S of the next tile seen complete by the early test
         for g, (u, j, nkv) in enumerate(tiles):
-            yield from wait("SF", g & 1, g)
+            if not sf_t:
+                yield from wait("SF", g & 1, g)
             if g not in st["qk_done"]:
                 raise ProtocolError(f"S of tile {g} read before its MMA finished")
             yield "load"
@@ -428,14 +440,18 @@ def run_wide(units, cfg: WideConfig, seed: int, mutation=None, p_rescale=0.5):
                 raise ProtocolError(f"group {x} read the other group's tile max of tile "
                                     f"{st['xch'].get((slot, 1 - x))} at tile {g}")
             st["xch_read"][(slot, 1 - x)] = g
+            # the P buffer, tested before the codes and waited for after them
+            pe_t = g < 1 or test("PE", (g - 1) & 1, g - 1)
             for _ in range(rng.randint(0, 4)):
                 yield "codes"
-            if g >= 1 and mutation != "no_pe_wait":
+            if g >= 1 and not pe_t and mutation != "no_pe_wait":
                 yield from wait("PE", (g - 1) & 1, g - 1)
             if g >= 1 and (g - 1) not in st["pv_done"]:
                 raise ProtocolError(f"P or O touched for tile {g} before P V of tile {g - 1} finished")
             if rescale[g]:
                 yield "rescale"
+            # S of the next tile, tested before this tile's P store
+            sf_t = test("SF", (g + (2 if mutation == "early_sf_two_ahead" else 1)) & 1, g + 1)
             st["P"][x] = g
             bars["PF"].arrive(128)
             if j == nkv - 1 and x == 0:

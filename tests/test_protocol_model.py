@@ -57,7 +57,7 @@ def test_wide_tile_protocol_holds_on_random_schedules():
         run_wide(random_units(rng), WIDE, seed, p_rescale=(0.0, 0.3, 0.9)[seed % 3])
 
 
-@pytest.mark.parametrize("mutation", ["no_sc_wait", "no_mx_wait", "no_pe_wait"])
+@pytest.mark.parametrize("mutation", ["no_sc_wait", "no_mx_wait", "no_pe_wait", "early_sf_two_ahead"])
 def test_wide_model_catches_planted_mistakes(mutation):
     with pytest.raises(ProtocolError):
         for seed in range(200):
