@@ -27,6 +27,19 @@
 
 namespace zyfa {
 
+// Programmatic dependent launch.  The prepass kernels after the first one
+// are launched with programmatic stream serialization, so each may start
+// while the kernel before it is still running.  griddep_wait blocks until
+// that kernel has completed and its writes are visible (a no-op for a launch
+// without the attribute); griddep_launch_dependents lets the next kernel
+// start launching, whose CTAs then wait in griddep_wait before they touch
+// this kernel's results.  The inputs x were written before the first prepass
+// kernel, which launches in plain stream order, so reading them needs no wait.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 constexpr int kQuantThreads = 256;
 constexpr int kUnroll = 4;        // rotated paths: rows in flight per warp
 constexpr int kUnrollPlain = 4;   // plain paths: 16-byte loads in flight per thread
@@ -197,6 +210,7 @@ __device__ __forceinline__ uint32_t row_head(const QuantArgs& a, uint32_t v) {
 // Step 2 for sequence-row chunk `chunk` of batch b (one CTA); s_amax: [H].
 template <typename T, bool HAD>
 __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, int b, unsigned int* s_amax) {
+  griddep_launch_dependents();
   const int r0 = chunk * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
   for (int h = threadIdx.x; h < a.H; h += blockDim.x) s_amax[h] = 0u;
   __syncthreads();
@@ -279,6 +293,7 @@ __device__ __forceinline__ void quant_amax_cta(const QuantArgs& a, int chunk, in
     }
   }
   __syncthreads();
+  griddep_wait();   // the scale array holds zeros (the zero step has completed)
   for (int h = threadIdx.x; h < a.H; h += blockDim.x)
     atomicMax(reinterpret_cast<unsigned int*>(a.scale) + static_cast<size_t>(b) * a.H + h, s_amax[h]);
 }
@@ -387,6 +402,8 @@ __device__ __forceinline__ void quant_codes_loop(const QuantArgs& a, int r0, int
 
 template <typename T, bool HAD>
 __device__ __forceinline__ void quant_codes_cta(const QuantArgs& a, int chunk, int b, float* s_sc) {
+  griddep_launch_dependents();
+  griddep_wait();   // every amax of the step is final
   const int r0 = chunk * a.rows_per_cta, r1 = min(a.S, r0 + a.rows_per_cta);
   float* s_rc = s_sc + a.H;   // RN(1 / scale) per head
   int fast = 1;
@@ -416,6 +433,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_codes_kernel(QuantArgs a)
 
 // Step 4.
 __global__ void quant_finalize_kernel(float* scale, int n) {
+  griddep_wait();   // every codes CTA has read the amax
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) scale[i] = head_scale(scale[i]);
 }
@@ -508,12 +526,14 @@ __global__ void __launch_bounds__(kQuantThreads) quant3v_codes_kernel(const __gr
 
 // Steps 1 and 4 for the three scale arrays (n[i] = B * H_i entries each).
 __global__ void quant3_zero_kernel(float* s0, float* s1, float* s2, int n0, int n1, int n2) {
+  griddep_launch_dependents();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n0) s0[i] = 0.0f;
   else if (i < n0 + n1) s1[i - n0] = 0.0f;
   else if (i < n0 + n1 + n2) s2[i - n0 - n1] = 0.0f;
 }
 __global__ void quant3_finalize_kernel(float* s0, float* s1, float* s2, int n0, int n1, int n2) {
+  griddep_wait();   // every codes CTA has read the amax
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   float* p = i < n0 ? s0 + i : (i < n0 + n1 ? s1 + (i - n0) : s2 + (i - n0 - n1));
   if (i < n0 + n1 + n2) *p = head_scale(*p);

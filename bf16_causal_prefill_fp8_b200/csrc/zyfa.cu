@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
+#include <utility>
 #include <numeric>
 #include <vector>
 
@@ -253,6 +254,25 @@ void set_div_magic(QuantArgs& t, int in_dtype) {
   t.mg_h = div_magic(static_cast<uint32_t>(t.H));
 }
 
+// Launch `kernel` with programmatic stream serialization: it may start while
+// the stream's previous kernel runs, and waits for that kernel's results in
+// griddep_wait (the prepass kernels after the first one).
+template <typename... P, typename... A>
+cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             A&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 // Sequence rows per prepass CTA: at most 2^30 elements of one batch entry
 // (the kernels count a chunk's rows and 16-byte vectors in 32 bits).
 long long prepass_rows(long long rows, int H, int D) {
@@ -424,25 +444,24 @@ extern "C" int zyfa_quantize(const void* x, int in_dtype, void* x_fp8, float* sc
   const size_t shm = static_cast<size_t>(H) * 8;   // amax, or scale and its reciprocal, per head
   if (cudaMemsetAsync(scale, 0, static_cast<size_t>(B) * H * sizeof(float), st) != cudaSuccess)
     return ZYFA_ERR_CUDA;
-  if (in_dtype == ZYFA_BF16) {
-    if (hadamard) {
-      quant_amax_kernel<__nv_bfloat16, true><<<grid, kQuantThreads, shm, st>>>(a);
-      quant_codes_kernel<__nv_bfloat16, true><<<grid, kQuantThreads, shm, st>>>(a);
-    } else {
-      quant_amax_kernel<__nv_bfloat16, false><<<grid, kQuantThreads, shm, st>>>(a);
-      quant_codes_kernel<__nv_bfloat16, false><<<grid, kQuantThreads, shm, st>>>(a);
-    }
-  } else {
-    if (hadamard) {
-      quant_amax_kernel<float, true><<<grid, kQuantThreads, shm, st>>>(a);
-      quant_codes_kernel<float, true><<<grid, kQuantThreads, shm, st>>>(a);
-    } else {
-      quant_amax_kernel<float, false><<<grid, kQuantThreads, shm, st>>>(a);
-      quant_codes_kernel<float, false><<<grid, kQuantThreads, shm, st>>>(a);
-    }
-  }
+  // the amax pass follows the memset in plain stream order; the codes and
+  // finalize passes are dependent launches
+  auto run = [&](auto amax_k, auto codes_k) -> cudaError_t {
+    amax_k<<<grid, kQuantThreads, shm, st>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    return e != cudaSuccess ? e : launch_dependent(codes_k, grid, dim3(kQuantThreads), shm, st, a);
+  };
+  cudaError_t e;
+  if (in_dtype == ZYFA_BF16)
+    e = hadamard ? run(quant_amax_kernel<__nv_bfloat16, true>, quant_codes_kernel<__nv_bfloat16, true>)
+                 : run(quant_amax_kernel<__nv_bfloat16, false>, quant_codes_kernel<__nv_bfloat16, false>);
+  else
+    e = hadamard ? run(quant_amax_kernel<float, true>, quant_codes_kernel<float, true>)
+                 : run(quant_amax_kernel<float, false>, quant_codes_kernel<float, false>);
+  if (e != cudaSuccess) return ZYFA_ERR_CUDA;
   const int n = B * H;
-  quant_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(scale, n);
+  if (launch_dependent(quant_finalize_kernel, dim3((n + 255) / 256), dim3(256), 0, st, scale, n) != cudaSuccess)
+    return ZYFA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
@@ -496,15 +515,22 @@ extern "C" int zyfa_quantize_qkv(const void* q, const void* k, const void* v, in
   const dim3 grid(static_cast<unsigned>(a.first[3]), static_cast<unsigned>(B));
   const size_t shm = static_cast<size_t>(max_h) * 8;   // amax, or scale and its reciprocal, per head
   const int n0 = B * Hq, n1 = B * Hkv, n2 = B * Hkv, n = n0 + n1 + n2;
+  // the zero step in plain stream order, the other three as dependent launches
   quant3_zero_kernel<<<(n + 255) / 256, 256, 0, st>>>(q_scale, k_scale, v_scale, n0, n1, n2);
+  if (cudaGetLastError() != cudaSuccess) return ZYFA_ERR_CUDA;
+  const dim3 blk(kQuantThreads);
+  cudaError_t e;
   if (in_dtype == ZYFA_BF16) {
-    quant3_amax_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
-    quant3_codes_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
+    e = launch_dependent(quant3_amax_kernel<__nv_bfloat16>, grid, blk, shm, st, a);
+    if (e == cudaSuccess) e = launch_dependent(quant3_codes_kernel<__nv_bfloat16>, grid, blk, shm, st, a);
   } else {
-    quant3_amax_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
-    quant3_codes_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
+    e = launch_dependent(quant3_amax_kernel<float>, grid, blk, shm, st, a);
+    if (e == cudaSuccess) e = launch_dependent(quant3_codes_kernel<float>, grid, blk, shm, st, a);
   }
-  quant3_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(q_scale, k_scale, v_scale, n0, n1, n2);
+  if (e == cudaSuccess)
+    e = launch_dependent(quant3_finalize_kernel, dim3((n + 255) / 256), dim3(256), 0, st, q_scale, k_scale,
+                         v_scale, n0, n1, n2);
+  if (e != cudaSuccess) return ZYFA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
@@ -612,19 +638,25 @@ static int quantize_varlen_n(int n, const void* const* xs, void* const* outs, fl
   const int nn = n0 + n1 + n2;
   float* s1 = n > 1 ? scs[1] : scs[0];
   float* s2 = n > 2 ? scs[2] : scs[0];
+  // the zero step in plain stream order, the others as dependent launches
   quant3_zero_kernel<<<(nn + 255) / 256, 256, 0, st>>>(scs[0], s1, s2, n0, n1, n2);
+  if (cudaGetLastError() != cudaSuccess) return ZYFA_ERR_CUDA;
+  cudaError_t e = cudaSuccess;
   if (q3.first[3] > 0) {   // some sequence has rows
-    const dim3 grid(static_cast<unsigned>(q3.first[3]), 1u);
+    const dim3 grid(static_cast<unsigned>(q3.first[3]), 1u), blk(kQuantThreads);
     const size_t shm = static_cast<size_t>(max_h) * 8;   // amax, or scale and its reciprocal, per head
     if (in_dtype == ZYFA_BF16) {
-      quant3v_amax_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
-      quant3v_codes_kernel<__nv_bfloat16><<<grid, kQuantThreads, shm, st>>>(a);
+      e = launch_dependent(quant3v_amax_kernel<__nv_bfloat16>, grid, blk, shm, st, a);
+      if (e == cudaSuccess) e = launch_dependent(quant3v_codes_kernel<__nv_bfloat16>, grid, blk, shm, st, a);
     } else {
-      quant3v_amax_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
-      quant3v_codes_kernel<float><<<grid, kQuantThreads, shm, st>>>(a);
+      e = launch_dependent(quant3v_amax_kernel<float>, grid, blk, shm, st, a);
+      if (e == cudaSuccess) e = launch_dependent(quant3v_codes_kernel<float>, grid, blk, shm, st, a);
     }
   }
-  quant3_finalize_kernel<<<(nn + 255) / 256, 256, 0, st>>>(scs[0], s1, s2, n0, n1, n2);
+  if (e == cudaSuccess)
+    e = launch_dependent(quant3_finalize_kernel, dim3((nn + 255) / 256), dim3(256), 0, st, scs[0], s1, s2, n0, n1,
+                         n2);
+  if (e != cudaSuccess) return ZYFA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ZYFA_OK : ZYFA_ERR_CUDA;
 }
 
