@@ -33,9 +33,14 @@
 // own MMAs; the hand-offs between them go through the barriers).
 // Work unit = (batch, query head, 128-row query tile); KV tiles 0..qt only
 // (fully masked tiles are never issued), ascending, so results are
-// deterministic.  S has two TMEM buffers: the MMA of S for tile j+2 runs
-// as soon as the softmax has read S of tile j; P V of tile j runs while the
-// softmax works on tile j+1.
+// deterministic.  FP8 and BF16 with Dqk 192: S has two TMEM buffers, and the
+// MMA of S for tile j+2 runs as soon as the softmax has read S of tile j.
+// BF16 with Dqk 128: Q sits in TMEM (copied from shared memory once per unit
+// with tcgen05.cp) and S is a TS MMA, A from TMEM and only K from shared
+// memory; with both operands in shared memory the N = 128 MMA is bound by
+// shared-memory bandwidth.  Q takes the second S buffer's columns, so S of
+// tile j+1 runs as soon as the softmax has read S of tile j.  P V of tile j
+// runs while the softmax works on tile j+1.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -116,6 +121,8 @@ struct AttnCfg {
   // V(g + 1), whose stage frees a whole softmax pass later (P V(g - 1)).
   static constexpr int KLEAD = FP8 ? STK - STV + 1 : STK;
   static constexpr int NPB = FP8 ? 3 : 2;            // P buffers (tile g uses g % NPB)
+  // BF16 Dqk 128: Q in TMEM (A of the S MMAs), one S buffer
+  static constexpr bool QTM = !FP8 && DQK == 128;
   static constexpr int NK_QK = ROWB / 32;            // QK MMA K-steps of 32 bytes
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBUF * QB;
@@ -141,12 +148,17 @@ struct AttnCfg {
   static constexpr int NBAR = VE + STV;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
-  // tensor-memory columns (512 allocated)
-  static constexpr uint32_t TS0 = 0, TS1 = 128, TO = 256;
+  // tensor-memory columns (512 allocated).  S buffers 0..127 and 128..255 (one
+  // S buffer at 0 with Q in TMEM), O 256..383 (128..255 with Q in TMEM), Q
+  // 384..447 (bf16 pairs, the A layout of the S MMA)
+  static constexpr uint32_t TS0 = 0, TS1 = QTM ? 0 : 128, TO = QTM ? 128 : 256, TQ = 384;
   static constexpr uint32_t TL = 384, TSFB = 400;
   // P buffer b: FP8 32 columns of packed codes at 416 + 32 b; BF16 64 columns
-  // of bf16 pairs at 384 + 64 b; FP8 scale factors of P buffer b at 404 + 4 b
-  static __device__ __forceinline__ uint32_t tp(uint32_t b) { return FP8 ? 416 + 32 * b : 384 + 64 * b; }
+  // of bf16 pairs at 384 + 64 b (256 + 64 b with Q in TMEM); FP8 scale
+  // factors of P buffer b at 404 + 4 b
+  static __device__ __forceinline__ uint32_t tp(uint32_t b) {
+    return FP8 ? 416 + 32 * b : (QTM ? 256 : 384) + 64 * b;
+  }
   static __device__ __forceinline__ uint32_t tsfa(uint32_t b) { return 404 + 4 * b; }
   static constexpr uint32_t IDESC_QK = idesc_dense(FP8 ? 0 : 1, FP8 ? 0 : 1, 0, 0, 128, 128);
   static constexpr uint32_t IDESC_PV_BF16 = idesc_dense(1, 1, 0, 1, 128, 128);
@@ -554,8 +566,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
    } else if (warp == 13 || warp == 14) {
     // ------------------------------------------------------------ MMA issuers
     // warp 13: S for tile g is issued as soon as its K tile is loaded and the
-    // softmax has read S of tile g-2 (two S buffers).  warp 14: P V of tile g
-    // once the softmax has written P (and rescaled O, when it had to).
+    // softmax has read S of tile g-2 (two S buffers; g-1 with Q in TMEM).
+    // warp 14: P V of tile g once the softmax has written P (and rescaled O,
+    // when it had to).
     TS ts;
     ts.init(gridDim.x, blockIdx.x, a, vs);
     bool ok = true;
@@ -570,14 +583,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     auto issue_qk = [&](const TS& t) -> bool {
       const uint32_t slot = t.u % Cf::QBUF;
       if (t.j == 0 && !wait1(bar(Cf::QF0 + slot), (t.u / Cf::QBUF) & 1)) return false;
-      const uint32_t st = t.g % Cf::STK, buf = t.g & 1;
+      const uint32_t st = t.g % Cf::STK, buf = Cf::QTM ? 0 : (t.g & 1);
       if (!wait1(bar(Cf::KF + st), (t.g / Cf::STK) & 1)) return false;
-      if (t.g >= 2 && !wait1(bar(Cf::SC0 + buf), ((t.g >> 1) - 1) & 1)) return false;
+      if (Cf::QTM) {
+        // one S buffer: the softmax has read S of the previous tile (so the
+        // S MMAs of the previous unit, which read Q from TMEM, are done)
+        if (t.g >= 1 && !wait1(bar(Cf::SC0), (t.g - 1) & 1)) return false;
+      } else if (t.g >= 2 && !wait1(bar(Cf::SC0 + buf), ((t.g >> 1) - 1) & 1)) {
+        return false;
+      }
       tc_fence_after();
       const uint64_t dqs = dq + ((slot * Cf::QB) >> 4), dqs_t = dq_t + ((slot * Cf::QB) >> 4);
       const uint64_t dks = dk + ((st * Cf::KB) >> 4), dks_t = dk_t + ((st * Cf::KB) >> 4);
       const uint32_t ts = tbase + (buf ? Cf::TS1 : Cf::TS0);
-      if (leader) {
+      if (Cf::QTM && leader) {
+        if (t.j == 0) {
+          // the unit's Q tile into TMEM, one 128 x 32-byte K slice per copy,
+          // in the lane / column layout of an A operand; the copies run
+          // before the MMAs issued after them
+#pragma unroll
+          for (int kk = 0; kk < Cf::NK_QK; ++kk)
+            tmem_cp_128x256b(tbase + Cf::TQ + 8 * kk, dqs + (((kk >> 2) * Cf::CHUNK + (kk & 3) * 32) >> 4));
+          tc_commit(bar(Cf::QE0 + slot));   // the Q slot in shared memory is free
+        }
+#pragma unroll
+        for (int kk = 0; kk < Cf::NK_QK; ++kk)
+          mma_f16_ts(ts, tbase + Cf::TQ + 8 * kk, dks + (((kk >> 2) * Cf::CHUNK + (kk & 3) * 32) >> 4),
+                     Cf::IDESC_QK, kk > 0 ? 1u : 0u);
+        tc_commit(bar(Cf::SF0));
+        tc_commit(bar(Cf::KE + st));
+      } else if (leader) {
 #pragma unroll
         for (int kk = 0; kk < Cf::NK_QK; ++kk) {
           uint64_t ad, bd;
@@ -653,8 +688,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     reg_alloc<kRegSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
     // Two groups alternate over the KV tiles: group x = warp / 4 takes the
-    // tiles with (g & 1) == x, i.e. always S buffer x, so one group computes
-    // while the other waits for its next S.  Thread t of a group owns row
+    // tiles with (g & 1) == x, i.e. always S buffer x (with Q in TMEM the one
+    // S buffer, taken in turns), so one group computes while the other waits
+    // for its next S.  Thread t of a group owns row
     // 32 (w % 4) + lane (TMEM lane quarter w % 4) and all 128 keys of its
     // tiles.  The running max crosses between the groups once per tile (smem
     // + per-buffer barrier MX), the only serial dependency.
@@ -690,7 +726,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       if ((g & 1) == static_cast<uint32_t>(grp)) {
         const bool diag = t.j == t.qt;
-        if (!(ok = warp_wait(bar(Cf::SF0 + grp), (g >> 1) & 1, ctl))) break;
+        // one S buffer: the other group's max of tile g-1, published after
+        // it read S of tile g-1, keeps the wait on S at most one phase behind
+        if (Cf::QTM && g >= 1 &&
+            !(ok = warp_wait(bar(Cf::MX0 + ((g - 1) & 1)), ((g - 1) >> 1) & 1, ctl))) break;
+        if (!(ok = warp_wait(bar(Cf::SF0 + (Cf::QTM ? 0 : grp)), Cf::QTM ? (g & 1) : ((g >> 1) & 1), ctl))) break;
         tc_fence_after();
         // the whole 128-key row of S in one TMEM round trip; the S buffer is
         // free for the tile after next right away
@@ -699,7 +739,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld64p(ts + 64, &r[64]);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(bar(Cf::SC0 + grp));
+        mbar_arrive(bar(Cf::SC0 + (Cf::QTM ? 0 : grp)));
         if (diag) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -711,7 +751,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float m_prev = __int_as_float(0xff800000);
         if (g >= 1) {
           const uint32_t pb = (g - 1) & 1;
-          if (!(ok = warp_wait(bar(Cf::MX0 + pb), ((g - 1) >> 1) & 1, ctl))) break;
+          if (!Cf::QTM && !(ok = warp_wait(bar(Cf::MX0 + pb), ((g - 1) >> 1) & 1, ctl))) break;
           if (t.j > 0) m_prev = xch_s[pb * 128 + row];
         }
         // reference max after this tile (FP8: A carries a factor 8)

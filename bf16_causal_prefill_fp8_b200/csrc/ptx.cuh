@@ -278,6 +278,9 @@ __device__ __forceinline__ void mma_mxf8_ts(uint32_t d, uint32_t a_tmem, uint64_
 
 // Copy a 32-row x 128-bit matrix from shared memory (matrix descriptor) into
 // TMEM columns taddr .. taddr+3, replicated into all four 32-lane quarters.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }

@@ -39,6 +39,7 @@ class Config:
     fp8: bool     # FP8 or BF16 (the same protocol)
     hand: int = 8  # unit hand-over slots (and their barriers)
     lead: int = 0  # K tiles the producer keeps ahead of V (0: stk - stv + 1)
+    one_s: bool = False  # one S buffer, Q copied into TMEM at each unit's first tile
 
     @property
     def klead(self):
@@ -47,7 +48,7 @@ class Config:
 
 # the kernel's three instantiations
 FP8 = Config(stk=4, stv=4, qbuf=2, npb=3, fp8=True)
-BF16_D128 = Config(stk=3, stv=2, qbuf=1, npb=2, fp8=False, lead=3)
+BF16_D128 = Config(stk=3, stv=2, qbuf=1, npb=2, fp8=False, lead=3, one_s=True)
 BF16_D192 = Config(stk=2, stv=2, qbuf=1, npb=2, fp8=False, lead=2)
 
 
@@ -93,7 +94,8 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_produce
     tiles = [(u, j, nkv) for u, nkv in enumerate(units) for j in range(nkv)]
     fifos = {"qk": [], "pv": []}
     tma = []
-    st = {"P": {}, "O_unit": None, "pv_done": set(), "qk_done": set(), "Sread": {}, "xch": {}, "hand": {}}
+    st = {"P": {}, "O_unit": None, "pv_done": set(), "qk_done": set(), "Sread": {}, "xch": {}, "hand": {},
+          "Qsmem": {}, "Qtmem": None}
 
     def wait(name, parity, need):
         b = bars[name]
@@ -115,7 +117,7 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_produce
             slot, n = u % cfg.qbuf, u // cfg.qbuf
             if n > 0:
                 yield from wait(f"QE{slot}", (n - 1) & 1, n - 1)
-            tma.append([rng.randint(5, 40), f"QF{slot}"])
+            tma.append([rng.randint(5, 40), f"QF{slot}", ("Q", slot, u)])
         s_, n = g % cfg.stk, g // cfg.stk
         if n > 0:
             yield from wait(f"KE{s_}", (n - 1) & 1, n - 1)
@@ -153,14 +155,28 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_produce
             slot = u % cfg.qbuf
             if j == 0:
                 yield from wait(f"QF{slot}", (u // cfg.qbuf) & 1, u // cfg.qbuf)
-            s_, buf = g % cfg.stk, g & 1
+            s_, buf = g % cfg.stk, (0 if cfg.one_s else g & 1)
             yield from wait(f"KF{s_}", (g // cfg.stk) & 1, g // cfg.stk)
-            if g >= 2 and mutation != "no_sc_wait":
-                yield from wait(f"SC{buf}", ((g >> 1) - 1) & 1, (g >> 1) - 1)
-            if g >= 2 and st["Sread"].get(buf, -1) < g - 2:
-                raise ProtocolError(f"S buffer {buf} overwritten by tile {g} before tile {g - 2} read it")
-            fifos["qk"].append([rng.randint(5, 30), "qk", g])
-            fifos["qk"].append([0, "commit", [f"SF{buf}", f"KE{s_}"] + ([f"QE{slot}"] if j == nkv - 1 else [])])
+            back = 1 if cfg.one_s else 2        # tiles per S buffer
+            if g >= back and mutation != "no_sc_wait":
+                n = g // back - 1 if not cfg.one_s else g - 1
+                yield from wait(f"SC{buf}", n & 1, n)
+            if g >= back and st["Sread"].get(buf, -1) < g - back:
+                raise ProtocolError(f"S buffer {buf} overwritten by tile {g} before tile {g - back} read it")
+            if cfg.one_s:
+                if j == 0:
+                    # the unit's Q copied from its shared-memory slot into TMEM,
+                    # in order with the MMAs; the slot is free once it is done
+                    if mutation == "q_slot_freed_before_copy":
+                        fifos["qk"].append([0, "commit", [f"QE{slot}"]])
+                    fifos["qk"].append([rng.randint(3, 12), "cp", (u, slot)])
+                    if mutation != "q_slot_freed_before_copy":
+                        fifos["qk"].append([0, "commit", [f"QE{slot}"]])
+                fifos["qk"].append([rng.randint(5, 30), "qk", g])
+                fifos["qk"].append([0, "commit", [f"SF{buf}", f"KE{s_}"]])
+            else:
+                fifos["qk"].append([rng.randint(5, 30), "qk", g])
+                fifos["qk"].append([0, "commit", [f"SF{buf}", f"KE{s_}"] + ([f"QE{slot}"] if j == nkv - 1 else [])])
             yield "step"
 
     def pv_issuer():
@@ -183,8 +199,15 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_produce
     def softmax_group(grp):
         for g, (u, j, nkv) in enumerate(tiles):
             if (g & 1) == grp:
-                buf = grp
-                yield from wait(f"SF{buf}", (g >> 1) & 1, g >> 1)
+                if cfg.one_s and g >= 1 and mutation != "mx_after_sf":
+                    # one S buffer: the other group's max of tile g-1 (published
+                    # after it read S of tile g-1) keeps this wait on S at most
+                    # one phase behind
+                    pb = (g - 1) & 1
+                    yield from wait(f"MX{pb}", ((g - 1) >> 1) & 1, (g - 1) >> 1)
+                buf = 0 if cfg.one_s else grp
+                n = g if cfg.one_s else g >> 1
+                yield from wait(f"SF{buf}", n & 1, n)
                 if g not in st["qk_done"]:
                     raise ProtocolError(f"S of tile {g} read before its MMA finished")
                 yield "load"
@@ -193,7 +216,8 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_produce
                 yield "max"
                 if g >= 1:
                     pb = (g - 1) & 1
-                    yield from wait(f"MX{pb}", ((g - 1) >> 1) & 1, (g - 1) >> 1)
+                    if not cfg.one_s or mutation == "mx_after_sf":
+                        yield from wait(f"MX{pb}", ((g - 1) >> 1) & 1, (g - 1) >> 1)
                     if st["xch"].get(pb) != g - 1:
                         raise ProtocolError(f"reference max of tile {g - 1} overwritten before tile {g} read it")
                 st["xch"][grp] = g
@@ -268,12 +292,24 @@ def run(units, cfg: Config, seed: int, mutation=None, p_rescale=0.5, two_produce
             else:
                 e[0] -= 1
                 if e[0] <= 0:
-                    (st["qk_done"] if e[1] == "qk" else st["pv_done"]).add(e[2])
+                    if e[1] == "cp":
+                        u_, slot_ = e[2]
+                        if st["Qsmem"].get(slot_) != u_:
+                            raise ProtocolError(f"Q of unit {u_} copied to TMEM from slot {slot_} holding unit "
+                                                f"{st['Qsmem'].get(slot_)}")
+                        st["Qtmem"] = u_
+                    else:
+                        if e[1] == "qk" and cfg.one_s and st["Qtmem"] != tiles[e[2]][0]:
+                            raise ProtocolError(f"S of tile {e[2]} computed with the Q of unit {st['Qtmem']}")
+                        (st["qk_done"] if e[1] == "qk" else st["pv_done"]).add(e[2])
                     f.pop(0)
             progressed = True
         for t in list(tma):
             t[0] -= 1
             if t[0] <= 0:
+                if len(t) > 2:
+                    _, slot_, u_ = t[2]
+                    st["Qsmem"][slot_] = u_
                 bars[t[1]].arrive()
                 tma.remove(t)
             progressed = True

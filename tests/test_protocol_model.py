@@ -28,6 +28,18 @@ def test_model_catches_planted_mistakes(mutation, cfg):
             run(random_units(rng), cfg, seed, mutation=mutation)
 
 
+@pytest.mark.parametrize("mutation", ["q_slot_freed_before_copy", "mx_after_sf"])
+def test_model_catches_planted_mistakes_with_q_in_tmem(mutation):
+    """BF16 Dqk 128 (one S buffer, Q copied into TMEM per unit): releasing the
+    Q slot before the copy has read it, and waiting for S before the other
+    group's max of the previous tile (a wait two phases behind), must fail."""
+    assert BF16_D128.one_s
+    with pytest.raises(ProtocolError):
+        for seed in range(300):
+            rng = random.Random(seed)
+            run(random_units(rng), BF16_D128, seed, mutation=mutation)
+
+
 def test_model_catches_a_short_hand_over_ring():
     # the unit hand-over ring needs more slots than units a softmax group can
     # run ahead of the epilogue; with 2 the model finds the overwrite
