@@ -259,3 +259,89 @@ def test_e2e_pipeline_has_no_buffer_hazards():
             _FakeTensor.copy_ = orig_copy
         assert sorted(got) == list(range(steps))
         assert not any(s.q for s in cuda.streams)
+
+
+class _GemmTorch:
+    """Just enough of torch for bench.measure_gemm_peaks on the CPU: every
+    GEMM call and every sustained-loop start is logged in order."""
+
+    float8_e4m3fn = "e4m3"
+    bfloat16 = "bf16"
+
+    def __init__(self, log):
+        self.log = log
+        t = self
+
+        class _Tensor:
+            def to(self, dtype):
+                return self
+
+            def t(self):
+                return self
+
+        class _Event:
+            def __init__(self, enable_timing=False):
+                self.n = 0
+
+            def record(self, stream=None):
+                self.n = len(t.log)
+
+            def elapsed_time(self, other):
+                return 0.5 * max(1, other.n - self.n)
+
+        class _Cuda:
+            Event = _Event
+
+            @staticmethod
+            def synchronize():
+                pass
+
+            @staticmethod
+            def empty_cache():
+                pass
+
+        class _Generator:
+            def __init__(self, device=None):
+                pass
+
+            def manual_seed(self, s):
+                return self
+
+        self.cuda = _Cuda
+        self.Generator = _Generator
+        self._tensor = _Tensor
+
+    def randn(self, *shape, device=None, generator=None):
+        return self._tensor()
+
+    def ones(self, shape, device=None):
+        return self._tensor()
+
+    def matmul(self, a, b):
+        self.log.append("bf16")
+
+    def _scaled_mm(self, a, b, scale_a=None, scale_b=None, out_dtype=None):
+        self.log.append("fp8_e4m3")
+
+
+def test_gemm_bursts_run_before_the_sustained_loops(monkeypatch):
+    """Both burst measurements come before either sustained loop: a burst timed
+    right after a seconds-long loop runs on a GPU held at its power cap."""
+    log = []
+
+    class _Sampler:
+        def start(self):
+            log.append("sustained")
+
+        def stop(self):
+            return {"sm_mhz": 1300, "power_w_median": 990.0, "reasons": ["sw_power_cap"]}
+
+    monkeypatch.setattr(bench, "make_sampler", lambda bus: _Sampler())
+    out = bench.measure_gemm_peaks(_GemmTorch(log), "cuda:0", None, 0.001)
+    first_loop = log.index("sustained")
+    bursts = log[:first_loop]
+    assert "bf16" in bursts and "fp8_e4m3" in bursts
+    assert log.count("sustained") == 2
+    assert set(out) == {"bf16", "fp8_e4m3"}
+    for entry in out.values():
+        assert entry["burst_tflops"] > 0 and entry["sustained_tflops"] > 0 and "burst_ms" not in entry
