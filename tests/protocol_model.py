@@ -19,10 +19,19 @@ when the completed-phase count has the other parity.  The model checks that
 `two_producers` splits the TMA producer into a K (and Q) warp and a V warp,
 each walking the tiles on its own (a variant that was once tried).
 
+`Config.one_s` (BF16 with Dqk 128) models one S buffer taken by the two
+groups in turns, with Q copied from its shared-memory slot into tensor
+memory at each unit's first tile: the copy is a queue entry in order with
+the S MMAs, must find its own unit's Q in the slot, and every S MMA must
+find its unit's Q in tensor memory.  Each group waits for the other group's
+max of the previous tile before its wait on S.
+
 `run_wide` models the FP8 kernel with 256-key tiles (csrc/attn_fwd_wide.cuh):
 one S buffer and one P buffer, both softmax groups on every tile (each on
 its own 128-key half), the tile max exchanged through a two-slot buffer under
 one barrier both groups arrive on, and the hand-over written by group 0.
+It also takes the kernel's two early, non-blocking tests (the next tile's
+S, the P buffer), each checked for aliasing when it passes.
 
 `mutation` plants a known mistake, for the tests that show the model catches it.
 """
